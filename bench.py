@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""MoE FFN layer forward on B200: tokens/s and grouped-GEMM TFLOP/s.
+
+One step = one pass of the whole layer path on one batch: router, dispatch,
+grouped SwiGLU experts (+ shared expert), combine, then the per-expert counts
+are summed over data-parallel ranks (NCCL all-reduce, N > 1 only) and the
+selection-bias update runs.  Each rank holds a full replica of the layer and
+its own T tokens (weak scaling); ``value`` is the tokens of all ranks per
+second, timed on the device (CUDA events, max over ranks).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_ffn_bias_b200 import inputs as I  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/sec and grouped-GEMM TFLOP/s (% bf16 peak) on 1 B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- #
+# workload arithmetic                                                          #
+# --------------------------------------------------------------------------- #
+def layer_flops(s: I.MoEShape) -> dict:
+    R = s.T * s.top_k
+    return {
+        "router": 2 * s.T * s.d_model * s.n_experts,
+        "gate_up": 4 * R * s.d_model * s.d_ff,
+        "down": 2 * R * s.d_ff * s.d_model,
+        "shared": 6 * s.T * s.d_model * s.d_ff_shared * s.n_shared,
+    }
+
+
+def describe(s: I.MoEShape) -> str:
+    gate = "softmax" if s.gate == I.GATE_SOFTMAX else "sigmoid"
+    dt = "bf16" if s.dtype == I.DTYPE_BF16 else "fp32"
+    sh = f" + {s.n_shared} shared (F={s.d_ff_shared})" if s.n_shared else ""
+    return (f"{s.name}: T={s.T} d_model={s.d_model} E={s.n_experts} routed (F={s.d_ff}){sh} "
+            f"top-{s.top_k} {gate}{'+renorm' if s.norm_topk_prob else ''} {dt}")
+
+
+def load_peaks() -> tuple:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("grouped_gemm_sm100.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_ffn_bias_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary,
+    or None when the summary is missing or was taken on other kernel source."""
+    p = os.path.join(ROOT, "profiles", f"grouped_gemm_gateup_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != gemm_source_hash():
+        return None
+    return float(m.group(1))
+
+
+# --------------------------------------------------------------------------- #
+# clocks during the timed region                                              #
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle (baseline and reference arm)                                      #
+# --------------------------------------------------------------------------- #
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+class OracleRunner:
+    """The oracle as it stands, on windows of the workload's tokens.  Weights
+    are handed to it already widened to float64 (same values), so a window's
+    cost is its own arithmetic."""
+
+    def __init__(self, shape: I.MoEShape, host: dict):
+        from oracle import moe_oracle as O
+        self.O = O
+        self.shape = shape
+        self.host = {k: (v.astype(np.float64) if k != "x" else v) for k, v in host.items()}
+        self.pos = 0
+
+    def run(self, n: int) -> float:
+        s = self.shape
+        lo = self.pos % s.T
+        hi = min(lo + n, s.T)
+        self.pos = hi
+        win = dict(self.host)
+        win["x"] = self.host["x"][lo:hi]
+        t0 = time.perf_counter()
+        r = self.O.router(win["x"], win["w_router"], s.top_k, s.gate, bool(s.norm_topk_prob),
+                          win.get("sel_bias"), win.get("logit_offset"))
+        self.O.dispatch(r.topk_idx, s.n_experts)
+        self.O.moe_forward(win, s.top_k, s.gate, bool(s.norm_topk_prob), routing=r)
+        return time.perf_counter() - t0, hi - lo
+
+    def calibrate(self, seconds: float) -> int:
+        """Tokens per window so that one window takes about `seconds`."""
+        n = 16
+        for _ in range(6):
+            t, m = self.run(n)
+            if t >= 0.5 * seconds or n >= self.shape.T:
+                break
+            n = min(self.shape.T, max(n + 1, int(n * min(8.0, seconds / max(t, 1e-3)))))
+        return max(1, min(self.shape.T, int(n * seconds / max(t, 1e-3))))
+
+
+def cpu_baseline(shape, host, seconds=15.0) -> dict:
+    runner = OracleRunner(shape, host)
+    n = runner.calibrate(seconds / 3)
+    t, m = runner.run(n)
+    tot_t, tot_m = t, m
+    while tot_t < seconds and m > 0:
+        t, m = runner.run(n)
+        tot_t += t
+        tot_m += m
+    return {"value": tot_m / tot_t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{tot_m} of the workload's tokens in windows of {n}: router, dispatch, "
+                      f"{shape.n_experts} experts{' + shared' if shape.n_shared else ''}, "
+                      f"combine, fp64 numpy ({tot_t:.1f} s)"}
+
+
+def run_reference(args, shape, rank: int, world: int):
+    if rank != 0:
+        return
+    host = I.make_inputs(shape)
+    runner = OracleRunner(shape, host)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = runner.calibrate(budget)
+    for _ in range(args.warmup):
+        runner.run(n)
+    ts, ms = 0.0, 0
+    for _ in range(args.steps):
+        t, m = runner.run(n)
+        ts += t
+        ms += m
+    value = ms / ts
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * ts / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(shape), "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} tokens per step (of {shape.T}), full layer in fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# GPU arm                                                                      #
+# --------------------------------------------------------------------------- #
+def run_ours(args, shape, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_ffn_bias_b200 import binding as B
+    from mixture_experts_ffn_bias_b200.layer import MoELayer
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    host = I.make_inputs(shape)
+    if rank > 0:
+        host["x"] = I.make_tokens(shape, seed=1000 * (shape.seed + 1) + rank)
+    layer = MoELayer(shape, host, dev)
+    if layer.sel_bias is None:
+        layer.sel_bias = torch.zeros(shape.n_experts, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    nph = B.FORWARD_PHASES
+
+    def step(evs=None, x=None):
+        if evs is None:
+            layer.forward(x=x)
+        else:
+            B.moe_forward_profiled(layer.cfg, layer.x if x is None else x, layer.w_router,
+                                   layer.sel_bias, layer.logit_offset, layer.weights, layer.out,
+                                   layer.topk_idx, layer.topk_w, layer.counts, layer.ws, evs)
+        if world > 1:
+            dist.all_reduce(layer.counts)
+        layer.bias_update()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    st, flags = layer.device_status()
+    if st != B.MOE_OK:
+        raise SystemExit(f"device status after warm-up: {B.status_string(st)} ({flags})")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank))
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier()
+    t_ms = start.elapsed_time(end)
+    phases = [statistics.mean(evs[i][p].elapsed_time(evs[i][p + 1]) for i in range(args.steps))
+              for p in range(nph)]
+    st, flags = layer.device_status()
+    if st != B.MOE_OK:
+        raise SystemExit(f"device status after timing: {B.status_string(st)} ({flags})")
+
+    # end-to-end: pinned host x in, result back, through the public layer call
+    e2e_steps = max(3, min(args.steps, 50))
+    x_host = layer.x.to("cpu").pin_memory()
+    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
+    x_dev = torch.empty_like(layer.x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x=x_dev)
+        out_host.copy_(layer.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    if world > 1:
+        t = torch.tensor([t_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank == 0:
+        ms = t_ms / args.steps
+        fl = layer_flops(shape)
+        peaks, peak_kind = load_peaks()
+        sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        t_gateup = phases[2] * 1e-3
+        t_gemm = (phases[2] + phases[3] + phases[4]) * 1e-3
+        achieved = fl["gate_up"] / t_gateup / 1e12
+        gemm_tflops = (fl["gate_up"] + fl["down"] + fl["shared"]) / t_gemm / 1e12
+        per_step_launches = 2 + 3 + 2 + 2 * shape.n_shared + 1 + 1
+        line = {
+            "metric": METRIC, "value": shape.T * world / (ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if shape.dtype == I.DTYPE_BF16 else "f32", "data": "synthetic",
+            "config": {"workload": describe(shape), "tokens_per_gpu": shape.T,
+                       "parallelism": f"dp{world} (replicated layer, counts all-reduce)",
+                       "l2": "not flushed: each step streams > 2 GB (weights + activations) "
+                             "through the 126 MB L2"},
+            "grouped_gemm": {"tflops": gemm_tflops, "frac_of_sustained": gemm_tflops / sus,
+                             "frac_of_burst": gemm_tflops / burst, "peaks": peak_kind},
+            "phases_ms": dict(zip(["router", "dispatch", "gate_up", "down", "shared", "combine"],
+                                  phases)),
+            "roofline": {"kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)", "bound": "tensor",
+                         "achieved": achieved, "peak": sus, "unit": "TFLOP/s",
+                         "frac": achieved / sus, "peak_kind": f"bf16_tflops_sustained ({peak_kind})",
+                         "traffic": profiled_traffic(shape.name)},
+            "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": layer.x.numel() * layer.x.element_size(),
+                    "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()},
+            "gpu_launches": per_step_launches * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(shape, host)
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=I.WORKLOAD_ORDER, default="qwen3_30b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    shape = I.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, shape, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, shape, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: the forward pass of a Mixture-of-Experts
+ * FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources by page title and section):
+ *   router    logits = x . Wr^T in fp32, scores = sigmoid(logits) or softmax
+ *             over all experts, selection keys = logits + sel_bias, top-k of
+ *             the keys, combine weights = the unbiased scores of the chosen
+ *             experts, optionally divided by (their sum + 1e-9).
+ *             ("moe-200m-qwen3-100b" README, "SigmoidRouter"; SpecForge PR
+ *             #930, "What this adds": qwen3 preset, softmax + norm_topk_prob.)
+ *   experts   E routed SwiGLU experts  y = W2 (silu(W1 x) * (W3 x)), weights
+ *             stacked [E, out, in] (SpecForge PR #930, "Why FSDP is enough
+ *             here"; per-expert keys w1/w2/w3 in SpecForge PR #931, "What
+ *             works"), plus optionally one always-on shared SwiGLU expert.
+ *   combine   out = shared(x) + sum_j w_j * expert_{idx_j}(x)
+ *             ("moe-200m-qwen3-100b" README, "Architecture diagram").
+ *   bias      aux-loss-free controller from per-expert counts
+ *             ("moe-200m-qwen3-100b" README, "SigmoidRouter", step_bias_update).
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates or frees device memory.  Scratch comes from the caller's
+ *     workspace `ws` of `ws_bytes` bytes (>= moe_workspace_size(cfg)), 256-byte
+ *     aligned.  Tensors are dense row-major.  "act" below means the activation /
+ *     weight dtype cfg->dtype (fp32 or bf16); router logits, scores, weights and
+ *     the selection bias are fp32 whatever the act dtype.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on it and performs no host synchronisation, except
+ *     moe_device_status().
+ *   - Arguments are validated before anything is launched; on error nothing
+ *     is launched and an error code is returned.  T == 0 is a valid no-op.
+ *   - Problems only the device can see (an expert id outside [0, E) in a
+ *     caller-supplied topk_idx; a bounded wait inside a kernel that gave up)
+ *     never fault: the kernel records them in a status word inside `ws` and
+ *     skips the offending work.  Each call clears the word when it starts;
+ *     read it with moe_device_status().
+ *   - No global state, no exceptions.  Calls on different streams with
+ *     different workspaces may run concurrently.
+ *   - Limits: 1 <= top_k <= min(E, 32), E <= 256.  bf16: d_model, d_ff and
+ *     d_ff_shared multiples of 128; fp32: d_model multiple of 4.  Pointers
+ *     16-byte aligned.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID = 1,      /* bad argument: null pointer, size, alignment     */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid layer, but outside this build's limits    */
+  MOE_ERR_WORKSPACE = 3,    /* ws_bytes < moe_workspace_size(cfg)               */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed             */
+  MOE_ERR_TIMEOUT = 5,      /* device status: a bounded wait gave up            */
+  MOE_ERR_DATA = 6          /* device status: expert id outside [0, E) skipped  */
+} moe_status;
+
+typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 } moe_gate;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Shape and recipe of one MoE layer (MoEModelConfig fields of the
+ * "moe-200m-qwen3-100b" README, plus the qwen3 preset switches of SpecForge
+ * PR #930).  Plain int32 fields so the layout is the same from every language. */
+typedef struct {
+  int32_t T;               /* tokens in the batch                          */
+  int32_t d_model;         /* hidden size d                                */
+  int32_t n_experts;       /* routed experts E                             */
+  int32_t d_ff;            /* routed expert width F                        */
+  int32_t top_k;           /* experts per token k                          */
+  int32_t n_shared;        /* 0 or 1 always-on shared expert               */
+  int32_t d_ff_shared;     /* shared expert width (0 when n_shared == 0)   */
+  int32_t gate;            /* moe_gate                                     */
+  int32_t norm_topk_prob;  /* 1: w /= (sum_j w_j + 1e-9)                   */
+  int32_t dtype;           /* moe_dtype of x, weights, out and the
+                              intermediate activations                     */
+} moe_config;
+
+/* Expert weights, stacked [E, out, in] (SpecForge PR #930):
+ *   w1 [E, F, d] gate, w3 [E, F, d] up, w2 [E, d, F] down;
+ *   ws1 [Fs, d], ws3 [Fs, d], ws2 [d, Fs] for the shared expert (NULL when
+ *   n_shared == 0).  All act dtype. */
+typedef struct {
+  const void* w1;
+  const void* w3;
+  const void* w2;
+  const void* ws1;
+  const void* ws3;
+  const void* ws2;
+} moe_expert_weights;
+
+/* Bytes of workspace every call below needs for this configuration
+ * (0 on an invalid configuration). */
+size_t moe_workspace_size(const moe_config* cfg);
+
+/* Validate a configuration without launching anything. */
+moe_status moe_check_config(const moe_config* cfg);
+
+/* Router: logits, gate, biased selection, top-k and combine weights.
+ * ("moe-200m-qwen3-100b" README, "SigmoidRouter" forward; "Per-layer
+ * numerics": routing in fp32.  SpecForge PR #930 "What this adds".)
+ *   x [T, d] act;  w_router [E, d] act;  sel_bias [E] fp32 or NULL (moves the
+ *   selection only, never the weights); logit_offset [E] fp32 or NULL (a
+ *   per-expert constant added to the logits before the gate and the
+ *   selection).
+ *   out: topk_idx [T, k] int32, descending selection key, equal keys -> lower
+ *   expert id; topk_w [T, k] fp32.  Logits: products of the inputs in fp32
+ *   (exact for bf16 inputs), summed in fp32 over 32-wide K chunks, chunk sums
+ *   added in fp64; selection keys, gate scores and the renormalisation in
+ *   fp64; weights stored as fp32. */
+moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router,
+                           const float* sel_bias, const float* logit_offset,
+                           int32_t* topk_idx, float* topk_w,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch: per-expert counts, offsets, and the stable expert-contiguous
+ * permutation of the T*k routed rows, with x gathered into that order.
+ * (Grouped-GEMM dispatch, SpecForge PR #930 "Why FSDP is enough here" and
+ * PR #931 "What works": grouped GEMM checked against a sorted loop.)
+ *   topk_idx [T, k] int32 (a pair whose id is outside [0, E) or repeats an
+ *   id earlier in the same token is skipped and reported as MOE_ERR_DATA by
+ *   moe_device_status); x [T, d] act.
+ *   out: counts [E] int32; offsets [E+1] int32 (exclusive prefix of counts);
+ *   slot_pos [T, k] int32 = row of pair (t, j) in the permuted order, i.e. the
+ *   position of (expert, t) in the stable sort of all pairs by (expert, token)
+ *   (-1 for a skipped pair); perm_src [T*k] int32 = token of each row;
+ *   x_perm [T*k, d] act, x_perm[slot_pos[t, j]] = x[t]. */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* slot_pos,
+                       int32_t* perm_src, void* x_perm,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Experts: grouped SwiGLU over the expert segments of x_perm, and the shared
+ * expert over x.  ("moe-200m-qwen3-100b" README, "Architecture diagram":
+ * routed SwiGLU experts and one always-on shared expert.)
+ *   x_perm [T*k, d] act; offsets [E+1] int32 (rows of expert e are
+ *   offsets[e] .. offsets[e+1]-1, offsets[E] <= T*k); weights as above;
+ *   x [T, d] act (read only when n_shared == 1).
+ *   out: y_perm [T*k, d] act, row r = expert_e(x_perm[r]) for the e owning r
+ *   (rows at or past offsets[E] are left untouched); y_shared [T, d] act or
+ *   NULL when n_shared == 0.  bf16: fp32 accumulation, the SwiGLU product
+ *   h = silu(g) * u is rounded to bf16 before the down projection. */
+moe_status moe_grouped_swiglu(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                              const moe_expert_weights* w, const void* x,
+                              void* y_perm, void* y_shared,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* Combine: out[t] = y_shared[t] + sum_{j<k, j ascending} topk_w[t, j] *
+ * y_perm[slot_pos[t, j]], accumulated in fp32, stored once in act dtype.
+ * ("moe-200m-qwen3-100b" README, "Architecture diagram": weighted sum.)
+ *   y_shared may be NULL (no shared expert); slot_pos entries < 0 are skipped. */
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
+                       const float* topk_w, const void* y_shared, void* out, void* stream);
+
+/* Selection-bias update from per-expert counts, in place, fp32, in the
+ * order of step_bias_update ("moe-200m-qwen3-100b" README, "SigmoidRouter"):
+ *   p = c / max(sum c, 1);  err = fp32(1/E) - p;
+ *   err += fp32(starved_add) where p < fp32(starved_frac * (1/E));
+ *   bias = clamp(bias + err * fp32(rate), -fp32(clamp), +fp32(clamp)).
+ * Each step is one correctly rounded fp32 operation (no fused multiply-add).
+ * counts must already be summed over data-parallel ranks (the README's
+ * all-reduce before the update).  Defaults on the page: rate 1e-3,
+ * starved_frac 0.1, starved_add 0.5, clamp 10. */
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* sel_bias,
+                           double rate, double starved_frac, double starved_add,
+                           double clamp, void* stream);
+
+/* The whole layer forward: router, dispatch, grouped SwiGLU experts (+ shared
+ * expert), combine.  Inputs as above; out [T, d] act.  Also returns the
+ * routing (topk_idx [T, k], topk_w [T, k]) and counts [E] for the caller's
+ * bias update; intermediates live in ws. */
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
+                       const float* sel_bias, const float* logit_offset,
+                       const moe_expert_weights* w, void* out,
+                       int32_t* topk_idx, float* topk_w, int32_t* counts,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward with CUDA events (cudaEvent_t, created by the caller) recorded
+ * on `stream` at the phase boundaries, for per-phase device timing:
+ *   events[0] start            events[1] after the router
+ *   events[2] after dispatch   events[3] after the routed gate/up GEMM
+ *   events[4] after the routed down GEMM
+ *   events[5] after the shared expert (== events[4] time when none)
+ *   events[6] after the combine (end)
+ * Same launches and results as moe_forward. */
+#define MOE_FORWARD_PHASES 6
+moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void* w_router,
+                                const float* sel_bias, const float* logit_offset,
+                                const moe_expert_weights* w, void* out,
+                                int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                void* ws, size_t ws_bytes, void* stream,
+                                void* const* events);
+
+/* Synchronise `stream`, read and clear the device status word in ws.
+ * Returns MOE_OK, MOE_ERR_DATA, MOE_ERR_TIMEOUT or MOE_ERR_CUDA; the raw
+ * flag bits are stored in *flags when flags is not NULL. */
+moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,213 @@
+"""Python binding of libmoe_b200.so (the C ABI declared in include/moe.h).
+
+Argument marshalling only: every function takes torch CUDA tensors (or None
+for optional pointers), passes their device addresses and sizes to the C entry
+point of the same name, and raises :class:`MoEError` on a non-zero status
+unless ``check=False``.  All arithmetic happens in the library's CUDA kernels;
+there is no fallback.  ``stream=None`` means torch's current stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Dict, Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "moe.h")
+
+MOE_OK = 0
+MOE_ERR_INVALID = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_WORKSPACE = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_TIMEOUT = 5
+MOE_ERR_DATA = 6
+
+GATE_SOFTMAX = 0
+GATE_SIGMOID = 1
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{msg} (status {status})")
+        self.status = status
+
+
+class MoEConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "T", "d_model", "n_experts", "d_ff", "top_k", "n_shared", "d_ff_shared",
+        "gate", "norm_topk_prob", "dtype")]
+
+
+class MoEExpertWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2")]
+
+
+_VP, _SZ, _I32, _F64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_double
+_CFG = ctypes.POINTER(MoEConfig)
+_WTS = ctypes.POINTER(MoEExpertWeights)
+_SIGNATURES = {
+    "moe_workspace_size": (_SZ, [_CFG]),
+    "moe_check_config": (_I32, [_CFG]),
+    "moe_router_topk": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_permute": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_grouped_swiglu": (_I32, [_CFG, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_combine": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_bias_update": (_I32, [_CFG, _VP, _VP, _F64, _F64, _F64, _F64, _VP]),
+    "moe_forward": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_forward_profiled": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ,
+                                     _VP, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_device_status": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_uint32)]),
+    "moe_status_string": (ctypes.c_char_p, [_I32]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (it must have been built; there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m mixture_experts_ffn_bias_b200.build` (needs nvcc)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/moe.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\*]+\s+\**(moe_\w+)\s*\(", text, re.M)))
+
+
+def status_string(st: int) -> str:
+    return lib().moe_status_string(int(st)).decode()
+
+
+def _check(st: int, check: bool) -> int:
+    if check and st != MOE_OK:
+        raise MoEError(st, status_string(st))
+    return st
+
+
+def make_config(T, d_model, n_experts, d_ff, top_k, n_shared=0, d_ff_shared=0,
+                gate=GATE_SOFTMAX, norm_topk_prob=1, dtype=DTYPE_BF16) -> MoEConfig:
+    return MoEConfig(T, d_model, n_experts, d_ff, top_k, n_shared,
+                     d_ff_shared if n_shared else 0, gate, norm_topk_prob, dtype)
+
+
+def config_from_shape(shape, T: Optional[int] = None) -> MoEConfig:
+    """MoEConfig for a workload of mixture_experts_ffn_bias_b200.inputs."""
+    return make_config(shape.T if T is None else T, shape.d_model, shape.n_experts,
+                       shape.d_ff, shape.top_k, shape.n_shared, shape.d_ff_shared,
+                       shape.gate, shape.norm_topk_prob, shape.dtype)
+
+
+def _p(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _s(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _nbytes(ws) -> int:
+    return ws.numel() * ws.element_size()
+
+
+def expert_weights(w: Dict) -> MoEExpertWeights:
+    return MoEExpertWeights(_p(w["w1"]), _p(w["w3"]), _p(w["w2"]),
+                            _p(w.get("ws1")), _p(w.get("ws3")), _p(w.get("ws2")))
+
+
+def moe_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_check_config(cfg: MoEConfig) -> int:
+    return int(lib().moe_check_config(ctypes.byref(cfg)))
+
+
+def moe_router_topk(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws,
+                    stream=None, check=True) -> int:
+    st = lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
+                               _p(logit_offset), _p(topk_idx), _p(topk_w), _p(ws),
+                               _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src, x_perm, ws,
+                stream=None, check=True) -> int:
+    st = lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts), _p(offsets),
+                           _p(slot_pos), _p(perm_src), _p(x_perm), _p(ws),
+                           _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_grouped_swiglu(cfg, x_perm, offsets, weights: Dict, x, y_perm, y_shared, ws,
+                       stream=None, check=True) -> int:
+    w = expert_weights(weights)
+    st = lib().moe_grouped_swiglu(ctypes.byref(cfg), _p(x_perm), _p(offsets), ctypes.byref(w),
+                                  _p(x), _p(y_perm), _p(y_shared), _p(ws),
+                                  _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_combine(cfg, y_perm, slot_pos, topk_w, y_shared, out, stream=None, check=True) -> int:
+    st = lib().moe_combine(ctypes.byref(cfg), _p(y_perm), _p(slot_pos), _p(topk_w),
+                           _p(y_shared), _p(out), _s(stream))
+    return _check(st, check)
+
+
+def moe_bias_update(cfg, counts, sel_bias, rate=1e-3, starved_frac=0.1, starved_add=0.5,
+                    clamp=10.0, stream=None, check=True) -> int:
+    st = lib().moe_bias_update(ctypes.byref(cfg), _p(counts), _p(sel_bias), rate,
+                               starved_frac, starved_add, clamp, _s(stream))
+    return _check(st, check)
+
+
+def moe_forward(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, topk_idx,
+                topk_w, counts, ws, stream=None, check=True) -> int:
+    w = expert_weights(weights)
+    st = lib().moe_forward(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
+                           _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),
+                           _p(topk_w), _p(counts), _p(ws),
+                           _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+FORWARD_PHASES = 6
+
+
+def moe_forward_profiled(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, topk_idx,
+                         topk_w, counts, ws, events, stream=None, check=True) -> int:
+    """``events``: FORWARD_PHASES + 1 torch.cuda.Event objects (timing enabled)."""
+    w = expert_weights(weights)
+    arr = (ctypes.c_void_p * (FORWARD_PHASES + 1))(*[e.cuda_event for e in events])
+    st = lib().moe_forward_profiled(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
+                                    _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),
+                                    _p(topk_w), _p(counts), _p(ws),
+                                    _nbytes(ws) if ws is not None else 0, _s(stream), arr)
+    return _check(st, check)
+
+
+def moe_device_status(ws, stream=None):
+    """(status, raw flag bits); synchronises the stream."""
+    flags = ctypes.c_uint32(0)
+    st = lib().moe_device_status(_p(ws), _nbytes(ws), _s(stream), ctypes.byref(flags))
+    return int(st), int(flags.value)

@@ -1,0 +1,435 @@
+// Grouped GEMM over expert segments on 5th-generation tensor cores (tcgen05).
+//
+// For every group g (an expert, or the single shared-expert group) with rows
+// [off[g], off[g+1]) of A:
+//   SWIGLU pass (gate/up):  h[r, n] = silu(A[r] . W1[g][n]) * (A[r] . W3[g][n])
+//   plain pass  (down):     y[r, n] = A[r] . W2[g][n]
+// i.e. the two halves of the SwiGLU expert y = W2 (silu(W1 x) * (W3 x)) run
+// over the expert-contiguous rows that grouped_mm dispatch consumes (SpecForge
+// PR #930, "Why FSDP is enough here": compute scales with routed tokens, not
+// with the number of experts; weights stacked [E, out, in]).
+//
+// Kernel design (one CTA per SM, persistent, static round-robin over tiles):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile(s) N x 64 per stage,
+//               128-byte swizzle, STAGES-deep ring of shared-memory buffers.
+//   warp 1      allocates TMEM (2 accumulators), one lane issues
+//               tcgen05.mma (M=128, N=BN_ACC, K=16, bf16 x bf16 -> fp32) and
+//               tcgen05.commit to release smem stages / publish accumulators.
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (thread = row), apply
+//               SwiGLU (gate and up columns of the same output column sit in
+//               the same accumulator: B rows 0-127 come from W1, 128-255 from
+//               W3), round to bf16 and store the row segment.
+// The TMEM accumulator is double buffered so the epilogue of tile i overlaps
+// the MMAs of tile i+1.  Tile order is (group, m-tile, n-tile) with n fastest,
+// so CTAs running at the same time share the A tile and one expert's weights
+// in L2.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                    // 64 bf16 = 128 bytes = one swizzle row
+constexpr int A_STAGE_BYTES = BM * BK * 2;
+constexpr int NUM_THREADS = 192;          // 6 warps
+constexpr int MAX_GROUPS = 257;
+
+template <int BN_ACC>
+struct GemmCfg {
+  static constexpr int B_STAGE_BYTES = BN_ACC * BK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int TMEM_COLS = 2 * BN_ACC;      // double-buffered accumulator
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*bars*/;
+};
+
+struct GemmArgs {
+  const int32_t* offsets;  // [G+1] device, or nullptr: one group [0, rows_single)
+  int num_groups;
+  int rows_single;
+  int n_per_group;         // output columns per group (= B rows per group)
+  int K;
+  __nv_bfloat16* C;
+  int ldc;
+  uint32_t* status;
+};
+
+__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// One warp computes per-group tile prefixes: prefix[g] = sum_{g' < g} m_tiles(g') * n_tiles.
+__device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, int* s_prefix) {
+  const int lane = threadIdx.x & 31;
+  const int G = a.num_groups;
+  if (a.offsets == nullptr) {
+    if (lane == 0) {
+      s_off[0] = 0;
+      s_off[1] = a.rows_single;
+      s_prefix[0] = 0;
+      s_prefix[1] = ((a.rows_single + BM - 1) / BM) * n_tiles;
+    }
+    __syncwarp();
+    return;
+  }
+  for (int i = lane; i <= G; i += 32) s_off[i] = a.offsets[i];
+  __syncwarp();
+  const int per = (G + 31) / 32;
+  const int g0 = lane * per;
+  int local = 0;
+  for (int g = g0; g < g0 + per && g < G; ++g) {
+    const int rows = s_off[g + 1] - s_off[g];
+    local += ((rows > 0 ? rows : 0) + BM - 1) / BM * n_tiles;
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - local;
+  for (int g = g0; g < g0 + per && g < G; ++g) {
+    s_prefix[g] = run;
+    const int rows = s_off[g + 1] - s_off[g];
+    run += ((rows > 0 ? rows : 0) + BM - 1) / BM * n_tiles;
+  }
+  if (lane == 31) s_prefix[G] = incl;
+  __syncwarp();
+}
+
+// Largest g with prefix[g] <= tile (groups with no tiles are skipped).
+__device__ __forceinline__ int find_group(const int* s_prefix, int G, int tile) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int BN_ACC, bool SWIGLU>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1,
+                    const GemmArgs args) {
+  using Cfg = GemmCfg<BN_ACC>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN_ACC);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smemA = smem;
+  uint8_t* smemB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* tfull_bar = bars + 2 * STAGES;
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+
+  __shared__ int s_off[MAX_GROUPS + 1];
+  __shared__ int s_prefix[MAX_GROUPS + 1];
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = args.n_per_group / BN_OUT;
+  const int G = args.offsets == nullptr ? 1 : args.num_groups;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (SWIGLU) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem_base, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 2) build_tile_prefix(args, n_tiles, s_off, s_prefix);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int total_tiles = s_prefix[G];
+  volatile int* abort_flag = &s_abort;
+  const int kblocks = args.K / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;     // stages with a load in flight at exit
+      uint32_t issued_phase = 0;    // parity of that load's phase
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+        const int g = find_group(s_prefix, G, tile);
+        const int local = tile - s_prefix[g];
+        const int m = local / n_tiles;
+        const int n = local - m * n_tiles;
+        const int arow = s_off[g] + m * BM;
+        const int brow = g * args.n_per_group + n * BN_OUT;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
+          uint8_t* b = smemB + stage * Cfg::B_STAGE_BYTES;
+          if (SWIGLU) {
+            tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
+            tma_load_2d(b + (BN_ACC / 2) * BK * 2, &tmB1, &full_bar[stage], kb * BK, brow);
+          } else {
+            tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // Let every TMA copy this CTA started land before the CTA exits.
+        for (int s = 0; s < STAGES; ++s) {
+          if (!(issued_mask & (1u << s))) continue;
+          const uint32_t par = (issued_phase >> s) & 1u;
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full_bar[s], par)) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN_ACC;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smemA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(smemB + stage * Cfg::B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_addr + kk * 32);
+            const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
+            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull_bar[acc]);
+      }
+      if (!ok && issued_any) {
+        // Wait (bounded) for the MMAs already issued before TMEM is freed.
+        tc_commit(drain_bar);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                   // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;            // accumulator row owned by this thread
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      // every lane waits (memory ordering); the decision is made warp-uniform
+      // so the .sync.aligned TMEM loads below never run with a lane missing
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int g = find_group(s_prefix, G, tile);
+      const int local = tile - s_prefix[g];
+      const int m = local / n_tiles;
+      const int n = local - m * n_tiles;
+      const int rows_g = s_off[g + 1] - s_off[g];
+      const bool valid = (m * BM + row) < rows_g;
+      __nv_bfloat16* crow = args.C + static_cast<size_t>(s_off[g] + m * BM + row) * args.ldc +
+                            static_cast<size_t>(n) * BN_OUT;
+      const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN_OUT / 16; ++c) {
+        uint32_t v[16];
+        uint32_t packed[8];
+        if (SWIGLU) {
+          uint32_t u[16];
+          tmem_ld16(t_addr + c * 16, v);
+          tmem_ld16(t_addr + BN_OUT + c * 16, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+            const float h1 = silu_f32(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+            packed[i] = pack_bf16x2(h0, h1);
+          }
+        } else {
+          tmem_ld16(t_addr + c * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(crow + c * 16);
+          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && s_abort) atomicOr(args.status, kDevTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of box_rows x 64 with the
+// 128-byte swizzle; rows past `rows` read as zero.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int BN_ACC, bool SWIGLU>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                   const GemmArgs& args, int rows_upper, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN_ACC>;
+  constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
+  auto kern = grouped_gemm_kernel<BN_ACC, SWIGLU>;
+  static unsigned long long attr_done = 0;   // one bit per device (attribute is per device)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_done & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done |= bit;
+  }
+  const int G = args.offsets == nullptr ? 1 : args.num_groups;
+  const long long m_tiles_upper = (rows_upper + BM - 1) / BM + (G > 1 ? G : 0);
+  const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
+  if (tiles_upper <= 0) return cudaSuccess;
+  const int grid = static_cast<int>(tiles_upper < num_sms() ? tiles_upper : num_sms());
+  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// h[r] = silu(A[r] W1[g]^T) * (A[r] W3[g]^T), bf16 out.
+cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                       int num_groups, int rows_single, const void* W1,
+                                       const void* W3, int F, int K, void* H, uint32_t* status,
+                                       cudaStream_t stream) {
+  CUtensorMap ta, tb0, tb1;
+  const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
+      !make_map(&tb1, W3, b_rows, K, 128))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, rows_single, F, K,
+                static_cast<__nv_bfloat16*>(H), F, status};
+  const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  return launch<256, true>(ta, tb0, tb1, args, rows_upper, stream);
+}
+
+// Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.
+cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                              int num_groups, int rows_single, const void* W2, int N, int K,
+                              void* Y, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
+  const int bn = (N % 256 == 0) ? 256 : 128;
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, rows_single, N, K,
+                static_cast<__nv_bfloat16*>(Y), N, status};
+  const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (bn == 256) return launch<256, false>(ta, tb, tb, args, rows_upper, stream);
+  return launch<128, false>(ta, tb, tb, args, rows_upper, stream);
+}
+
+}  // namespace moe

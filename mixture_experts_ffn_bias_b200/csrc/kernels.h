@@ -1,0 +1,57 @@
+// Launchers of the CUDA kernels behind the C ABI (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace moe {
+
+// Bits of the device status word kept at the start of the workspace.
+constexpr uint32_t kDevBadIndex = 1u;   // expert id outside [0, E) or repeated in a token
+constexpr uint32_t kDevTimeout = 2u;    // a bounded wait inside a kernel gave up
+
+// Router ---------------------------------------------------------------------
+// logits[T, E] (fp64 scratch) = x . w_router^T (+ logit_offset), exact products
+// with fp32 partial sums over 32-wide K chunks added in fp64.
+cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
+                          const float* logit_offset, int T, int d, int E, double* logits,
+                          cudaStream_t stream);
+// gate scores, biased selection, top-k, combine weights from the logits.
+cudaError_t router_select(const double* logits, const float* sel_bias, int T, int E, int k,
+                          int gate, int renorm, int32_t* topk_idx, float* topk_w,
+                          cudaStream_t stream);
+
+// Dispatch -------------------------------------------------------------------
+constexpr int kRankBlock = 256;   // tokens per histogram block
+inline int rank_blocks(int T) { return (T + kRankBlock - 1) / kRankBlock; }
+cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,
+                          int32_t* rank_out, uint32_t* status, cudaStream_t stream);
+cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
+                          int32_t* offsets, cudaStream_t stream);
+cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
+                             const int32_t* blk_bases, int32_t* slot_pos, int32_t* perm_src,
+                             void* x_perm, int T, int d, int k, int E, cudaStream_t stream);
+
+// Experts --------------------------------------------------------------------
+cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                       int num_groups, int rows_single, const void* W1,
+                                       const void* W3, int F, int K, void* H, uint32_t* status,
+                                       cudaStream_t stream);
+cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                              int num_groups, int rows_single, const void* W2, int N, int K,
+                              void* Y, uint32_t* status, cudaStream_t stream);
+cudaError_t grouped_swiglu_gateup_f32(const float* A, int64_t a_rows, const int32_t* offsets,
+                                      int num_groups, int rows_single, const float* W1,
+                                      const float* W3, int F, int K, float* H,
+                                      cudaStream_t stream);
+cudaError_t grouped_down_f32(const float* A, int64_t a_rows, const int32_t* offsets,
+                             int num_groups, int rows_single, const float* W2, int N, int K,
+                             float* Y, cudaStream_t stream);
+
+// Combine / bias ---------------------------------------------------------------
+cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
+                    const void* y_shared, void* out, int T, int d, int k, cudaStream_t stream);
+cudaError_t bias_update(const int32_t* counts, float* bias, int E, float target, float thresh,
+                        float starved_add, float rate, float clamp, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,371 @@
+// C ABI of the MoE FFN layer (declared in include/moe.h): argument
+// validation, workspace layout and the launch sequence of each call.
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// Workspace layout shared by every call.  Byte offsets from the base.
+struct Layout {
+  size_t status, blk, offsets, slot_pos, perm_src, logits, x_perm, h, y_perm, h_sh, y_sh, total;
+};
+
+inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
+
+Layout layout(const moe_config& c) {
+  const size_t T = static_cast<size_t>(c.T), d = c.d_model, E = c.n_experts, F = c.d_ff,
+               k = c.top_k, R = T * k, es = esize(c);
+  const size_t Fs = c.n_shared ? static_cast<size_t>(c.d_ff_shared) : 0;
+  Layout L{};
+  size_t o = 0;
+  L.status = o;   o += up(sizeof(uint32_t));
+  L.blk = o;      o += up(static_cast<size_t>(moe::rank_blocks(c.T)) * E * 4);
+  L.offsets = o;  o += up((E + 1) * 4);
+  L.slot_pos = o; o += up(R * 4);
+  L.perm_src = o; o += up(R * 4);
+  L.logits = o;   o += up(T * E * 8);
+  L.x_perm = o;   o += up(R * d * es);
+  L.h = o;        o += up(R * F * es);
+  L.y_perm = o;   o += up(R * d * es);
+  L.h_sh = o;     o += up(T * Fs * es);
+  L.y_sh = o;     o += up(c.n_shared ? T * d * es : 0);
+  L.total = o;
+  return L;
+}
+
+template <typename P>
+inline P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+moe_status check_cfg(const moe_config* c) {
+  if (c == nullptr) return MOE_ERR_INVALID;
+  if (c->T < 0 || c->d_model < 1 || c->n_experts < 1 || c->d_ff < 1 || c->top_k < 1)
+    return MOE_ERR_INVALID;
+  if (c->top_k > c->n_experts) return MOE_ERR_INVALID;
+  if (c->n_shared != 0 && c->n_shared != 1) return MOE_ERR_INVALID;
+  if (c->n_shared == 1 && c->d_ff_shared < 1) return MOE_ERR_INVALID;
+  if (c->gate != MOE_GATE_SOFTMAX && c->gate != MOE_GATE_SIGMOID) return MOE_ERR_INVALID;
+  if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1) return MOE_ERR_INVALID;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (c->n_experts > 256 || c->top_k > 32) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(c->T) * c->top_k > 0x3fffffffLL) return MOE_ERR_UNSUPPORTED;
+  if (c->dtype == MOE_BF16) {
+    if (c->d_model % 128 || c->d_ff % 128 || (c->n_shared && c->d_ff_shared % 128))
+      return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (c->d_model % 4) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config* c, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MOE_ERR_INVALID;
+  if (ws_bytes < layout(*c).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+#define MOE_TRY(expr)                                   \
+  do {                                                  \
+    if ((expr) != cudaSuccess) return MOE_ERR_CUDA;     \
+  } while (0)
+
+moe_status clear_status(void* ws, cudaStream_t s) {
+  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, sizeof(uint32_t), s));
+  return MOE_OK;
+}
+
+// Router into caller buffers; logits scratch in ws.
+moe_status run_router(const moe_config* c, const void* x, const void* w_router,
+                      const float* sel_bias, const float* logit_offset, int32_t* topk_idx,
+                      float* topk_w, void* ws, cudaStream_t s) {
+  const Layout L = layout(*c);
+  double* logits = at<double>(ws, L.logits);
+  MOE_TRY(moe::router_logits(c->dtype == MOE_BF16, x, w_router, logit_offset, c->T, c->d_model,
+                             c->n_experts, logits, s));
+  MOE_TRY(moe::router_select(logits, sel_bias, c->T, c->n_experts, c->top_k, c->gate,
+                             c->norm_topk_prob, topk_idx, topk_w, s));
+  return MOE_OK;
+}
+
+moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_src,
+                       void* x_perm, void* ws, cudaStream_t s) {
+  const Layout L = layout(*c);
+  int32_t* blk = at<int32_t>(ws, L.blk);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  const int nblk = moe::rank_blocks(c->T);
+  MOE_TRY(moe::dispatch_rank(topk_idx, c->T, c->top_k, c->n_experts, blk, slot_pos, status, s));
+  MOE_TRY(moe::dispatch_scan(blk, nblk, c->n_experts, counts, offsets, s));
+  MOE_TRY(moe::dispatch_scatter(c->dtype == MOE_BF16, x, topk_idx, blk, slot_pos, perm_src,
+                                x_perm, c->T, c->d_model, c->top_k, c->n_experts, s));
+  return MOE_OK;
+}
+
+// Optional CUDA events recorded between the phases of moe_forward_profiled.
+struct Marks {
+  void* const* ev;
+  cudaStream_t s;
+  bool rec(int i) const {
+    return ev == nullptr || cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess;
+  }
+};
+
+moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* offsets,
+                       const moe_expert_weights* w, const void* x, void* y_perm, void* y_shared,
+                       void* ws, cudaStream_t s, const Marks& mk) {
+  const Layout L = layout(*c);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  const int64_t R = static_cast<int64_t>(c->T) * c->top_k;
+  const int E = c->n_experts, F = c->d_ff, d = c->d_model;
+  void* h = at<void>(ws, L.h);
+  if (c->dtype == MOE_BF16) {
+    MOE_TRY(moe::grouped_swiglu_gateup_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d, h,
+                                            status, s));
+    if (!mk.rec(3)) return MOE_ERR_CUDA;
+    MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s));
+    if (!mk.rec(4)) return MOE_ERR_CUDA;
+    if (c->n_shared) {
+      void* hs = at<void>(ws, L.h_sh);
+      const int Fs = c->d_ff_shared;
+      MOE_TRY(moe::grouped_swiglu_gateup_bf16(x, c->T, nullptr, 1, c->T, w->ws1, w->ws3, Fs, d,
+                                              hs, status, s));
+      MOE_TRY(moe::grouped_down_bf16(hs, c->T, nullptr, 1, c->T, w->ws2, d, Fs, y_shared,
+                                     status, s));
+    }
+  } else {
+    float* hf = static_cast<float*>(h);
+    MOE_TRY(moe::grouped_swiglu_gateup_f32(static_cast<const float*>(x_perm), R, offsets, E, 0,
+                                           static_cast<const float*>(w->w1),
+                                           static_cast<const float*>(w->w3), F, d, hf, s));
+    if (!mk.rec(3)) return MOE_ERR_CUDA;
+    MOE_TRY(moe::grouped_down_f32(hf, R, offsets, E, 0, static_cast<const float*>(w->w2), d, F,
+                                  static_cast<float*>(y_perm), s));
+    if (!mk.rec(4)) return MOE_ERR_CUDA;
+    if (c->n_shared) {
+      float* hs = at<float>(ws, L.h_sh);
+      const int Fs = c->d_ff_shared;
+      MOE_TRY(moe::grouped_swiglu_gateup_f32(static_cast<const float*>(x), c->T, nullptr, 1,
+                                             c->T, static_cast<const float*>(w->ws1),
+                                             static_cast<const float*>(w->ws3), Fs, d, hs, s));
+      MOE_TRY(moe::grouped_down_f32(hs, c->T, nullptr, 1, c->T,
+                                    static_cast<const float*>(w->ws2), d, Fs,
+                                    static_cast<float*>(y_shared), s));
+    }
+  }
+  if (!mk.rec(5)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_config* c, const moe_expert_weights* w) {
+  if (w == nullptr || !w->w1 || !w->w3 || !w->w2) return MOE_ERR_INVALID;
+  if (!aligned16(w->w1) || !aligned16(w->w3) || !aligned16(w->w2)) return MOE_ERR_INVALID;
+  if (c->n_shared) {
+    if (!w->ws1 || !w->ws3 || !w->ws2) return MOE_ERR_INVALID;
+    if (!aligned16(w->ws1) || !aligned16(w->ws3) || !aligned16(w->ws2)) return MOE_ERR_INVALID;
+  }
+  return MOE_OK;
+}
+
+moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_router,
+                        const float* sel_bias, const float* logit_offset,
+                        const moe_expert_weights* w, void* out, int32_t* topk_idx,
+                        float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream,
+                        void* const* events) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts) return MOE_ERR_INVALID;
+  if (cfg->T == 0) {
+    MOE_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, S(stream)));
+    return MOE_OK;
+  }
+  if (!x || !w_router || !out || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  if ((st = check_weights(cfg, w)) != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(out) || !aligned4(topk_idx) ||
+      !aligned4(topk_w) || !aligned4(counts) || (sel_bias && !aligned4(sel_bias)) ||
+      (logit_offset && !aligned4(logit_offset)))
+    return MOE_ERR_INVALID;
+  if (events)
+    for (int i = 0; i <= MOE_FORWARD_PHASES; ++i)
+      if (!events[i]) return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  const Layout L = layout(*cfg);
+  cudaStream_t s = S(stream);
+  const Marks mk{events, s};
+  if ((st = clear_status(ws, s)) != MOE_OK) return st;
+  if (!mk.rec(0)) return MOE_ERR_CUDA;
+  if ((st = run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, s)) !=
+      MOE_OK)
+    return st;
+  if (!mk.rec(1)) return MOE_ERR_CUDA;
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* slot_pos = at<int32_t>(ws, L.slot_pos);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* y_perm = at<void>(ws, L.y_perm);
+  void* y_sh = cfg->n_shared ? at<void>(ws, L.y_sh) : nullptr;
+  if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, at<int32_t>(ws, L.perm_src),
+                        x_perm, ws, s)) != MOE_OK)
+    return st;
+  if (!mk.rec(2)) return MOE_ERR_CUDA;
+  if ((st = run_experts(cfg, x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk)) != MOE_OK)
+    return st;
+  MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_sh, out, cfg->T,
+                       cfg->d_model, cfg->top_k, s));
+  if (!mk.rec(MOE_FORWARD_PHASES)) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return layout(*cfg).total;
+}
+
+moe_status moe_check_config(const moe_config* cfg) { return check_cfg(cfg); }
+
+moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router,
+                           const float* sel_bias, const float* logit_offset, int32_t* topk_idx,
+                           float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned4(topk_idx) || !aligned4(topk_w) ||
+      (sel_bias && !aligned4(sel_bias)) || (logit_offset && !aligned4(logit_offset)))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
+  return run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, S(stream));
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                       int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_src,
+                       void* x_perm, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets) return MOE_ERR_INVALID;
+  if (cfg->T == 0) {
+    MOE_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, S(stream)));
+    MOE_TRY(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (cfg->n_experts + 1), S(stream)));
+    return MOE_OK;
+  }
+  if (!topk_idx || !x || !slot_pos || !perm_src || !x_perm) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(x_perm) || !aligned4(topk_idx) || !aligned4(counts) ||
+      !aligned4(offsets) || !aligned4(slot_pos) || !aligned4(perm_src))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
+  return run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src, x_perm, ws,
+                     S(stream));
+}
+
+moe_status moe_grouped_swiglu(const moe_config* cfg, const void* x_perm, const int32_t* offsets,
+                              const moe_expert_weights* w, const void* x, void* y_perm,
+                              void* y_shared, void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x_perm || !offsets || !y_perm) return MOE_ERR_INVALID;
+  if ((st = check_weights(cfg, w)) != MOE_OK) return st;
+  if (cfg->n_shared && (!x || !y_shared)) return MOE_ERR_INVALID;
+  if (!cfg->n_shared && y_shared) return MOE_ERR_INVALID;
+  if (!aligned16(x_perm) || !aligned16(y_perm) || !aligned4(offsets) ||
+      (x && !aligned16(x)) || (y_shared && !aligned16(y_shared)))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
+  return run_experts(cfg, x_perm, offsets, w, x, y_perm, y_shared, ws, S(stream),
+                     Marks{nullptr, S(stream)});
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
+                       const float* topk_w, const void* y_shared, void* out, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!y_perm || !slot_pos || !topk_w || !out) return MOE_ERR_INVALID;
+  if (cfg->n_shared && !y_shared) return MOE_ERR_INVALID;
+  if (!cfg->n_shared && y_shared) return MOE_ERR_INVALID;
+  if (!aligned16(y_perm) || !aligned16(out) || !aligned4(slot_pos) || !aligned4(topk_w) ||
+      (y_shared && !aligned16(y_shared)))
+    return MOE_ERR_INVALID;
+  MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_shared, out, cfg->T,
+                       cfg->d_model, cfg->top_k, S(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* sel_bias,
+                           double rate, double starved_frac, double starved_add, double clamp,
+                           void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !sel_bias || !aligned4(counts) || !aligned4(sel_bias)) return MOE_ERR_INVALID;
+  if (!(clamp >= 0.0)) return MOE_ERR_INVALID;
+  const double inv_e = 1.0 / static_cast<double>(cfg->n_experts);
+  MOE_TRY(moe::bias_update(counts, sel_bias, cfg->n_experts, static_cast<float>(inv_e),
+                           static_cast<float>(starved_frac * inv_e),
+                           static_cast<float>(starved_add), static_cast<float>(rate),
+                           static_cast<float>(clamp), S(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_router,
+                       const float* sel_bias, const float* logit_offset,
+                       const moe_expert_weights* w, void* out, int32_t* topk_idx, float* topk_w,
+                       int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, x, w_router, sel_bias, logit_offset, w, out, topk_idx, topk_w, counts,
+                      ws, ws_bytes, stream, nullptr);
+}
+
+moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void* w_router,
+                                const float* sel_bias, const float* logit_offset,
+                                const moe_expert_weights* w, void* out, int32_t* topk_idx,
+                                float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                void* stream, void* const* events) {
+  if (events == nullptr) return MOE_ERR_INVALID;
+  return forward_impl(cfg, x, w_router, sel_bias, logit_offset, w, out, topk_idx, topk_w, counts,
+                      ws, ws_bytes, stream, events);
+}
+
+moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags) {
+  if (ws == nullptr || ws_bytes < sizeof(uint32_t)) return MOE_ERR_INVALID;
+  uint32_t v = 0;
+  MOE_TRY(cudaStreamSynchronize(S(stream)));
+  MOE_TRY(cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost));
+  MOE_TRY(cudaMemset(ws, 0, sizeof(v)));
+  if (flags) *flags = v;
+  if (v & moe::kDevTimeout) return MOE_ERR_TIMEOUT;
+  if (v & moe::kDevBadIndex) return MOE_ERR_DATA;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "configuration outside the supported limits";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case MOE_ERR_DATA: return "expert index outside [0, E) or repeated within a token";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -201,6 +201,24 @@ def moe_forward(inp: dict, top_k: int, gate: int, norm_topk_prob: bool,
     return out, routing
 
 
+def combine(y_perm, slot_pos, topk_w, y_shared=None) -> np.ndarray:
+    """Weighted un-permute: out[t] = y_shared[t] + sum_j w[t, j] * y_perm[slot_pos[t, j]].
+
+    The "weighted sum" of the "Architecture diagram" in the
+    "moe-200m-qwen3-100b" README, with the routed outputs held in
+    expert-contiguous rows.  Pairs with a negative slot contribute nothing.
+    """
+    y = _as64(y_perm)
+    sp = np.asarray(slot_pos, dtype=np.int64)
+    w = _as64(topk_w)
+    T, k = sp.shape
+    out = np.zeros((T, y.shape[1])) if y_shared is None else _as64(y_shared).copy()
+    for j in range(k):
+        ok = sp[:, j] >= 0
+        out[ok] += w[ok, j:j + 1] * y[sp[ok, j]]
+    return out
+
+
 def moe_forward_dense_masked(inp: dict, top_k: int, gate: int, norm_topk_prob: bool):
     """Brute force: every expert on every token, masked by the combine weights.
 

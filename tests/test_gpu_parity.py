@@ -1,0 +1,323 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Small shapes span several tiles with ragged tails and are compared element by
+element; the full workload sizes (the ones the benchmark times) are compared on
+all routing decisions and on a sample of output rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import _parity as P
+from mixture_experts_ffn_bias_b200 import binding as B
+from mixture_experts_ffn_bias_b200 import build as build_mod
+from mixture_experts_ffn_bias_b200 import inputs as I
+from mixture_experts_ffn_bias_b200.layer import MoELayer, to_device
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": I.WORKLOADS["tiny"],
+    "page2_small": I.WORKLOADS["page2"].replace(T=640),
+    "qwen3_small": I.WORKLOADS["qwen3_30b"].replace(T=600, d_model=256, d_ff=256),
+    "wide_small": I.WORKLOADS["wide"].replace(T=200, d_model=512, d_ff=384),
+    "skew_small": I.WORKLOADS["skew"].replace(T=1000, d_model=256, d_ff=256, d_ff_shared=256),
+}
+FULL = ["page2", "qwen3_30b", "wide", "skew"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build_mod.build()
+    B.lib()
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy() if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
+
+
+def _tol(shape):
+    return P.OUT_TOL_BF16 if shape.dtype == I.DTYPE_BF16 else P.OUT_TOL_F32
+
+
+def _run(shape, host):
+    layer = MoELayer(shape, host)
+    layer.forward()
+    torch.cuda.synchronize()
+    st, flags = layer.device_status()
+    assert st == B.MOE_OK, (st, flags)
+    return layer
+
+
+def _check_layer(shape, host, layer, tokens=None):
+    r = P.oracle_routing(shape, host)
+    gidx, gw = _np(layer.topk_idx), _np(layer.topk_w)
+    excluded, ordered = P.check_routing(gidx, gw, r)
+    P.check_counts_vs_oracle(_np(layer.counts), r, gidx, shape.n_experts, excluded)
+    sel = np.arange(shape.T) if tokens is None else tokens
+    sel = sel[~excluded[sel]]
+    ref, _ = O.moe_forward(host, shape.top_k, shape.gate, bool(shape.norm_topk_prob),
+                           tokens=sel, routing=r)
+    err = P.rel_err(_np(layer.out)[sel], ref)
+    assert err <= _tol(shape), f"output relative error {err:.3e}"
+    return r, excluded, err
+
+
+# --------------------------------------------------------------------------- #
+# whole layer                                                                 #
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_small_elementwise(name):
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    layer = _run(shape, host)
+    _check_layer(shape, host, layer)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_forward_full_size_sampled(name):
+    shape = I.WORKLOADS[name]
+    host = I.make_inputs(shape)
+    layer = _run(shape, host)
+    _check_layer(shape, host, layer, tokens=P.sample_tokens(shape.T, 48))
+    del layer
+    torch.cuda.empty_cache()
+
+
+def test_skew_bias_update_then_deferred_forward():
+    """Skewed workload: forward, bias update from its counts (bit-exact), then a
+    second forward routes with the new bias (the update lands on the next
+    forward)."""
+    shape = I.WORKLOADS["skew"].replace(T=4096, d_model=512, d_ff=256, d_ff_shared=256)
+    host = I.make_inputs(shape)
+    layer = _run(shape, host)
+    r = P.oracle_routing(shape, host)
+    excluded, _ = P.check_routing(_np(layer.topk_idx), _np(layer.topk_w), r)
+    assert not excluded.any()
+    counts_ref = O.dispatch(r.topk_idx, shape.n_experts).counts
+    np.testing.assert_array_equal(_np(layer.counts), counts_ref)
+    assert (counts_ref == 0).any(), "Zipf offsets should starve some experts"
+    layer.bias_update(rate=1e-3, starved_frac=0.1, starved_add=0.5, clamp=10.0)
+    torch.cuda.synchronize()
+    bias_ref = O.bias_update(counts_ref, host["sel_bias"], 1e-3, 0.1, 0.5, 10.0)
+    np.testing.assert_array_equal(_np(layer.sel_bias), bias_ref)
+    layer.forward()
+    torch.cuda.synchronize()
+    r2 = P.oracle_routing(shape, host, sel_bias=bias_ref)
+    P.check_routing(_np(layer.topk_idx), _np(layer.topk_w), r2)
+
+
+# --------------------------------------------------------------------------- #
+# edge cases                                                                  #
+# --------------------------------------------------------------------------- #
+def test_single_token():
+    shape = SMALL["qwen3_small"].replace(T=1)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
+def test_zero_tokens_is_a_noop():
+    shape = SMALL["page2_small"].replace(T=0)
+    cfg = B.config_from_shape(shape)
+    counts = torch.full((shape.n_experts,), 7, dtype=torch.int32, device="cuda")
+    dummy = torch.empty(64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    w = {"w1": dummy, "w3": dummy, "w2": dummy, "ws1": dummy, "ws3": dummy, "ws2": dummy}
+    assert B.moe_forward(cfg, dummy, dummy, None, None, w, dummy, dummy, dummy, counts, ws) == 0
+    torch.cuda.synchronize()
+    assert int(counts.abs().sum()) == 0
+
+
+def test_one_expert_top1_is_dense_ffn():
+    shape = I.MoEShape("one", 300, 256, 1, 256, 1, 0, 0, I.GATE_SOFTMAX, 1, I.DTYPE_BF16,
+                       "none", 0.0, 7)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
+def test_top_k_equals_all_experts():
+    shape = I.MoEShape("all", 257, 128, 8, 128, 8, 0, 0, I.GATE_SOFTMAX, 1, I.DTYPE_BF16,
+                       "none", 0.0, 8)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
+def test_every_token_on_one_expert():
+    """A huge bias on one expert: one segment of T rows, all others empty."""
+    shape = SMALL["skew_small"].replace(T=700)
+    host = I.make_inputs(shape)
+    host["sel_bias"] = np.zeros(shape.n_experts, np.float32)
+    host["sel_bias"][37] = 50.0
+    layer = _run(shape, host)
+    c = _np(layer.counts)
+    assert c[37] == shape.T and c.sum() == shape.T * shape.top_k
+    _check_layer(shape, host, layer)
+
+
+@pytest.mark.parametrize("gate", [I.GATE_SOFTMAX, I.GATE_SIGMOID])
+def test_constant_bias_moves_nothing_on_gpu(gate):
+    shape = SMALL["qwen3_small"].replace(gate=gate, T=512)
+    host = I.make_inputs(shape)
+    a = _run(shape, host)
+    idx0, w0 = _np(a.topk_idx).copy(), _np(a.topk_w).copy()
+    host2 = dict(host)
+    host2["sel_bias"] = np.full(shape.n_experts, 0.25, np.float32)
+    b = _run(shape, host2)
+    np.testing.assert_array_equal(_np(b.topk_idx), idx0)
+    np.testing.assert_array_equal(_np(b.topk_w), w0)
+
+
+# --------------------------------------------------------------------------- #
+# the individual calls                                                        #
+# --------------------------------------------------------------------------- #
+def _buffers(shape):
+    cfg = B.config_from_shape(shape)
+    ws = torch.empty(B.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    return cfg, ws
+
+
+@pytest.mark.parametrize("name", ["tiny", "page2_small", "skew_small"])
+def test_router_topk_call(name):
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    cfg, ws = _buffers(shape)
+    dt = torch.bfloat16 if shape.dtype == I.DTYPE_BF16 else torch.float32
+    x = to_device(host["x"], dt, "cuda")
+    wr = to_device(host["w_router"], dt, "cuda")
+    bias = to_device(host["sel_bias"], torch.float32, "cuda") if "sel_bias" in host else None
+    off = (to_device(host["logit_offset"], torch.float32, "cuda")
+           if "logit_offset" in host else None)
+    idx = torch.empty((shape.T, shape.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.top_k), dtype=torch.float32, device="cuda")
+    B.moe_router_topk(cfg, x, wr, bias, off, idx, w, ws)
+    torch.cuda.synchronize()
+    P.check_routing(_np(idx), _np(w), P.oracle_routing(shape, host))
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3_small", "skew_small"])
+def test_permute_call_bit_exact(name):
+    """Oracle routing in, dispatch out: counts, offsets, slots, rows bit-exact."""
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    r = P.oracle_routing(shape, host)
+    ref = O.dispatch(r.topk_idx, shape.n_experts)
+    cfg, ws = _buffers(shape)
+    dt = torch.bfloat16 if shape.dtype == I.DTYPE_BF16 else torch.float32
+    T, k, E, d = shape.T, shape.top_k, shape.n_experts, shape.d_model
+    x = to_device(host["x"], dt, "cuda")
+    idx = torch.from_numpy(r.topk_idx.astype(np.int32)).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    slot = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    src = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((T * k, d), dtype=dt, device="cuda")
+    B.moe_permute(cfg, idx, x, counts, offsets, slot, src, xp, ws)
+    assert B.moe_device_status(ws)[0] == B.MOE_OK
+    np.testing.assert_array_equal(_np(counts), ref.counts)
+    np.testing.assert_array_equal(_np(offsets), ref.offsets)
+    np.testing.assert_array_equal(_np(slot), ref.slot_pos)
+    np.testing.assert_array_equal(_np(src), ref.perm_src)
+    np.testing.assert_array_equal(_np(xp), host["x"][ref.perm_src])
+
+
+def test_permute_skips_and_reports_bad_ids():
+    shape = SMALL["qwen3_small"].replace(T=300)
+    host = I.make_inputs(shape)
+    r = P.oracle_routing(shape, host)
+    bad = r.topk_idx.astype(np.int32).copy()
+    bad[5, 2] = -3                       # out of range
+    bad[17, 0] = shape.n_experts         # out of range
+    bad[40, 3] = bad[40, 1]              # repeated within the token
+    cfg, ws = _buffers(shape)
+    T, k, E, d = shape.T, shape.top_k, shape.n_experts, shape.d_model
+    x = to_device(host["x"], torch.bfloat16, "cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    slot = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    src = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    xp = torch.empty((T * k, d), dtype=torch.bfloat16, device="cuda")
+    B.moe_permute(cfg, torch.from_numpy(bad).cuda(), x, counts, offsets, slot, src, xp, ws)
+    st, flags = B.moe_device_status(ws)
+    assert st == B.MOE_ERR_DATA and flags & 1
+    s = _np(slot)
+    assert s[5, 2] == -1 and s[17, 0] == -1 and s[40, 3] == -1
+    valid = s >= 0
+    assert int(_np(offsets)[-1]) == valid.sum() == T * k - 3
+    # the valid pairs keep the stable (expert, token) order
+    e_of = bad.reshape(-1)[valid.reshape(-1)]
+    t_of = np.repeat(np.arange(T), k)[valid.reshape(-1)]
+    order = np.lexsort((t_of, e_of))
+    np.testing.assert_array_equal(np.sort(s[valid]), np.arange(valid.sum()))
+    np.testing.assert_array_equal(s.reshape(-1)[valid.reshape(-1)][order], np.arange(valid.sum()))
+
+
+@pytest.mark.parametrize("name", ["tiny", "page2_small", "wide_small"])
+def test_grouped_swiglu_call(name):
+    """Oracle dispatch in; every expert row against the oracle's expert."""
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    r = P.oracle_routing(shape, host)
+    dp = O.dispatch(r.topk_idx, shape.n_experts)
+    cfg, ws = _buffers(shape)
+    dt = torch.bfloat16 if shape.dtype == I.DTYPE_BF16 else torch.float32
+    T, k, d = shape.T, shape.top_k, shape.d_model
+    xp = to_device(host["x"][dp.perm_src], dt, "cuda")
+    offs = torch.from_numpy(dp.offsets.astype(np.int32)).cuda()
+    wts = {key: to_device(host[key], dt, "cuda") for key in ("w1", "w3", "w2", "ws1", "ws3", "ws2")
+           if key in host}
+    x = to_device(host["x"], dt, "cuda")
+    yp = torch.empty((T * k, d), dtype=dt, device="cuda")
+    ysh = torch.empty((T, d), dtype=dt, device="cuda") if shape.n_shared else None
+    B.moe_grouped_swiglu(cfg, xp, offs, wts, x if shape.n_shared else None, yp, ysh, ws)
+    assert B.moe_device_status(ws)[0] == B.MOE_OK
+    ref = np.concatenate([
+        O.swiglu_expert(host["x"][dp.perm_src[dp.offsets[e]:dp.offsets[e + 1]]],
+                        host["w1"][e], host["w3"][e], host["w2"][e])
+        for e in range(shape.n_experts)])
+    assert P.rel_err(_np(yp), ref) <= _tol(shape)
+    if shape.n_shared:
+        ref_sh = O.swiglu_expert(host["x"], host["ws1"], host["ws3"], host["ws2"])
+        assert P.rel_err(_np(ysh), ref_sh) <= _tol(shape)
+
+
+@pytest.mark.parametrize("bf16,shared", [(True, True), (True, False), (False, False)])
+def test_combine_call(bf16, shared):
+    rng = np.random.default_rng(5)
+    T, k, d = 333, 3, 256
+    R = T * k
+    dt = torch.bfloat16 if bf16 else torch.float32
+    y = I.round_to_bf16(rng.standard_normal((R, d)).astype(np.float32)) if bf16 else \
+        rng.standard_normal((R, d)).astype(np.float32)
+    ysh = I.round_to_bf16(rng.standard_normal((T, d)).astype(np.float32)) if shared else None
+    slot = rng.permutation(R).reshape(T, k).astype(np.int32)
+    slot[7, 1] = -1
+    w = rng.uniform(0, 1, (T, k)).astype(np.float32)
+    cfg = B.make_config(T, d, 8, 128, k, 1 if shared else 0, 128,
+                        dtype=B.DTYPE_BF16 if bf16 else B.DTYPE_F32)
+    out = torch.empty((T, d), dtype=dt, device="cuda")
+    B.moe_combine(cfg, to_device(y, dt, "cuda"), torch.from_numpy(slot).cuda(),
+                  torch.from_numpy(w).cuda(), to_device(ysh, dt, "cuda") if shared else None, out)
+    torch.cuda.synchronize()
+    ref = O.combine(y, slot, w, ysh)
+    assert P.rel_err(_np(out), ref) <= (4e-3 if bf16 else 1e-6)
+
+
+@pytest.mark.parametrize("E", [4, 16, 64, 128])
+def test_bias_update_call_bit_exact(E):
+    rng = np.random.default_rng(E)
+    for trial in range(4):
+        counts = rng.integers(0, 3000, E).astype(np.int32)
+        counts[rng.integers(0, E, 2)] = 0
+        bias = rng.uniform(-9.99, 9.99, E).astype(np.float32)
+        if trial == 3:
+            bias[:] = 9.9995   # saturation path
+        cfg = B.make_config(16, 128, E, 128, 1)
+        c_d = torch.from_numpy(counts).cuda()
+        b_d = torch.from_numpy(bias.copy()).cuda()
+        rate = [1e-3, 0.37, 1e-3, 1.0][trial]
+        B.moe_bias_update(cfg, c_d, b_d, rate, 0.1, 0.5, 10.0)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(_np(b_d), O.bias_update(counts, bias, rate, 0.1, 0.5, 10.0))

@@ -325,6 +325,25 @@ def test_dispatch_matches_bucket_loop():
     assert sorted(dp.slot_pos.reshape(-1).tolist()) == list(range(T * k))
 
 
+def test_combine_unpermutes_the_sorted_evaluation():
+    """Routed outputs computed per expert in sorted row order, combined through
+    slot_pos, equal the layer output; a one-hot k=1 combine is a row gather."""
+    rng = np.random.default_rng(15)
+    inp = _random_layer(rng, 40, 10, 5, 6, 2, shared=True, bias=True)
+    out, r = O.moe_forward(inp, 2, O.GATE_SIGMOID, True)
+    dp = O.dispatch(r.topk_idx, 5)
+    y_perm = np.concatenate([
+        O.swiglu_expert(inp["x"][dp.perm_src[dp.offsets[e]:dp.offsets[e + 1]]],
+                        inp["w1"][e], inp["w3"][e], inp["w2"][e]) for e in range(5)])
+    y_sh = O.swiglu_expert(inp["x"], inp["ws1"], inp["ws3"], inp["ws2"])
+    np.testing.assert_allclose(O.combine(y_perm, dp.slot_pos, r.topk_w, y_sh), out,
+                               rtol=1e-12, atol=1e-12)
+    y = rng.standard_normal((7, 3))
+    sp = np.array([[3], [0], [-1], [6]])
+    g = O.combine(y, sp, np.ones((4, 1)))
+    np.testing.assert_array_equal(g, np.stack([y[3], y[0], np.zeros(3), y[6]]))
+
+
 def test_dispatch_rejects_bad_index():
     with pytest.raises(ValueError):
         O.dispatch(np.array([[0, 4]]), 4)
