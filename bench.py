@@ -240,6 +240,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
     from mixture_experts_ffn_bias_b200 import binding as B
+    from mixture_experts_ffn_bias_b200.dp import allreduce_counts
     from mixture_experts_ffn_bias_b200.layer import MoELayer
 
     torch.cuda.set_device(local_rank)
@@ -260,8 +261,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
             B.moe_forward_profiled(layer.cfg, layer.x if x is None else x, layer.w_router,
                                    layer.sel_bias, layer.logit_offset, layer.weights, layer.out,
                                    layer.topk_idx, layer.topk_w, layer.counts, layer.ws, evs)
-        if world > 1:
-            dist.all_reduce(layer.counts)
+        allreduce_counts(layer.counts)
         layer.bias_update()
 
     def barrier():
@@ -364,6 +364,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=I.WORKLOAD_ORDER, default="qwen3_30b")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (smaller cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -372,6 +374,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     shape = I.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        shape = shape.replace(T=args.tokens)
     if args.impl == "reference":
         run_reference(args, shape, rank, world)
         return

@@ -198,6 +198,9 @@ def moe_forward_profiled(cfg, x, w_router, sel_bias, logit_offset, weights: Dict
                          topk_w, counts, ws, events, stream=None, check=True) -> int:
     """``events``: FORWARD_PHASES + 1 torch.cuda.Event objects (timing enabled)."""
     w = expert_weights(weights)
+    for e in events:
+        if e.cuda_event == 0:      # torch creates the CUDA event on first record
+            e.record()
     arr = (ctypes.c_void_p * (FORWARD_PHASES + 1))(*[e.cuda_event for e in events])
     st = lib().moe_forward_profiled(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
                                     _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),

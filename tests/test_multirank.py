@@ -1,0 +1,86 @@
+"""World-size-2 gloo test of the data-parallel exchange (CPU, no GPU).
+
+Each rank routes its own token shard (the oracle stands in for the GPU
+forward, which cannot run here), sums counts with the same helper the
+benchmark uses, and applies the bias update.  Both ranks must end with the
+same bias, equal to the single-process update from the whole batch; without
+the all-reduce the replicas drift apart (the failure the page-2 README warns
+about)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from mixture_experts_ffn_bias_b200 import inputs as I
+from mixture_experts_ffn_bias_b200.dp import allreduce_counts
+from oracle import moe_oracle as O
+
+SHAPE = I.WORKLOADS["skew"].replace(T=1024, d_model=128, d_ff=128, d_ff_shared=128)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _local_counts(rank, world, host):
+    lo, hi = rank * SHAPE.T // world, (rank + 1) * SHAPE.T // world
+    r = O.router(host["x"][lo:hi], host["w_router"], SHAPE.top_k, SHAPE.gate, True,
+                 host["sel_bias"], host["logit_offset"])
+    return O.dispatch(r.topk_idx, SHAPE.n_experts).counts
+
+
+def _worker(rank, world, port, q, do_allreduce):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        host = I.make_inputs(SHAPE)
+        c = torch.from_numpy(_local_counts(rank, world, host).astype(np.int32))
+        if do_allreduce:
+            allreduce_counts(c)
+        bias = O.bias_update(c.numpy(), host["sel_bias"])
+        q.put((rank, c.numpy().tolist(), bias.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(world, do_allreduce):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, do_allreduce))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict((r, (c, b)) for r, c, b in (q.get(timeout=120) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return res
+
+
+def test_counts_allreduce_keeps_replicas_identical():
+    res = _run(2, True)
+    host = I.make_inputs(SHAPE)
+    full = _local_counts(0, 1, host)
+    ref_bias = O.bias_update(full, host["sel_bias"])
+    for r in (0, 1):
+        assert res[r][0] == full.tolist()
+        np.testing.assert_array_equal(np.array(res[r][1], np.float32), ref_bias)
+
+
+def test_without_allreduce_replicas_drift():
+    res = _run(2, False)
+    assert res[0][1] != res[1][1]
+
+
+def test_single_process_is_a_noop():
+    c = torch.arange(5, dtype=torch.int32)
+    assert allreduce_counts(c).tolist() == [0, 1, 2, 3, 4]
