@@ -196,6 +196,32 @@ moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void
                                 void* ws, size_t ws_bytes, void* stream,
                                 void* const* events);
 
+/* moe_permute without a workspace, for callers that cannot allocate device
+ * memory: a host program that links only this library and has no device
+ * allocator, or a serving loop on a fixed memory plan that must not call
+ * cudaMalloc/cudaFree once running (they synchronise the device and can fail
+ * when memory is fragmented).  The pages have no counterpart; this is a
+ * deployment variant of the dispatch call above, with the same arguments
+ * minus ws/ws_bytes and the same outputs.
+ *   Scratch: a fixed array of MOE_PERMUTE_NOALLOC_MAX_BLOCK_COUNTS int32 block
+ *   counts (+256 B for a status word) in the library's own device memory,
+ *   one copy per GPU that loads the library, held until the process exits.
+ *   Limit: ceil(T/256) * E <= MOE_PERMUTE_NOALLOC_MAX_BLOCK_COUNTS (e.g.
+ *   T <= 524288 at E = 128); larger calls return MOE_ERR_WORKSPACE without
+ *   launching anything.
+ *   The first call on a device looks up that device's copy of the array
+ *   (cudaGetSymbolAddress, with the device current); make that first call
+ *   before any stream capture.  The call allocates nothing.
+ *   Every call shares the one array and leaves its contents behind; calls
+ *   whose work overlaps on the GPU (other streams, other threads) race on it
+ *   and must be serialised by the caller.  Pairs with an invalid or repeated
+ *   expert id are skipped (slot_pos -1, offsets[E] < T*k); there is no
+ *   workspace, so moe_device_status cannot report them. */
+#define MOE_PERMUTE_NOALLOC_MAX_BLOCK_COUNTS 262144
+moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, const void* x,
+                               int32_t* counts, int32_t* offsets, int32_t* slot_pos,
+                               int32_t* perm_src, void* x_perm, void* stream);
+
 /* Synchronise `stream`, read and clear the device status word in ws.
  * Returns MOE_OK, MOE_ERR_DATA, MOE_ERR_TIMEOUT or MOE_ERR_CUDA; the raw
  * flag bits are stored in *flags when flags is not NULL. */

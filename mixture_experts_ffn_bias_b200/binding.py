@@ -27,6 +27,7 @@ MOE_ERR_DATA = 6
 
 GATE_SOFTMAX = 0
 GATE_SIGMOID = 1
+NOALLOC_MAX_BLOCK_COUNTS = 262144   # MOE_PERMUTE_NOALLOC_MAX_BLOCK_COUNTS in moe.h
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 
@@ -61,6 +62,7 @@ _SIGNATURES = {
     "moe_forward": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_forward_profiled": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ,
                                      _VP, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_permute_noalloc": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_device_status": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
 }
@@ -156,6 +158,15 @@ def moe_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src, x_perm, w
     st = lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts), _p(offsets),
                            _p(slot_pos), _p(perm_src), _p(x_perm), _p(ws),
                            _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_permute_noalloc(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src, x_perm,
+                        stream=None, check=True) -> int:
+    """moe_permute with its scratch in the library's fixed device array (no workspace)."""
+    st = lib().moe_permute_noalloc(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts),
+                                   _p(offsets), _p(slot_pos), _p(perm_src), _p(x_perm),
+                                   _s(stream))
     return _check(st, check)
 
 
