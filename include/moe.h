@@ -118,6 +118,14 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
                            int32_t* topk_idx, float* topk_w,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Router GEMM alone: logits [T, E] fp32 = x . w_router^T (+ logit_offset),
+ * for bf16 layers (fp32 layers return MOE_ERR_UNSUPPORTED).  Tensor cores,
+ * exact bf16 products, fp32 accumulation: these are the logits moe_router_topk
+ * selects from before it re-decides near ties on exact logits. */
+moe_status moe_router_logits(const moe_config* cfg, const void* x, const void* w_router,
+                             const float* logit_offset, float* logits,
+                             void* ws, size_t ws_bytes, void* stream);
+
 /* Dispatch: per-expert counts, offsets, and the stable expert-contiguous
  * permutation of the T*k routed rows, with x gathered into that order.
  * (Grouped-GEMM dispatch, SpecForge PR #930 "Why FSDP is enough here" and

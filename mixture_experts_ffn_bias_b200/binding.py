@@ -55,6 +55,7 @@ _SIGNATURES = {
     "moe_workspace_size": (_SZ, [_CFG]),
     "moe_check_config": (_I32, [_CFG]),
     "moe_router_topk": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_router_logits": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_swiglu": (_I32, [_CFG, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP]),
@@ -150,6 +151,13 @@ def moe_router_topk(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, 
     st = lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
                                _p(logit_offset), _p(topk_idx), _p(topk_w), _p(ws),
                                _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_router_logits(cfg, x, w_router, logit_offset, logits, ws, stream=None, check=True) -> int:
+    st = lib().moe_router_logits(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_offset),
+                                 _p(logits), _p(ws), _nbytes(ws) if ws is not None else 0,
+                                 _s(stream))
     return _check(st, check)
 
 

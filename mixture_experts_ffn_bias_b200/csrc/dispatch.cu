@@ -80,17 +80,30 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
   }
 }
 
+// Block counts [nblk, E] -> block bases (in place), counts and offsets.  The
+// counts are staged in shared memory when they fit (kScanSmemInts), so the
+// per-expert running sums walk shared memory instead of global memory.
+constexpr int kScanSmemInts = 11776;   // 46 KB + the 1 KB scan array stay under 48 KB
+
 __global__ void __launch_bounds__(kMaxE)
 dispatch_scan_kernel(int32_t* __restrict__ blk, int nblk, int E, int32_t* __restrict__ counts,
                      int32_t* __restrict__ offsets) {
   __shared__ int s[kMaxE];
+  __shared__ int sblk[kScanSmemInts];
   const int e = threadIdx.x;
+  const int n = nblk * E;
+  const bool staged = n <= kScanSmemInts;
+  int32_t* col = staged ? sblk : blk;
+  if (staged) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) sblk[i] = blk[i];
+    __syncthreads();
+  }
   int run = 0;
   if (e < E) {
 #pragma unroll 8
     for (int b = 0; b < nblk; ++b) {
-      const int c = blk[static_cast<size_t>(b) * E + e];
-      blk[static_cast<size_t>(b) * E + e] = run;
+      const int c = col[static_cast<size_t>(b) * E + e];
+      col[static_cast<size_t>(b) * E + e] = run;
       run += c;
     }
     counts[e] = run;
@@ -106,7 +119,11 @@ dispatch_scan_kernel(int32_t* __restrict__ blk, int nblk, int E, int32_t* __rest
   const int excl = s[e] - ((e < E) ? run : 0);
   if (e < E) offsets[e] = excl;
   if (e == kMaxE - 1) offsets[E] = s[e];
-  if (e < E) {
+  if (staged) {
+    s[e] = excl;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) blk[i] = sblk[i] + s[i % E];
+  } else if (e < E) {
 #pragma unroll 8
     for (int b = 0; b < nblk; ++b) blk[static_cast<size_t>(b) * E + e] += excl;
   }

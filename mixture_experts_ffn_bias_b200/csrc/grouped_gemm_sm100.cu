@@ -50,14 +50,18 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*bars*/;
 };
 
+// Epilogue modes.
+constexpr int MODE_PLAIN_BF16 = 0;    // C = A B^T, rounded to bf16
+constexpr int MODE_SWIGLU_BF16 = 1;   // C = silu(A B0^T) * (A B1^T), rounded to bf16
+
 struct GemmArgs {
   const int32_t* offsets;  // [G+1] device, or nullptr: one group [0, rows_single)
   int num_groups;
   int rows_single;
   int n_per_group;         // output columns per group (= B rows per group)
   int K;
-  __nv_bfloat16* C;
-  int ldc;
+  void* C;
+  int ldc;                 // elements
   uint32_t* status;
 };
 
@@ -117,7 +121,7 @@ __device__ __forceinline__ int find_group(const int* s_prefix, int G, int tile) 
   return lo;
 }
 
-template <int BN_ACC, bool SWIGLU>
+template <int BN_ACC, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -125,6 +129,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const GemmArgs args) {
   using Cfg = GemmCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
   constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN_ACC);
 
@@ -285,8 +290,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const int n = local - m * n_tiles;
       const int rows_g = s_off[g + 1] - s_off[g];
       const bool valid = (m * BM + row) < rows_g;
-      __nv_bfloat16* crow = args.C + static_cast<size_t>(s_off[g] + m * BM + row) * args.ldc +
-                            static_cast<size_t>(n) * BN_OUT;
+      const size_t crow_off = static_cast<size_t>(s_off[g] + m * BM + row) * args.ldc +
+                              static_cast<size_t>(n) * BN_OUT;
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN_OUT / 16; ++c) {
@@ -311,7 +316,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + c * 16);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
+                                                c * 16);
           dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
           dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
         }
@@ -373,12 +379,12 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int BN_ACC, bool SWIGLU>
+template <int BN_ACC, int MODE>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                    const GemmArgs& args, int rows_upper, cudaStream_t stream) {
   using Cfg = GemmCfg<BN_ACC>;
-  constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
-  auto kern = grouped_gemm_kernel<BN_ACC, SWIGLU>;
+  constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
+  auto kern = grouped_gemm_kernel<BN_ACC, MODE>;
   static unsigned long long attr_done = 0;   // one bit per device (attribute is per device)
   int dev = 0;
   cudaGetDevice(&dev);
@@ -410,10 +416,9 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
       !make_map(&tb1, W3, b_rows, K, 128))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, F, K,
-                static_cast<__nv_bfloat16*>(H), F, status};
+  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  return launch<256, true>(ta, tb0, tb1, args, rows_upper, stream);
+  return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, args, rows_upper, stream);
 }
 
 // Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.
@@ -425,11 +430,11 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   const int bn = (N % 256 == 0) ? 256 : 128;
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, N, K,
-                static_cast<__nv_bfloat16*>(Y), N, status};
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  if (bn == 256) return launch<256, false>(ta, tb, tb, args, rows_upper, stream);
-  return launch<128, false>(ta, tb, tb, args, rows_upper, stream);
+  if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, args, rows_upper, stream);
+  return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, args, rows_upper, stream);
 }
+
 
 }  // namespace moe

@@ -21,6 +21,22 @@ cudaError_t router_select(const double* logits, const float* sel_bias, int T, in
                           int gate, int renorm, int32_t* topk_idx, float* topk_w,
                           cudaStream_t stream);
 
+// bf16 router: tensor-core fp32 logits, fast selection with near-tie
+// flagging, exact fp64 re-decision of the flagged tokens.
+cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
+                             float* logits, uint32_t* status, cudaStream_t stream);
+cudaError_t router_select_fast(const float* logits, const float* logit_offset,
+                               const float* sel_bias, int T, int E, int k, int gate, int renorm,
+                               int32_t* topk_idx, float* topk_w, int32_t* refine_count,
+                               int32_t* refine_list, cudaStream_t stream);
+cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
+                          const float* sel_bias, int T, int d, int E, int k, int gate,
+                          int renorm, const int32_t* refine_count, const int32_t* refine_list,
+                          int32_t* topk_idx, float* topk_w, int grid, cudaStream_t stream);
+
+// logits[t, e] += offset[e]
+cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream);
+
 // Dispatch -------------------------------------------------------------------
 constexpr int kRankBlock = 256;   // tokens per histogram block
 inline int rank_blocks(int T) { return (T + kRankBlock - 1) / kRankBlock; }

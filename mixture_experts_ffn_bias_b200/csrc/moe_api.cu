@@ -15,7 +15,8 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
-  size_t status, blk, offsets, slot_pos, perm_src, logits, x_perm, h, y_perm, h_sh, y_sh, total;
+  size_t status, blk, offsets, slot_pos, perm_src, refine, logits, x_perm, h, y_perm, h_sh, y_sh,
+      total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -31,6 +32,7 @@ Layout layout(const moe_config& c) {
   L.offsets = o;  o += up((E + 1) * 4);
   L.slot_pos = o; o += up(R * 4);
   L.perm_src = o; o += up(R * 4);
+  L.refine = o;   o += up(T * 4);
   L.logits = o;   o += up(T * E * 8);
   L.x_perm = o;   o += up(R * d * es);
   L.h = o;        o += up(R * F * es);
@@ -83,9 +85,18 @@ inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
     if ((expr) != cudaSuccess) return MOE_ERR_CUDA;     \
   } while (0)
 
+// Word 0: device status flags; word 1: number of tokens the router listed
+// for exact re-decision.
 moe_status clear_status(void* ws, cudaStream_t s) {
-  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, sizeof(uint32_t), s));
+  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, 2 * sizeof(uint32_t), s));
   return MOE_OK;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 // Router into caller buffers; logits scratch in ws.
@@ -93,9 +104,22 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
                       const float* sel_bias, const float* logit_offset, int32_t* topk_idx,
                       float* topk_w, void* ws, cudaStream_t s) {
   const Layout L = layout(*c);
+  if (c->dtype == MOE_BF16) {
+    float* logits = at<float>(ws, L.logits);
+    int32_t* count = at<int32_t>(ws, L.status) + 1;
+    int32_t* list = at<int32_t>(ws, L.refine);
+    MOE_TRY(moe::router_logits_tc(x, c->T, w_router, c->n_experts, c->d_model, logits,
+                                  at<uint32_t>(ws, L.status), s));
+    MOE_TRY(moe::router_select_fast(logits, logit_offset, sel_bias, c->T, c->n_experts, c->top_k,
+                                    c->gate, c->norm_topk_prob, topk_idx, topk_w, count, list, s));
+    MOE_TRY(moe::router_refine(x, w_router, logit_offset, sel_bias, c->T, c->d_model,
+                               c->n_experts, c->top_k, c->gate, c->norm_topk_prob, count, list,
+                               topk_idx, topk_w, device_sms(), s));
+    return MOE_OK;
+  }
   double* logits = at<double>(ws, L.logits);
-  MOE_TRY(moe::router_logits(c->dtype == MOE_BF16, x, w_router, logit_offset, c->T, c->d_model,
-                             c->n_experts, logits, s));
+  MOE_TRY(moe::router_logits(false, x, w_router, logit_offset, c->T, c->d_model, c->n_experts,
+                             logits, s));
   MOE_TRY(moe::router_select(logits, sel_bias, c->T, c->n_experts, c->top_k, c->gate,
                              c->norm_topk_prob, topk_idx, topk_w, s));
   return MOE_OK;
@@ -252,6 +276,25 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
   if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
   if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
   return run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, S(stream));
+}
+
+moe_status moe_router_logits(const moe_config* cfg, const void* x, const void* w_router,
+                             const float* logit_offset, float* logits, void* ws,
+                             size_t ws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !logits || !aligned16(x) || !aligned16(w_router) || !aligned4(logits) ||
+      (logit_offset && !aligned4(logit_offset)))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
+  MOE_TRY(moe::router_logits_tc(x, cfg->T, w_router, cfg->n_experts, cfg->d_model, logits,
+                                at<uint32_t>(ws, 0), S(stream)));
+  if (logit_offset)
+    MOE_TRY(moe::add_row_offset(logits, logit_offset, cfg->T, cfg->n_experts, S(stream)));
+  return MOE_OK;
 }
 
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,

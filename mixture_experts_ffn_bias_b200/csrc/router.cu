@@ -6,11 +6,19 @@
 // divided by their sum + 1e-9) and the qwen3 preset of SpecForge PR #930
 // (softmax over all experts, top-k weights renormalised).
 //
-// Precision: x and w_router hold bf16 (or fp32) values.  Products are formed
-// in fp32 (exact for bf16 x bf16), summed in fp32 over 32-wide K chunks and the
-// chunk sums are added in fp64, so a logit is within ~1e-8 of the exact dot
-// product for the layer sizes used here.  Selection keys, gate scores and the
-// renormalisation are then evaluated in fp64 and the weights stored as fp32.
+// bf16 layers (the production path):
+//   1. logits = x . Wr^T on the tensor cores (router_logits_tc in
+//      grouped_gemm_sm100.cu): exact bf16 x bf16 products, fp32 accumulation.
+//   2. router_select_fast_kernel: one warp per token, fp32 keys and gate;
+//      a token whose k-th / (k+1)-th keys, or two adjacent keys inside its
+//      top-k, are closer than kRefineMargin is not decided here but appended
+//      to a refine list.
+//   3. router_refine_kernel: for each listed token, exact logits (fp64 sums of
+//      exact products) and the selection and weights in fp64.
+//   The fp32 accumulation error of a logit is orders of magnitude below the
+//   margin, so every token's decision equals the one taken on exact logits.
+// fp32 layers: logits on CUDA cores (fp32 products summed in fp32 over
+// 32-wide K chunks, chunk sums added in fp64), selection in fp64.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -27,7 +35,9 @@ __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162flo
 constexpr int RT_TOK = 64;    // tokens per block
 constexpr int RT_EXP = 32;    // experts per block
 constexpr int RT_KC = 32;     // K chunk accumulated in fp32
+constexpr int kMaxPerLane = 8;   // E <= 256 = 8 x 32
 
+// ---------------------------------------------------------------- fp32 layers
 template <typename Tin>
 __global__ void __launch_bounds__(256)
 router_logits_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
@@ -98,32 +108,21 @@ router_logits_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
   }
 }
 
-constexpr int kMaxPerLane = 8;   // E <= 256 = 8 x 32
-
-// One warp per token.  Lane l holds experts l, l+32, ...
-__global__ void __launch_bounds__(256)
-router_select_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T,
-                     int E, int k, int gate, int renorm, int32_t* __restrict__ topk_idx,
-                     float* __restrict__ topk_w) {
+// Selection, gate and weights for one token in fp64, done by one warp.  `l`
+// holds the logits of experts lane + 32 i (offset already added).
+__device__ void warp_select_fp64(const double (&l)[kMaxPerLane], const float* __restrict__ bias,
+                                 int E, int k, int gate, int renorm,
+                                 int32_t* __restrict__ idx_row, float* __restrict__ w_row) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  double l[kMaxPerLane], key[kMaxPerLane], s[kMaxPerLane];
+  double key[kMaxPerLane], s[kMaxPerLane];
   bool taken[kMaxPerLane];
   double lmax = -INFINITY;
 #pragma unroll
   for (int i = 0; i < kMaxPerLane; ++i) {
     const int e = lane + 32 * i;
-    if (e < E) {
-      l[i] = logits[static_cast<size_t>(t) * E + e];
-      key[i] = l[i] + (bias ? static_cast<double>(bias[e]) : 0.0);
-      taken[i] = false;
-      lmax = fmax(lmax, l[i]);
-    } else {
-      l[i] = -INFINITY;
-      key[i] = -INFINITY;
-      taken[i] = true;
-    }
+    taken[i] = e >= E;
+    key[i] = e < E ? l[i] + (bias ? static_cast<double>(bias[e]) : 0.0) : -INFINITY;
+    if (e < E) lmax = fmax(lmax, l[i]);
   }
   if (gate == 1) {  // sigmoid
 #pragma unroll
@@ -142,7 +141,6 @@ router_select_kernel(const double* __restrict__ logits, const float* __restrict_
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i) s[i] = s[i] / sum;
   }
-
   int my_idx = 0;
   double my_w = 0.0, wsum = 0.0;
   for (int j = 0; j < k; ++j) {
@@ -183,12 +181,205 @@ router_select_kernel(const double* __restrict__ logits, const float* __restrict_
   }
   if (renorm) my_w = my_w / (wsum + 1e-9);
   if (lane < k) {
-    topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
-    topk_w[static_cast<size_t>(t) * k + lane] = static_cast<float>(my_w);
+    idx_row[lane] = my_idx;
+    w_row[lane] = static_cast<float>(my_w);
   }
 }
 
+// One warp per token, fp64 logits.
+__global__ void __launch_bounds__(256)
+router_select_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T,
+                     int E, int k, int gate, int renorm, int32_t* __restrict__ topk_idx,
+                     float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  double l[kMaxPerLane];
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    l[i] = e < E ? logits[static_cast<size_t>(t) * E + e] : -INFINITY;
+  }
+  warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
+                   topk_w + static_cast<size_t>(t) * k);
+}
+
+// ---------------------------------------------------------------- bf16 layers
+// Keys closer than this are re-decided on exact logits.  The fp32 tensor-core
+// accumulation error of a logit is ~1e-6 at d = 5120 (bf16 products are
+// exact; the error is the rounding of the running fp32 sum), and the fp32
+// keys add ~5e-7, so 1e-4 leaves a wide safety factor.
+constexpr float kRefineMargin = 1e-4f;
+
+// One warp per token, fp32 logits from the tensor cores.
+__global__ void __launch_bounds__(256)
+router_select_fast_kernel(const float* __restrict__ logits, const float* __restrict__ offset,
+                          const float* __restrict__ bias, int T, int E, int k, int gate,
+                          int renorm, int32_t* __restrict__ topk_idx,
+                          float* __restrict__ topk_w, int32_t* __restrict__ refine_count,
+                          int32_t* __restrict__ refine_list) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float l[kMaxPerLane], key[kMaxPerLane];
+  bool taken[kMaxPerLane];
+  float lmax = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      l[i] = logits[static_cast<size_t>(t) * E + e] + (offset ? offset[e] : 0.0f);
+      key[i] = l[i] + (bias ? bias[e] : 0.0f);
+      taken[i] = false;
+      lmax = fmaxf(lmax, l[i]);
+    } else {
+      l[i] = -INFINITY;
+      key[i] = -INFINITY;
+      taken[i] = true;
+    }
+  }
+  // top-(k+1) keys, descending, ties -> lower expert id
+  const int rounds = k < E ? k + 1 : k;
+  float prev = 0.f, min_gap = INFINITY, edge_gap = INFINITY;
+  int my_idx = 0;
+  float my_l = 0.f;
+  for (int j = 0; j < rounds; ++j) {
+    float bk = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      const int e = lane + 32 * i;
+      if (!taken[i] && (key[i] > bk || (key[i] == bk && e < be))) {
+        bk = key[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    const int owner = be & 31, slot = be >> 5;
+    float lsel = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+      if (lane == owner && i == slot) {
+        taken[i] = true;
+        lsel = l[i];
+      }
+    }
+    lsel = __shfl_sync(0xffffffffu, lsel, owner);
+    if (j > 0) {
+      const float gap = prev - bk;
+      if (j < k) min_gap = fminf(min_gap, gap);
+      else edge_gap = gap;
+    }
+    prev = bk;
+    if (lane == j && j < k) {
+      my_idx = be;
+      my_l = lsel;
+    }
+  }
+  if (fminf(min_gap, edge_gap) < kRefineMargin) {
+    if (lane == 0) refine_list[atomicAdd(refine_count, 1)] = t;
+    return;
+  }
+  // gate scores of the chosen experts and the weights
+  float s;
+  if (gate == 1) {
+    s = 1.0f / (1.0f + expf(-my_l));
+  } else {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i)
+      if (lane + 32 * i < E) sum += expf(l[i] - lmax);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    s = expf(my_l - lmax) / sum;
+  }
+  float ssum = lane < k ? s : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+  if (renorm) s = s / (ssum + 1e-9f);
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(t) * k + lane] = s;
+  }
+}
+
+// Exact re-decision of the listed tokens: fp64 sums of exact bf16 products,
+// then the fp64 selection.  Each block takes listed tokens round robin; the
+// experts' dot products are split over tpe threads each.
+__global__ void __launch_bounds__(256)
+router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+                     const float* __restrict__ offset, const float* __restrict__ bias, int d,
+                     int E, int k, int gate, int renorm, const int32_t* __restrict__ refine_count,
+                     const int32_t* __restrict__ refine_list, int32_t* __restrict__ topk_idx,
+                     float* __restrict__ topk_w) {
+  __shared__ double s_logit[256];
+  const int n = *refine_count;
+  int tpe = 1;
+  while (tpe < 32 && tpe * E * 2 <= 256) tpe *= 2;        // threads per expert
+  const int e = threadIdx.x / tpe, part = threadIdx.x % tpe;
+  const int vecs = d / 8;                                 // 16-byte vectors per row
+  for (int i = blockIdx.x; i < n; i += gridDim.x) {
+    const int t = refine_list[i];
+    double acc0 = 0.0, acc1 = 0.0;
+    if (e < E) {
+      const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+      const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * d);
+      for (int v = part; v < vecs; v += tpe) {
+        const uint4 a = __ldg(xr + v), b = __ldg(wrow + v);
+        const __nv_bfloat16* ah = reinterpret_cast<const __nv_bfloat16*>(&a);
+        const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&b);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          acc0 = fma(static_cast<double>(__bfloat162float(ah[j])),
+                     static_cast<double>(__bfloat162float(bh[j])), acc0);
+          acc1 = fma(static_cast<double>(__bfloat162float(ah[j + 1])),
+                     static_cast<double>(__bfloat162float(bh[j + 1])), acc1);
+        }
+      }
+    }
+    double acc = acc0 + acc1;
+    for (int o = tpe / 2; o > 0; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o, tpe);
+    if (e < E && part == 0) s_logit[e] = acc + (offset ? static_cast<double>(offset[e]) : 0.0);
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      double l[kMaxPerLane];
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) {
+        const int ee = threadIdx.x + 32 * j;
+        l[j] = ee < E ? s_logit[ee] : -INFINITY;
+      }
+      warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
+                       topk_w + static_cast<size_t>(t) * k);
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void add_row_offset_kernel(float* __restrict__ logits, const float* __restrict__ off,
+                                      long long n, int E) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    logits[i] += off[i % E];
+}
+
 }  // namespace
+
+cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream) {
+  const long long n = static_cast<long long>(T) * E;
+  const int grid = static_cast<int>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  add_row_offset_kernel<<<grid, 256, 0, stream>>>(logits, offset, n, E);
+  return cudaGetLastError();
+}
 
 cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
                           const float* logit_offset, int T, int d, int E, double* logits,
@@ -211,6 +402,29 @@ cudaError_t router_select(const double* logits, const float* sel_bias, int T, in
   const int warps = 8;
   router_select_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
       logits, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+cudaError_t router_select_fast(const float* logits, const float* logit_offset,
+                               const float* sel_bias, int T, int E, int k, int gate, int renorm,
+                               int32_t* topk_idx, float* topk_w, int32_t* refine_count,
+                               int32_t* refine_list, cudaStream_t stream) {
+  const int warps = 8;
+  router_select_fast_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
+      logits, logit_offset, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w, refine_count,
+      refine_list);
+  return cudaGetLastError();
+}
+
+cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
+                          const float* sel_bias, int T, int d, int E, int k, int gate,
+                          int renorm, const int32_t* refine_count, const int32_t* refine_list,
+                          int32_t* topk_idx, float* topk_w, int grid, cudaStream_t stream) {
+  if (grid > T) grid = T;
+  if (grid < 1) grid = 1;
+  router_refine_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
+      logit_offset, sel_bias, d, E, k, gate, renorm, refine_count, refine_list, topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,298 @@
+// Router logits on tcgen05 tensor cores with chunked accumulation.
+//
+// logits[t, e] = x[t] . Wr[e]  (the fp32 router linear of SigmoidRouter in
+// the "moe-200m-qwen3-100b" README, "Per-layer numerics": routing in fp32).
+//
+// bf16 x bf16 products are exact in fp32, so all the error of a tensor-core
+// logit is in the accumulation.  Accumulating the whole K (2048-5120) in one
+// TMEM accumulator gave errors up to ~1e-5 on unit-scale logits; here each
+// 128-wide K chunk is accumulated in a fresh TMEM slot (8 MMAs on a partial of
+// magnitude ~0.2) and the epilogue warps add the chunk partials into fp32
+// registers while the MMAs of the next chunks run.  This keeps the logit
+// error in the low 1e-6 range, far inside the router's re-decision margin.
+//
+// Warp roles (one 128-token tile at a time, persistent over tiles):
+//   warp 0        TMA: x tile 128 x 64 and Wr tile NPAD x 64 per stage
+//   warp 1        TMEM allocation, one lane issues tcgen05.mma into a ring of
+//                 NSLOT accumulator slots (one slot per K chunk)
+//   warps 2..     epilogue: one accumulator row per thread, NPAD <= 128
+//                 columns per warpgroup (two warpgroups for NPAD = 256)
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int RBM = 128;
+constexpr int RBK = 64;
+constexpr int KCH = 2;                       // k-blocks per accumulation chunk
+constexpr int R_A_BYTES = RBM * RBK * 2;
+
+template <int NPAD>
+struct RCfg {
+  static constexpr int EPI_WG = NPAD > 128 ? 2 : 1;
+  static constexpr int COLS = NPAD / EPI_WG;           // columns per epilogue thread
+  static constexpr int THREADS = 64 + 128 * EPI_WG;
+  static constexpr int B_BYTES = NPAD * RBK * 2;
+  static constexpr int STAGE_BYTES = R_A_BYTES + B_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int NSLOT = (512 / NPAD) > 8 ? 8 : (512 / NPAD);
+  static constexpr int TMEM_RAW = NSLOT * NPAD;
+  static constexpr int TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64
+                                   : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+};
+
+template <int NPAD>
+__global__ void __launch_bounds__(RCfg<NPAD>::THREADS, 1)
+router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 int T, int K, int E, float* __restrict__ logits, uint32_t* __restrict__ status) {
+  using C = RCfg<NPAD>;
+  constexpr uint32_t IDESC = idesc_bf16_f32(RBM, NPAD);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * R_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + C::STAGES;
+  uint64_t* sfull_bar = bars + 2 * C::STAGES;
+  uint64_t* sempty_bar = bars + 2 * C::STAGES + C::NSLOT;
+  uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = (T + RBM - 1) / RBM;
+  const int kblocks = K / RBK;
+  const int chunks = (kblocks + KCH - 1) / KCH;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(&sfull_bar[s], 1);
+      mbar_init(&sempty_bar[s], 4 * C::EPI_WG);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  volatile int* abort_flag = &s_abort;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+          tma_load_2d(sA + stage * R_A_BYTES, &tmX, &full_bar[stage], kb * RBK, tile * RBM);
+          tma_load_2d(sB + stage * C::B_BYTES, &tmW, &full_bar[stage], kb * RBK, 0);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < C::STAGES; ++s) {
+          if (!(issued_mask & (1u << s))) continue;
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full_bar[s], (issued_phase >> s) & 1u))
+            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0, cc = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        for (int ch = 0; ch < chunks && ok; ++ch, ++cc) {
+          const int slot = cc % C::NSLOT;
+          const uint32_t sph = (cc / C::NSLOT) & 1;
+          if (!mbar_wait(&sempty_bar[slot], sph ^ 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem + slot * NPAD;
+          const int kb_end = (ch + 1) * KCH < kblocks ? (ch + 1) * KCH : kblocks;
+          for (int kb = ch * KCH; kb < kb_end; ++kb) {
+            if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t a = smem_u32(sA + stage * R_A_BYTES);
+            const uint32_t b = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < RBK / 16; ++kk)
+              tc_mma_f16(d, smem_desc_sw128(a + kk * 32), smem_desc_sw128(b + kk * 32), IDESC,
+                         (kb > ch * KCH || kk > 0) ? 1u : 0u);
+            issued = true;
+            tc_commit(&empty_bar[stage]);
+            if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          tc_commit(&sfull_bar[slot]);
+        }
+      }
+      if (!ok && issued) {
+        tc_commit(drain_bar);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+  } else {
+    const int ew = warp - 2;                 // epilogue warp 0 .. 4*EPI_WG-1
+    const int wg = ew >> 2;                  // column half for NPAD = 256
+    const int q = warp & 3;                  // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;
+    int cc = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      float acc[C::COLS];
+#pragma unroll
+      for (int i = 0; i < C::COLS; ++i) acc[i] = 0.f;
+      for (int ch = 0; ch < chunks; ++ch, ++cc) {
+        const int slot = cc % C::NSLOT;
+        const uint32_t sph = (cc / C::NSLOT) & 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[slot], sph, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t taddr =
+            tmem + slot * NPAD + wg * C::COLS + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < C::COLS / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[c * 16 + i] += __uint_as_float(v[i]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty_bar[slot]);
+      }
+      if (!ok) break;
+      const int t = tile * RBM + row;
+      if (t < T) {
+        float* dst = logits + static_cast<size_t>(t) * E + wg * C::COLS;
+        const int ncol = E - wg * C::COLS;
+        if ((E & 3) == 0 && ncol >= C::COLS) {
+#pragma unroll
+          for (int i = 0; i < C::COLS; i += 4)
+            *reinterpret_cast<float4*>(dst + i) =
+                make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < C::COLS; ++i)
+            if (i < ncol) dst[i] = acc[i];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && s_abort) atomicOr(status, kDevTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool map2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(RBK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int NPAD>
+cudaError_t launch_router(const CUtensorMap& mx, const CUtensorMap& mw, int T, int K, int E,
+                          float* logits, uint32_t* status, cudaStream_t stream) {
+  using C = RCfg<NPAD>;
+  auto kern = router_tc_kernel<NPAD>;
+  static unsigned long long attr_done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_done & bit)) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done |= bit;
+  }
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int tiles = (T + RBM - 1) / RBM;
+  const int grid = tiles < sms ? tiles : (sms > 0 ? sms : 148);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mx, mw, T, K, E, logits, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
+                             float* logits, uint32_t* status, cudaStream_t stream) {
+  int npad = 16;
+  while (npad < E) npad *= 2;
+  if (npad > 256 || T <= 0) return T <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+  CUtensorMap mx, mw;
+  if (!map2d(&mx, x, T, K, RBM) || !map2d(&mw, w_router, E, K, npad))
+    return cudaErrorInvalidValue;
+  switch (npad) {
+    case 16: return launch_router<16>(mx, mw, T, K, E, logits, status, stream);
+    case 32: return launch_router<32>(mx, mw, T, K, E, logits, status, stream);
+    case 64: return launch_router<64>(mx, mw, T, K, E, logits, status, stream);
+    case 128: return launch_router<128>(mx, mw, T, K, E, logits, status, stream);
+    default: return launch_router<256>(mx, mw, T, K, E, logits, status, stream);
+  }
+}
+
+}  // namespace moe

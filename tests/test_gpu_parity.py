@@ -197,6 +197,25 @@ def test_router_topk_call(name):
     P.check_routing(_np(idx), _np(w), P.oracle_routing(shape, host))
 
 
+@pytest.mark.parametrize("name", FULL)
+def test_tensor_core_logit_error_is_far_below_the_refine_margin(name):
+    """The router decides from tensor-core fp32 logits and re-decides on exact
+    logits any token whose keys lie within 1e-4 of each other.  That is only
+    sound if the fp32 logits are much closer than 1e-4 to the exact ones;
+    measure it on every logit of the full workload."""
+    shape = I.WORKLOADS[name]
+    rng_host = I.make_inputs(shape)
+    cfg, ws = _buffers(shape)
+    x = to_device(rng_host["x"], torch.bfloat16, "cuda")
+    wr = to_device(rng_host["w_router"], torch.bfloat16, "cuda")
+    logits = torch.empty((shape.T, shape.n_experts), dtype=torch.float32, device="cuda")
+    B.moe_router_logits(cfg, x, wr, None, logits, ws)
+    torch.cuda.synchronize()
+    exact = rng_host["x"].astype(np.float64) @ rng_host["w_router"].astype(np.float64).T
+    err = float(np.max(np.abs(_np(logits) - exact)))
+    assert err < 5e-6, f"max |fp32 tensor-core logit - exact| = {err:.3e}"
+
+
 @pytest.mark.parametrize("name", ["tiny", "qwen3_small", "skew_small"])
 def test_permute_call_bit_exact(name):
     """Oracle routing in, dispatch out: counts, offsets, slots, rows bit-exact."""
