@@ -294,6 +294,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
     st, flags = layer.device_status()
     if st != B.MOE_OK:
         raise SystemExit(f"device status after timing: {B.status_string(st)} ({flags})")
+    refined = B.moe_router_refined_tokens(layer.ws)
 
     # end-to-end: pinned host x in, result back, through the public layer call
     e2e_steps = max(3, min(args.steps, 50))
@@ -350,6 +351,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
             "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": layer.x.numel() * layer.x.element_size(),
                     "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()},
+            "router_refined_tokens_last_step": refined,
             "gpu_launches": per_step_launches * args.steps,
             "clocks": clocks,
         }

@@ -235,6 +235,12 @@ moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, c
  * flag bits are stored in *flags when flags is not NULL. */
 moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags);
 
+/* Synchronise `stream` and store in *count how many tokens the last bf16
+ * router call of this workspace re-decided on exact logits (tokens whose
+ * top-(k+1) selection keys held two keys closer than the router's margin).
+ * Diagnostic only; 0 for fp32 layers. */
+moe_status moe_router_refined_tokens(void* ws, size_t ws_bytes, void* stream, int32_t* count);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -65,6 +65,7 @@ _SIGNATURES = {
                                      _VP, ctypes.POINTER(ctypes.c_void_p)]),
     "moe_permute_noalloc": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_device_status": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_uint32)]),
+    "moe_router_refined_tokens": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
 }
 
@@ -233,3 +234,10 @@ def moe_device_status(ws, stream=None):
     flags = ctypes.c_uint32(0)
     st = lib().moe_device_status(_p(ws), _nbytes(ws), _s(stream), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def moe_router_refined_tokens(ws, stream=None) -> int:
+    """Tokens the last bf16 router call re-decided on exact logits (synchronises)."""
+    c = ctypes.c_int32(0)
+    _check(lib().moe_router_refined_tokens(_p(ws), _nbytes(ws), _s(stream), ctypes.byref(c)), True)
+    return int(c.value)

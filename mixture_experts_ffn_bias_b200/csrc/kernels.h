@@ -22,7 +22,17 @@ cudaError_t router_select(const double* logits, const float* sel_bias, int T, in
                           cudaStream_t stream);
 
 // bf16 router: tensor-core fp32 logits, fast selection with near-tie
-// flagging, exact fp64 re-decision of the flagged tokens.
+// flagging, exact fp64 re-decision of the flagged tokens.  Tokens whose
+// top-(k+1) selection keys contain two keys closer than kRefineMargin are
+// re-decided on exact logits.  The tensor-core logits are within 5e-6 of the
+// exact ones (measured on every logit of the full workloads), so a key gap
+// above the margin cannot change order.
+constexpr float kRefineMargin = 1e-4f;
+bool router_fused_supported(int E, int k);
+cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, int K,
+                           const float* logit_offset, const float* sel_bias, int k, int gate,
+                           int renorm, int32_t* topk_idx, float* topk_w, int32_t* refine_count,
+                           int32_t* refine_list, uint32_t* status, cudaStream_t stream);
 cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
                              float* logits, uint32_t* status, cudaStream_t stream);
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,

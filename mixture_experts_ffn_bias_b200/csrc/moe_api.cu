@@ -108,10 +108,17 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
     float* logits = at<float>(ws, L.logits);
     int32_t* count = at<int32_t>(ws, L.status) + 1;
     int32_t* list = at<int32_t>(ws, L.refine);
-    MOE_TRY(moe::router_logits_tc(x, c->T, w_router, c->n_experts, c->d_model, logits,
-                                  at<uint32_t>(ws, L.status), s));
-    MOE_TRY(moe::router_select_fast(logits, logit_offset, sel_bias, c->T, c->n_experts, c->top_k,
-                                    c->gate, c->norm_topk_prob, topk_idx, topk_w, count, list, s));
+    if (moe::router_fused_supported(c->n_experts, c->top_k)) {
+      MOE_TRY(moe::router_topk_tc(x, c->T, w_router, c->n_experts, c->d_model, logit_offset,
+                                  sel_bias, c->top_k, c->gate, c->norm_topk_prob, topk_idx,
+                                  topk_w, count, list, at<uint32_t>(ws, L.status), s));
+    } else {
+      MOE_TRY(moe::router_logits_tc(x, c->T, w_router, c->n_experts, c->d_model, logits,
+                                    at<uint32_t>(ws, L.status), s));
+      MOE_TRY(moe::router_select_fast(logits, logit_offset, sel_bias, c->T, c->n_experts,
+                                      c->top_k, c->gate, c->norm_topk_prob, topk_idx, topk_w,
+                                      count, list, s));
+    }
     MOE_TRY(moe::router_refine(x, w_router, logit_offset, sel_bias, c->T, c->d_model,
                                c->n_experts, c->top_k, c->gate, c->norm_topk_prob, count, list,
                                topk_idx, topk_w, device_sms(), s));
@@ -395,6 +402,14 @@ moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
   if (flags) *flags = v;
   if (v & moe::kDevTimeout) return MOE_ERR_TIMEOUT;
   if (v & moe::kDevBadIndex) return MOE_ERR_DATA;
+  return MOE_OK;
+}
+
+moe_status moe_router_refined_tokens(void* ws, size_t ws_bytes, void* stream, int32_t* count) {
+  if (ws == nullptr || ws_bytes < 2 * sizeof(int32_t) || count == nullptr) return MOE_ERR_INVALID;
+  MOE_TRY(cudaStreamSynchronize(S(stream)));
+  MOE_TRY(cudaMemcpy(count, static_cast<int32_t*>(ws) + 1, sizeof(int32_t),
+                     cudaMemcpyDeviceToHost));
   return MOE_OK;
 }
 

@@ -205,12 +205,6 @@ router_select_kernel(const double* __restrict__ logits, const float* __restrict_
 }
 
 // ---------------------------------------------------------------- bf16 layers
-// Keys closer than this are re-decided on exact logits.  The fp32 tensor-core
-// accumulation error of a logit is ~1e-6 at d = 5120 (bf16 products are
-// exact; the error is the rounding of the running fp32 sum), and the fp32
-// keys add ~5e-7, so 1e-4 leaves a wide safety factor.
-constexpr float kRefineMargin = 1e-4f;
-
 // One warp per token, fp32 logits from the tensor cores.
 __global__ void __launch_bounds__(256)
 router_select_fast_kernel(const float* __restrict__ logits, const float* __restrict__ offset,
@@ -314,48 +308,64 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
 }
 
 // Exact re-decision of the listed tokens: fp64 sums of exact bf16 products,
-// then the fp64 selection.  Each block takes listed tokens round robin; the
-// experts' dot products are split over tpe threads each.
+// then the fp64 selection.  One block per listed token (round robin): the x
+// row is staged in shared memory as fp32, each warp takes experts w, w+8, ...
+// (two at a time) and reads the expert's router row with coalesced 16-byte
+// loads, fp64 accumulation, warp reduction.
 __global__ void __launch_bounds__(256)
 router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
                      const float* __restrict__ offset, const float* __restrict__ bias, int d,
                      int E, int k, int gate, int renorm, const int32_t* __restrict__ refine_count,
                      const int32_t* __restrict__ refine_list, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w) {
+  extern __shared__ float4 s_x4[];          // d floats
+  float* s_x = reinterpret_cast<float*>(s_x4);
   __shared__ double s_logit[256];
   const int n = *refine_count;
-  int tpe = 1;
-  while (tpe < 32 && tpe * E * 2 <= 256) tpe *= 2;        // threads per expert
-  const int e = threadIdx.x / tpe, part = threadIdx.x % tpe;
-  const int vecs = d / 8;                                 // 16-byte vectors per row
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int t = refine_list[i];
-    double acc0 = 0.0, acc1 = 0.0;
-    if (e < E) {
-      const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
-      const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * d);
-      for (int v = part; v < vecs; v += tpe) {
-        const uint4 a = __ldg(xr + v), b = __ldg(wrow + v);
-        const __nv_bfloat16* ah = reinterpret_cast<const __nv_bfloat16*>(&a);
-        const __nv_bfloat16* bh = reinterpret_cast<const __nv_bfloat16*>(&b);
+    for (int c = threadIdx.x; c < d; c += blockDim.x)
+      s_x[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
+    __syncthreads();
+    const float4* sx4 = reinterpret_cast<const float4*>(s_x);
+    for (int e0 = warp; e0 < E; e0 += 16) {
+      const int e1 = e0 + 8;
+      const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
+      const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1 < E ? e1 : e0) * d);
+      double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
+      for (int c0 = lane * 8; c0 < d; c0 += 256) {
+        const uint4 u0 = __ldg(r0 + c0 / 8), u1 = __ldg(r1 + c0 / 8);
+        const float4 xa = sx4[c0 / 4], xb = sx4[c0 / 4 + 1];
+        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
+        const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          acc0 = fma(static_cast<double>(__bfloat162float(ah[j])),
-                     static_cast<double>(__bfloat162float(bh[j])), acc0);
-          acc1 = fma(static_cast<double>(__bfloat162float(ah[j + 1])),
-                     static_cast<double>(__bfloat162float(bh[j + 1])), acc1);
+        for (int j = 0; j < 8; ++j) {
+          // bf16 x bf16 products are exact in fp32; the sums run in fp64
+          a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
+          b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
         }
       }
+      double a0 = (a[0] + a[1]) + (a[2] + a[3]);
+      double a1 = (b[0] + b[1]) + (b[2] + b[3]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+      }
+      if (lane == 0) {
+        s_logit[e0] = a0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
+        if (e1 < E) s_logit[e1] = a1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+      }
     }
-    double acc = acc0 + acc1;
-    for (int o = tpe / 2; o > 0; o >>= 1) acc += __shfl_down_sync(0xffffffffu, acc, o, tpe);
-    if (e < E && part == 0) s_logit[e] = acc + (offset ? static_cast<double>(offset[e]) : 0.0);
     __syncthreads();
-    if (threadIdx.x < 32) {
+    if (warp == 0) {
       double l[kMaxPerLane];
 #pragma unroll
       for (int j = 0; j < kMaxPerLane; ++j) {
-        const int ee = threadIdx.x + 32 * j;
+        const int ee = lane + 32 * j;
         l[j] = ee < E ? s_logit[ee] : -INFINITY;
       }
       warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
@@ -422,7 +432,14 @@ cudaError_t router_refine(const void* x, const void* w_router, const float* logi
                           int32_t* topk_idx, float* topk_w, int grid, cudaStream_t stream) {
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
-  router_refine_kernel<<<grid, 256, 0, stream>>>(
+  const size_t smem = static_cast<size_t>(d) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(router_refine_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  router_refine_kernel<<<grid, 256, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
       logit_offset, sel_bias, d, E, k, gate, renorm, refine_count, refine_list, topk_idx, topk_w);
   return cudaGetLastError();

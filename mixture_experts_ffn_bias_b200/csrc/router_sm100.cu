@@ -11,6 +11,15 @@
 // registers while the MMAs of the next chunks run.  This keeps the logit
 // error in the low 1e-6 range, far inside the router's re-decision margin.
 //
+// With up to 128 experts and top-k <= 8 the epilogue thread that owns a
+// token's row also takes the routing decision (fused select): it holds all of
+// the token's logits in registers, forms the gate statistics and the
+// selection keys, picks the top-(k+1) keys (descending, ties to the lower
+// expert id) and either writes the token's experts and weights or, when two
+// of those keys lie within kRefineMargin of each other, lists the token for
+// the exact re-decision kernel.  Otherwise the logits are written out and
+// router_select_fast_kernel decides.
+//
 // Warp roles (one 128-token tile at a time, persistent over tiles):
 //   warp 0        TMA: x tile 128 x 64 and Wr tile NPAD x 64 per stage
 //   warp 1        TMEM allocation, one lane issues tcgen05.mma into a ring of
@@ -34,33 +43,146 @@ constexpr int RBK = 64;
 constexpr int KCH = 2;                       // k-blocks per accumulation chunk
 constexpr int R_A_BYTES = RBM * RBK * 2;
 
-template <int NPAD>
+template <int NPAD, bool FUSED = false>
 struct RCfg {
   static constexpr int EPI_WG = NPAD > 128 ? 2 : 1;
   static constexpr int COLS = NPAD / EPI_WG;           // columns per epilogue thread
   static constexpr int THREADS = 64 + 128 * EPI_WG;
   static constexpr int B_BYTES = NPAD * RBK * 2;
   static constexpr int STAGE_BYTES = R_A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  // fused select keeps each token's logits in a shared-memory column
+  static constexpr int LOGIT_BYTES = FUSED ? NPAD * 128 * 4 : 0;
+  static constexpr int STAGE_BUDGET = 196608 - LOGIT_BYTES;
+  static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
   static constexpr int NSLOT = (512 / NPAD) > 8 ? 8 : (512 / NPAD);
   static constexpr int TMEM_RAW = NSLOT * NPAD;
   static constexpr int TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64
                                    : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LOGIT_BYTES + 1024 + 1024;
 };
 
-template <int NPAD>
-__global__ void __launch_bounds__(RCfg<NPAD>::THREADS, 1)
+constexpr int KMAX_FUSED = 8;
+
+struct RouterOut {
+  float* logits;                 // unfused: [T, E] fp32
+  const float* offset;           // fused: per-expert logit offset or null
+  const float* bias;             // fused: selection bias or null
+  int k, gate, renorm;
+  int32_t* topk_idx;             // fused outputs
+  float* topk_w;
+  int32_t* refine_count;
+  int32_t* refine_list;
+  uint32_t* status;
+};
+
+// Routing decision for one token from its logits held in registers (fused
+// select).  acc[i] = logit of expert i (i < E), overwritten with the
+// selection keys; the logits (with the per-expert offset) are kept in the
+// thread's shared-memory column s_log[i * 128] so the weights use them
+// exactly.
+template <int COLS>
+__device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int* s_seli,
+                                          const float* s_off, const float* s_bias, int E, int t,
+                                          const RouterOut& o) {
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < COLS; ++i) {
+    const float l = i < E ? acc[i] + s_off[i] : -INFINITY;
+    s_log[i * 128] = l;
+    acc[i] = i < E ? l + s_bias[i] : -INFINITY;
+    m = fmaxf(m, l);
+  }
+  float S = 0.f;
+  if (o.gate == 0) {
+#pragma unroll 8
+    for (int i = 0; i < COLS; ++i)
+      if (i < E) S += expf(s_log[i * 128] - m);
+  }
+  // top-(k+1) keys: each round takes the largest key strictly after the
+  // previous pick in (descending key, ascending expert id) order.  The round
+  // loop stays rolled (an unrolled 9 x 128 body overflows the instruction
+  // cache); four independent arg-max chains per round give the scheduler
+  // independent work.  Picks go to the thread's shared-memory columns.
+  const int rounds = o.k < E ? o.k + 1 : o.k;
+  float pv = INFINITY;
+  int pi = -1;
+  float min_gap = INFINITY;
+#pragma unroll 1
+  for (int j = 0; j < rounds; ++j) {
+    float bv[4];
+    int bi[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      bv[c] = -INFINITY;
+      bi[c] = 0x7fffffff;
+    }
+#pragma unroll
+    for (int i = 0; i < COLS; ++i) {
+      const int c = i & 3;
+      const float v = acc[i];
+      const bool after = v < pv || (v == pv && i > pi);
+      if (after && (v > bv[c] || bi[c] == 0x7fffffff)) {
+        bv[c] = v;
+        bi[c] = i;
+      }
+    }
+    // merge the chains: larger key wins, equal keys -> lower expert id
+#pragma unroll
+    for (int c = 1; c < 4; ++c) {
+      if (bi[c] != 0x7fffffff &&
+          (bi[0] == 0x7fffffff || bv[c] > bv[0] || (bv[c] == bv[0] && bi[c] < bi[0]))) {
+        bv[0] = bv[c];
+        bi[0] = bi[c];
+      }
+    }
+    if (j > 0) min_gap = fminf(min_gap, pv - bv[0]);
+    pv = bv[0];
+    pi = bi[0];
+    s_seli[j * 128] = bi[0];
+  }
+  if (min_gap < kRefineMargin) {
+    o.refine_list[atomicAdd(o.refine_count, 1)] = t;
+    return;
+  }
+  float sc[KMAX_FUSED];
+  int sid[KMAX_FUSED];
+  float ssum = 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX_FUSED; ++j) {
+    sc[j] = 0.f;
+    sid[j] = 0;
+    if (j < o.k) {
+      sid[j] = s_seli[j * 128];
+      const float l = s_log[sid[j] * 128];
+      sc[j] = o.gate == 1 ? 1.0f / (1.0f + expf(-l)) : expf(l - m) / S;
+      ssum += sc[j];
+    }
+  }
+  int32_t* irow = o.topk_idx + static_cast<size_t>(t) * o.k;
+  float* wrow = o.topk_w + static_cast<size_t>(t) * o.k;
+#pragma unroll
+  for (int j = 0; j < KMAX_FUSED; ++j) {
+    if (j < o.k) {
+      irow[j] = sid[j];
+      wrow[j] = o.renorm ? sc[j] / (ssum + 1e-9f) : sc[j];
+    }
+  }
+}
+
+template <int NPAD, bool FUSED>
+__global__ void __launch_bounds__(RCfg<NPAD, FUSED>::THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                 int T, int K, int E, float* __restrict__ logits, uint32_t* __restrict__ status) {
-  using C = RCfg<NPAD>;
+                 int T, int K, int E, const RouterOut out) {
+  using C = RCfg<NPAD, FUSED>;
   constexpr uint32_t IDESC = idesc_bf16_f32(RBM, NPAD);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * R_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  float* s_logits = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::LOGIT_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* sfull_bar = bars + 2 * C::STAGES;
@@ -68,6 +190,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  __shared__ float s_off[NPAD];
+  __shared__ float s_bias[NPAD];
+  __shared__ int s_sel[FUSED ? (KMAX_FUSED + 1) * 128 : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = (T + RBM - 1) / RBM;
@@ -90,6 +215,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
+  }
+  if (FUSED && warp >= 2) {
+    for (int e = threadIdx.x - 64; e < NPAD; e += 128) {
+      s_off[e] = (e < E && out.offset) ? out.offset[e] : 0.f;
+      s_bias[e] = (e < E && out.bias) ? out.bias[e] : 0.f;
+    }
   }
   if (warp == 1) {
     tmem_alloc(&s_tmem, C::TMEM_COLS);
@@ -196,8 +327,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       }
       if (!ok) break;
       const int t = tile * RBM + row;
-      if (t < T) {
-        float* dst = logits + static_cast<size_t>(t) * E + wg * C::COLS;
+      if (t >= T) continue;
+      if constexpr (FUSED) {
+        route_row<C::COLS>(acc, s_logits + (threadIdx.x - 64), s_sel + (threadIdx.x - 64),
+                           s_off, s_bias, E, t, out);
+      } else {
+        float* dst = out.logits + static_cast<size_t>(t) * E + wg * C::COLS;
         const int ncol = E - wg * C::COLS;
         if ((E & 3) == 0 && ncol >= C::COLS) {
 #pragma unroll
@@ -214,7 +349,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && s_abort) atomicOr(status, kDevTimeout);
+  if (threadIdx.x == 0 && s_abort) atomicOr(out.status, kDevTimeout);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -253,11 +388,11 @@ bool map2d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box
          CUDA_SUCCESS;
 }
 
-template <int NPAD>
+template <int NPAD, bool FUSED>
 cudaError_t launch_router(const CUtensorMap& mx, const CUtensorMap& mw, int T, int K, int E,
-                          float* logits, uint32_t* status, cudaStream_t stream) {
-  using C = RCfg<NPAD>;
-  auto kern = router_tc_kernel<NPAD>;
+                          const RouterOut& out, cudaStream_t stream) {
+  using C = RCfg<NPAD, FUSED>;
+  auto kern = router_tc_kernel<NPAD, FUSED>;
   static unsigned long long attr_done = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -272,26 +407,57 @@ cudaError_t launch_router(const CUtensorMap& mx, const CUtensorMap& mw, int T, i
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = (T + RBM - 1) / RBM;
   const int grid = tiles < sms ? tiles : (sms > 0 ? sms : 148);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mx, mw, T, K, E, logits, status);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mx, mw, T, K, E, out);
   return cudaGetLastError();
+}
+
+int npad_for(int E) {
+  int npad = 16;
+  while (npad < E) npad *= 2;
+  return npad;
+}
+
+bool maps(const void* x, int T, const void* w_router, int E, int K, CUtensorMap* mx,
+          CUtensorMap* mw) {
+  return map2d(mx, x, T, K, RBM) && map2d(mw, w_router, E, K, npad_for(E));
 }
 
 }  // namespace
 
+bool router_fused_supported(int E, int k) { return npad_for(E) <= 128 && k <= KMAX_FUSED; }
+
 cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
                              float* logits, uint32_t* status, cudaStream_t stream) {
-  int npad = 16;
-  while (npad < E) npad *= 2;
-  if (npad > 256 || T <= 0) return T <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+  if (T <= 0) return cudaSuccess;
+  const int npad = npad_for(E);
+  if (npad > 256) return cudaErrorInvalidValue;
   CUtensorMap mx, mw;
-  if (!map2d(&mx, x, T, K, RBM) || !map2d(&mw, w_router, E, K, npad))
-    return cudaErrorInvalidValue;
+  if (!maps(x, T, w_router, E, K, &mx, &mw)) return cudaErrorInvalidValue;
+  RouterOut o{logits, nullptr, nullptr, 0, 0, 0, nullptr, nullptr, nullptr, nullptr, status};
   switch (npad) {
-    case 16: return launch_router<16>(mx, mw, T, K, E, logits, status, stream);
-    case 32: return launch_router<32>(mx, mw, T, K, E, logits, status, stream);
-    case 64: return launch_router<64>(mx, mw, T, K, E, logits, status, stream);
-    case 128: return launch_router<128>(mx, mw, T, K, E, logits, status, stream);
-    default: return launch_router<256>(mx, mw, T, K, E, logits, status, stream);
+    case 16: return launch_router<16, false>(mx, mw, T, K, E, o, stream);
+    case 32: return launch_router<32, false>(mx, mw, T, K, E, o, stream);
+    case 64: return launch_router<64, false>(mx, mw, T, K, E, o, stream);
+    case 128: return launch_router<128, false>(mx, mw, T, K, E, o, stream);
+    default: return launch_router<256, false>(mx, mw, T, K, E, o, stream);
+  }
+}
+
+cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, int K,
+                           const float* logit_offset, const float* sel_bias, int k, int gate,
+                           int renorm, int32_t* topk_idx, float* topk_w, int32_t* refine_count,
+                           int32_t* refine_list, uint32_t* status, cudaStream_t stream) {
+  if (T <= 0) return cudaSuccess;
+  if (!router_fused_supported(E, k)) return cudaErrorInvalidValue;
+  CUtensorMap mx, mw;
+  if (!maps(x, T, w_router, E, K, &mx, &mw)) return cudaErrorInvalidValue;
+  RouterOut o{nullptr, logit_offset, sel_bias, k, gate, renorm, topk_idx, topk_w,
+              refine_count, refine_list, status};
+  switch (npad_for(E)) {
+    case 16: return launch_router<16, true>(mx, mw, T, K, E, o, stream);
+    case 32: return launch_router<32, true>(mx, mw, T, K, E, o, stream);
+    case 64: return launch_router<64, true>(mx, mw, T, K, E, o, stream);
+    default: return launch_router<128, true>(mx, mw, T, K, E, o, stream);
   }
 }
 

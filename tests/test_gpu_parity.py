@@ -157,6 +157,35 @@ def test_every_token_on_one_expert():
     _check_layer(shape, host, layer)
 
 
+@pytest.mark.parametrize("E,k,gate", [(256, 4, I.GATE_SOFTMAX), (32, 12, I.GATE_SIGMOID),
+                                      (200, 3, I.GATE_SIGMOID)])
+def test_router_paths_without_fused_select(E, k, gate):
+    """More than 128 experts or top-k above 8: logits are written out and a
+    separate selection kernel decides."""
+    shape = I.MoEShape("unfused", 300, 256, E, 128, k, 0, 0, gate, 1, I.DTYPE_BF16,
+                       "uniform", 0.0, 9)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
+@pytest.mark.parametrize("gate", [I.GATE_SOFTMAX, I.GATE_SIGMOID])
+def test_exact_key_ties_are_redecided_to_the_lower_expert(gate):
+    """Two experts with identical router rows and bias tie exactly on every
+    token; those tokens go through the exact re-decision, which must pick the
+    lower expert id first, as the oracle does."""
+    shape = SMALL["qwen3_small"].replace(T=400, gate=gate)
+    host = I.make_inputs(shape)
+    host["w_router"][77] = host["w_router"][5]
+    host["sel_bias"] = np.zeros(shape.n_experts, np.float32)
+    layer = _run(shape, host)
+    r = P.oracle_routing(shape, host)
+    gidx = _np(layer.topk_idx)
+    both = np.isin(r.topk_idx, [5, 77]).sum(1) == 2
+    assert both.any()
+    _check_layer(shape, host, layer)
+    np.testing.assert_array_equal(gidx[both], r.topk_idx[both])
+
+
 @pytest.mark.parametrize("gate", [I.GATE_SOFTMAX, I.GATE_SIGMOID])
 def test_constant_bias_moves_nothing_on_gpu(gate):
     shape = SMALL["qwen3_small"].replace(gate=gate, T=512)
