@@ -47,7 +47,10 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr int TMEM_COLS = 2 * BN_ACC;      // double-buffered accumulator
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*bars*/;
+  // epilogue staging: per epilogue warp 32 rows x 64 bf16 (128-byte swizzle)
+  static constexpr int EPI_BYTES = 4 * 32 * 128;
+  static constexpr int SMEM_BYTES =
+      STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + 1024 /*bars*/;
 };
 
 // Epilogue modes.
@@ -126,6 +129,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmC,
                     const GemmArgs args) {
   using Cfg = GemmCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
@@ -138,7 +142,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* smemA = smem;
   uint8_t* smemB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* smemEpi = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smemEpi + Cfg::EPI_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -172,6 +177,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     if (SWIGLU) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(&s_tmem_base, Cfg::TMEM_COLS);
@@ -290,42 +296,77 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const int n = local - m * n_tiles;
       const int rows_g = s_off[g + 1] - s_off[g];
       const bool valid = (m * BM + row) < rows_g;
+      // a warp whose 32 rows all belong to this group stages its rows in
+      // shared memory and writes them with one TMA store per 64 columns;
+      // a warp that straddles the end of the group stores its valid rows
+      // directly, so the next group's rows are never touched
+      const bool warp_full = (m * BM + q * 32 + 32) <= rows_g;
+      const int warp_row0 = s_off[g] + m * BM + q * 32;
+      uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
       const size_t crow_off = static_cast<size_t>(s_off[g] + m * BM + row) * args.ldc +
                               static_cast<size_t>(n) * BN_OUT;
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN_OUT / 16; ++c) {
-        uint32_t v[16];
-        uint32_t packed[8];
-        if (SWIGLU) {
-          uint32_t u[16];
-          tmem_ld16(t_addr + c * 16, v);
-          tmem_ld16(t_addr + BN_OUT + c * 16, u);
-          tmem_ld_wait();
+      for (int cb = 0; cb < BN_OUT / 64; ++cb) {
+        uint32_t packed[32];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
-            const float h1 = silu_f32(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-            packed[i] = pack_bf16x2(h0, h1);
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = cb * 64 + half * 32;      // first output column of this half
+          uint32_t v[32];
+          if (SWIGLU) {
+            uint32_t u[32];
+            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_ld16(t_addr + BN_OUT + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+            tmem_ld16(t_addr + BN_OUT + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 =
+                  silu_f32(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              packed[half * 16 + i] = pack_bf16x2(h0, h1);
+            }
+          } else {
+            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[half * 16 + i] =
+                  pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
           }
-        } else {
-          tmem_ld16(t_addr + c * 16, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            packed[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
-        if (valid) {
+        if (warp_full) {
+          if (lane == 0) bulk_wait_read_all();     // previous store has left the buffer
+          __syncwarp();
+          // row `lane`, 16-byte chunk c lands at chunk c ^ (lane % 8) (128-byte swizzle)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stage_buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                           packed[4 * c + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, stage_buf, n * BN_OUT + cb * 64, warp_row0);
+            bulk_commit();
+          }
+        } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
-                                                c * 16);
-          dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-          dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                                                cb * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                                packed[4 * c + 3]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
     }
+    if (lane == 0) bulk_wait_all();            // this warp's TMA stores are complete
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -381,7 +422,8 @@ int num_sms() {
 
 template <int BN_ACC, int MODE>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                   const GemmArgs& args, int rows_upper, cudaStream_t stream) {
+                   const CUtensorMap& c, const GemmArgs& args, int rows_upper,
+                   cudaStream_t stream) {
   using Cfg = GemmCfg<BN_ACC>;
   constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
   auto kern = grouped_gemm_kernel<BN_ACC, MODE>;
@@ -400,7 +442,7 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
   if (tiles_upper <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles_upper < num_sms() ? tiles_upper : num_sms());
-  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, args);
+  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, args);
   return cudaGetLastError();
 }
 
@@ -411,29 +453,32 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
                                        cudaStream_t stream) {
-  CUtensorMap ta, tb0, tb1;
+  CUtensorMap ta, tb0, tb1, tc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
+  const int64_t c_rows = offsets ? a_rows : rows_single;
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
-      !make_map(&tb1, W3, b_rows, K, 128))
+      !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, args, rows_upper, stream);
+  return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
 }
 
 // Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
+  const int64_t c_rows = offsets ? a_rows : rows_single;
   const int bn = (N % 256 == 0) ? 256 : 128;
-  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn))
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn) ||
+      !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, args, rows_upper, stream);
-  return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, args, rows_upper, stream);
+  if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+  return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
 }
 
 

@@ -39,10 +39,12 @@ cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
                                int32_t* topk_idx, float* topk_w, int32_t* refine_count,
                                int32_t* refine_list, cudaStream_t stream);
+// exact_scratch: fp64 [T, E] (rows indexed by position in the refine list).
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
                           int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          int32_t* topk_idx, float* topk_w, int grid, cudaStream_t stream);
+                          double* exact_scratch, int32_t* topk_idx, float* topk_w, int sms,
+                          cudaStream_t stream);
 
 // logits[t, e] += offset[e]
 cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream);

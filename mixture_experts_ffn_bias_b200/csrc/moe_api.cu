@@ -119,9 +119,11 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
                                       c->top_k, c->gate, c->norm_topk_prob, topk_idx, topk_w,
                                       count, list, s));
     }
+    // the fp32 logits (unfused path) are consumed before the exact logits of
+    // the listed tokens reuse the same scratch region
     MOE_TRY(moe::router_refine(x, w_router, logit_offset, sel_bias, c->T, c->d_model,
                                c->n_experts, c->top_k, c->gate, c->norm_topk_prob, count, list,
-                               topk_idx, topk_w, device_sms(), s));
+                               at<double>(ws, L.logits), topk_idx, topk_w, device_sms(), s));
     return MOE_OK;
   }
   double* logits = at<double>(ws, L.logits);

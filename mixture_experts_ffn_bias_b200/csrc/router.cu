@@ -307,71 +307,90 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
   }
 }
 
-// Exact re-decision of the listed tokens: fp64 sums of exact bf16 products,
-// then the fp64 selection.  One block per listed token (round robin): the x
-// row is staged in shared memory as fp32, each warp takes experts w, w+8, ...
-// (two at a time) and reads the expert's router row with coalesced 16-byte
-// loads, fp64 accumulation, warp reduction.
+// Exact re-decision of the listed tokens, in two kernels.
+// router_refine_logits_kernel: blocks are (listed token, chunk of 16
+// experts); the token's x row is staged in shared memory as fp32, each warp
+// computes two experts' exact logits (bf16 x bf16 products are exact in fp32,
+// the sums run in fp64) from coalesced 16-byte reads of the router rows, and
+// writes them to exact[i, e] (fp64 scratch, i = position in the list).
+// Spreading one token's experts over several blocks keeps the per-token
+// latency low when only a handful of tokens are listed.
+constexpr int kRefineExperts = 16;
+
 __global__ void __launch_bounds__(256)
-router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
-                     const float* __restrict__ offset, const float* __restrict__ bias, int d,
-                     int E, int k, int gate, int renorm, const int32_t* __restrict__ refine_count,
-                     const int32_t* __restrict__ refine_list, int32_t* __restrict__ topk_idx,
-                     float* __restrict__ topk_w) {
-  extern __shared__ float4 s_x4[];          // d floats
-  float* s_x = reinterpret_cast<float*>(s_x4);
-  __shared__ double s_logit[256];
+router_refine_logits_kernel(const __nv_bfloat16* __restrict__ x,
+                            const __nv_bfloat16* __restrict__ wr,
+                            const float* __restrict__ offset, int d, int E,
+                            const int32_t* __restrict__ refine_count,
+                            const int32_t* __restrict__ refine_list,
+                            double* __restrict__ exact) {
+  extern __shared__ float4 s_x4[];           // d floats
+  const float* s_x = reinterpret_cast<const float*>(s_x4);
   const int n = *refine_count;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e0 = blockIdx.y * kRefineExperts + warp;
+  const int e1 = e0 + 8;
   for (int i = blockIdx.x; i < n; i += gridDim.x) {
     const int t = refine_list[i];
+    __syncthreads();
     for (int c = threadIdx.x; c < d; c += blockDim.x)
-      s_x[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
+      reinterpret_cast<float*>(s_x4)[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
     __syncthreads();
+    if (e0 >= E) continue;
+    const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
+    const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1 < E ? e1 : e0) * d);
     const float4* sx4 = reinterpret_cast<const float4*>(s_x);
-    for (int e0 = warp; e0 < E; e0 += 16) {
-      const int e1 = e0 + 8;
-      const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
-      const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1 < E ? e1 : e0) * d);
-      double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 2
-      for (int c0 = lane * 8; c0 < d; c0 += 256) {
-        const uint4 u0 = __ldg(r0 + c0 / 8), u1 = __ldg(r1 + c0 / 8);
-        const float4 xa = sx4[c0 / 4], xb = sx4[c0 / 4 + 1];
-        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
-        const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int c0 = lane * 8; c0 < d; c0 += 256) {
+      const uint4 u0 = __ldg(r0 + c0 / 8), u1 = __ldg(r1 + c0 / 8);
+      const float4 xa = sx4[c0 / 4], xb = sx4[c0 / 4 + 1];
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
+      const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // bf16 x bf16 products are exact in fp32; the sums run in fp64
-          a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
-          b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
-        }
-      }
-      double a0 = (a[0] + a[1]) + (a[2] + a[3]);
-      double a1 = (b[0] + b[1]) + (b[2] + b[3]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        a0 += __shfl_xor_sync(0xffffffffu, a0, o);
-        a1 += __shfl_xor_sync(0xffffffffu, a1, o);
-      }
-      if (lane == 0) {
-        s_logit[e0] = a0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
-        if (e1 < E) s_logit[e1] = a1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+      for (int j = 0; j < 8; ++j) {
+        a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
+        b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
       }
     }
-    __syncthreads();
-    if (warp == 0) {
-      double l[kMaxPerLane];
+    double s0 = (a[0] + a[1]) + (a[2] + a[3]);
+    double s1 = (b[0] + b[1]) + (b[2] + b[3]);
 #pragma unroll
-      for (int j = 0; j < kMaxPerLane; ++j) {
-        const int ee = lane + 32 * j;
-        l[j] = ee < E ? s_logit[ee] : -INFINITY;
-      }
-      warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
-                       topk_w + static_cast<size_t>(t) * k);
+    for (int o = 16; o > 0; o >>= 1) {
+      s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
     }
-    __syncthreads();
+    if (lane == 0) {
+      exact[static_cast<size_t>(i) * E + e0] = s0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
+      if (e1 < E)
+        exact[static_cast<size_t>(i) * E + e1] =
+            s1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+    }
+  }
+}
+
+// router_refine_select_kernel: one warp per listed token, fp64 selection on
+// the exact logits.
+__global__ void __launch_bounds__(256)
+router_refine_select_kernel(const double* __restrict__ exact, const float* __restrict__ bias,
+                            int E, int k, int gate, int renorm,
+                            const int32_t* __restrict__ refine_count,
+                            const int32_t* __restrict__ refine_list,
+                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int n = *refine_count;
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+    const int t = refine_list[i];
+    double l[kMaxPerLane];
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j) {
+      const int e = lane + 32 * j;
+      l[j] = e < E ? exact[static_cast<size_t>(i) * E + e] : -INFINITY;
+    }
+    warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
+                     topk_w + static_cast<size_t>(t) * k);
   }
 }
 
@@ -429,19 +448,27 @@ cudaError_t router_select_fast(const float* logits, const float* logit_offset,
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
                           int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          int32_t* topk_idx, float* topk_w, int grid, cudaStream_t stream) {
-  if (grid > T) grid = T;
-  if (grid < 1) grid = 1;
+                          double* exact_scratch, int32_t* topk_idx, float* topk_w, int sms,
+                          cudaStream_t stream) {
+  const int gx = sms < T ? sms : T;
+  const dim3 grid(gx > 0 ? gx : 1, (E + kRefineExperts - 1) / kRefineExperts);
   const size_t smem = static_cast<size_t>(d) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_refine_kernel,
+    cudaError_t e = cudaFuncSetAttribute(router_refine_logits_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  router_refine_kernel<<<grid, 256, smem, stream>>>(
+  router_refine_logits_kernel<<<grid, 256, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
-      logit_offset, sel_bias, d, E, k, gate, renorm, refine_count, refine_list, topk_idx, topk_w);
+      logit_offset, d, E, refine_count, refine_list, exact_scratch);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int warps = 8;
+  int gs = (T + warps - 1) / warps;
+  if (gs > sms) gs = sms > 0 ? sms : 1;
+  router_refine_select_kernel<<<gs, warps * 32, 0, stream>>>(
+      exact_scratch, sel_bias, E, k, gate, renorm, refine_count, refine_list, topk_idx, topk_w);
   return cudaGetLastError();
 }
 
