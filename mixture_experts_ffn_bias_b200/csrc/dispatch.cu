@@ -170,7 +170,35 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
   }
 }
 
+// One thread per token: final rows and the token of each row, no copy.
+__global__ void __launch_bounds__(256)
+dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ bases,
+                          int32_t* __restrict__ slot_pos, int32_t* __restrict__ perm_src, int T,
+                          int k, int E) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const int32_t* b = bases + static_cast<size_t>(t / kRankBlock) * E;
+  for (int j = 0; j < k; ++j) {
+    const size_t p = static_cast<size_t>(t) * k + j;
+    const int r = slot_pos[p];
+    int slot = -1;
+    if (r >= 0) {
+      slot = b[topk_idx[p]] + r;
+      perm_src[slot] = t;
+    }
+    slot_pos[p] = slot;
+  }
+}
+
 }  // namespace
+
+cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
+                               int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
+                               cudaStream_t stream) {
+  dispatch_positions_kernel<<<(T + 255) / 256, 256, 0, stream>>>(topk_idx, blk_bases, slot_pos,
+                                                                 perm_src, T, k, E);
+  return cudaGetLastError();
+}
 
 cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream) {

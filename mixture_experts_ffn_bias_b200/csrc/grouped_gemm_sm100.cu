@@ -66,6 +66,8 @@ struct GemmArgs {
   void* C;
   int ldc;                 // elements
   uint32_t* status;
+  const int32_t* gather_rows;  // GATHER: A row of output row r is gather_src[gather_rows[r]]
+  const void* gather_src;      // GATHER: [rows, K] bf16
 };
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
@@ -124,7 +126,7 @@ __device__ __forceinline__ int find_group(const int* s_prefix, int G, int tile) 
   return lo;
 }
 
-template <int BN_ACC, int MODE>
+template <int BN_ACC, int MODE, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
@@ -174,7 +176,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
+    if (!GATHER) tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     if (SWIGLU) tma_prefetch_desc(&tmB1);
     tma_prefetch_desc(&tmC);
@@ -195,23 +197,58 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued_mask = 0;     // stages with a load in flight at exit
-      uint32_t issued_phase = 0;    // parity of that load's phase
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-        const int g = find_group(s_prefix, G, tile);
-        const int local = tile - s_prefix[g];
-        const int m = local / n_tiles;
-        const int n = local - m * n_tiles;
-        const int arow = s_off[g] + m * BM;
-        const int brow = g * args.n_per_group + n * BN_OUT;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
-          tma_load_2d(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
+    // Lane 0 drives the ring.  With GATHER the whole warp fills the A tile
+    // with 16-byte cp.async: warp instruction i copies rows 4i..4i+3 (lane
+    // / 8 picks the row, lane % 8 the 16-byte chunk), written at the
+    // 128-byte-swizzled position the MMA descriptor expects; each lane's
+    // copies are tracked on the stage barrier by cp.async.mbarrier.arrive.
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0;     // stages with a load in flight at exit
+    uint32_t issued_phase = 0;    // parity of that load's phase
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+      const int g = find_group(s_prefix, G, tile);
+      const int local = tile - s_prefix[g];
+      const int m = local / n_tiles;
+      const int n = local - m * n_tiles;
+      const int arow = s_off[g] + m * BM;
+      const int brow = g * args.n_per_group + n * BN_OUT;
+      int tok[GATHER ? 32 : 1];
+      if (GATHER) {
+        // rows past the group's end read a valid row (the first of the
+        // tile); the epilogue never stores them
+        const int rows_g = s_off[g + 1] - s_off[g];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          tok[i] = args.gather_rows[m * BM + r < rows_g ? arow + r : arow];
+        }
+      }
+      for (int kb = 0; kb < kblocks; ++kb) {
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
+        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) { ok = false; break; }
+        if (GATHER) {
+          const int c = lane & 7;
+          uint8_t* a_tile = smemA + stage * A_STAGE_BYTES;
+          const __nv_bfloat16* xa = static_cast<const __nv_bfloat16*>(args.gather_src) +
+                                    kb * BK + c * 8;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int r = 4 * i + (lane >> 3);
+            cp_async_16(a_tile + r * 128 + ((c ^ (r & 7)) << 4),
+                        xa + static_cast<size_t>(tok[i]) * args.K);
+          }
+          cp_async_arrive(&full_bar[stage]);
+          __syncwarp();
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full_bar[stage],
+                                GATHER ? Cfg::B_STAGE_BYTES : Cfg::STAGE_BYTES);
+          if (!GATHER)
+            tma_load_2d(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
           uint8_t* b = smemB + stage * Cfg::B_STAGE_BYTES;
           if (SWIGLU) {
             tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
@@ -219,20 +256,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           } else {
             tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
           }
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) {
-        // Let every TMA copy this CTA started land before the CTA exits.
-        for (int s = 0; s < STAGES; ++s) {
-          if (!(issued_mask & (1u << s))) continue;
-          const uint32_t par = (issued_phase >> s) & 1u;
-          const unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full_bar[s], par)) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-          }
+    }
+    if (!ok && lane == 0) {
+      // Let every TMA copy this CTA started land before the CTA exits.
+      for (int s = 0; s < STAGES; ++s) {
+        if (!(issued_mask & (1u << s))) continue;
+        const uint32_t par = (issued_phase >> s) & 1u;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full_bar[s], par)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
         }
       }
     }
@@ -252,6 +289,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t d_tmem = tmem_base + acc * BN_ACC;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          // cp.async wrote the A tile through the generic proxy; make it
+          // visible to the tensor core's async-proxy reads
+          if (GATHER) fence_async_shared();
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smemA + stage * A_STAGE_BYTES);
           const uint32_t b_addr = smem_u32(smemB + stage * Cfg::B_STAGE_BYTES);
@@ -420,13 +460,13 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int BN_ACC, int MODE>
+template <int BN_ACC, int MODE, bool GATHER = false>
 cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                    const CUtensorMap& c, const GemmArgs& args, int rows_upper,
                    cudaStream_t stream) {
   using Cfg = GemmCfg<BN_ACC>;
   constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
-  auto kern = grouped_gemm_kernel<BN_ACC, MODE>;
+  auto kern = grouped_gemm_kernel<BN_ACC, MODE, GATHER>;
   static unsigned long long attr_done = 0;   // one bit per device (attribute is per device)
   int dev = 0;
   cudaGetDevice(&dev);
@@ -459,9 +499,26 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
       !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status};
+  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
+}
+
+// Gate/up pass whose A rows are gathered from X [x_rows, K]: output row r
+// (expert-contiguous order, r < R) reads X[rows[r]].  H is [R, F].
+cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows,
+                                              int64_t R, const int32_t* offsets, int num_groups,
+                                              const void* W1, const void* W3, int F, int K,
+                                              void* H, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap tb0, tb1, tc;
+  const int64_t b_rows = static_cast<int64_t>(num_groups) * F;
+  (void)x_rows;
+  if (!make_map(&tb0, W1, b_rows, K, 128) || !make_map(&tb1, W3, b_rows, K, 128) ||
+      !make_map(&tc, H, R, F, 32))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X};
+  // tmA is unused in gather mode (A comes through cp.async)
+  return launch<256, MODE_SWIGLU_BF16, true>(tb0, tb0, tb1, tc, args, static_cast<int>(R), stream);
 }
 
 // Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.
@@ -475,7 +532,7 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status};
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
   return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);

@@ -56,6 +56,10 @@ cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t*
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream);
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream);
+// slot_pos (in: rank, out: row) and perm_src only, no row copy.
+cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
+                               int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
+                               cudaStream_t stream);
 cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              const int32_t* blk_bases, int32_t* slot_pos, int32_t* perm_src,
                              void* x_perm, int T, int d, int k, int E, cudaStream_t stream);
@@ -65,6 +69,10 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
                                        cudaStream_t stream);
+cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows,
+                                              int64_t R, const int32_t* offsets, int num_groups,
+                                              const void* W1, const void* W3, int F, int K,
+                                              void* H, uint32_t* status, cudaStream_t stream);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream);

@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cstdlib>
 
 #include "../../include/moe.h"
 #include "kernels.h"
@@ -143,6 +144,11 @@ moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void*
   const int nblk = moe::rank_blocks(c->T);
   MOE_TRY(moe::dispatch_rank(topk_idx, c->T, c->top_k, c->n_experts, blk, slot_pos, status, s));
   MOE_TRY(moe::dispatch_scan(blk, nblk, c->n_experts, counts, offsets, s));
+  if (x_perm == nullptr) {   // rows only; the experts gather x through perm_src
+    MOE_TRY(moe::dispatch_positions(topk_idx, blk, slot_pos, perm_src, c->T, c->top_k,
+                                    c->n_experts, s));
+    return MOE_OK;
+  }
   MOE_TRY(moe::dispatch_scatter(c->dtype == MOE_BF16, x, topk_idx, blk, slot_pos, perm_src,
                                 x_perm, c->T, c->d_model, c->top_k, c->n_experts, s));
   return MOE_OK;
@@ -157,17 +163,24 @@ struct Marks {
   }
 };
 
+// x_perm == nullptr (bf16 only): the gate/up GEMM gathers its rows from x
+// through gather_rows (perm_src) instead of reading a permuted copy.
 moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* offsets,
                        const moe_expert_weights* w, const void* x, void* y_perm, void* y_shared,
-                       void* ws, cudaStream_t s, const Marks& mk) {
+                       void* ws, cudaStream_t s, const Marks& mk,
+                       const int32_t* gather_rows = nullptr) {
   const Layout L = layout(*c);
   uint32_t* status = at<uint32_t>(ws, L.status);
   const int64_t R = static_cast<int64_t>(c->T) * c->top_k;
   const int E = c->n_experts, F = c->d_ff, d = c->d_model;
   void* h = at<void>(ws, L.h);
   if (c->dtype == MOE_BF16) {
-    MOE_TRY(moe::grouped_swiglu_gateup_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d, h,
-                                            status, s));
+    if (x_perm == nullptr)
+      MOE_TRY(moe::grouped_swiglu_gateup_gather_bf16(x, c->T, gather_rows, R, offsets, E, w->w1,
+                                                     w->w3, F, d, h, status, s));
+    else
+      MOE_TRY(moe::grouped_swiglu_gateup_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d, h,
+                                              status, s));
     if (!mk.rec(3)) return MOE_ERR_CUDA;
     MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s));
     if (!mk.rec(4)) return MOE_ERR_CUDA;
@@ -249,11 +262,20 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   void* y_sh = cfg->n_shared ? at<void>(ws, L.y_sh) : nullptr;
-  if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, at<int32_t>(ws, L.perm_src),
-                        x_perm, ws, s)) != MOE_OK)
+  // Default: dispatch writes the permuted copy x_perm and the gate/up GEMM
+  // reads it with TMA tiles.  MOE_B200_GATHER_A=1 (bf16 only) skips the copy
+  // and lets the gate/up GEMM gather its rows from x by perm_src; it moves
+  // less memory but measured slower on B200 (each of an m-tile's n-tile CTAs
+  // gathers the same rows again).
+  const char* ga = std::getenv("MOE_B200_GATHER_A");
+  const bool gather = cfg->dtype == MOE_BF16 && ga != nullptr && ga[0] == '1';
+  int32_t* perm_src = at<int32_t>(ws, L.perm_src);
+  if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
+                        gather ? nullptr : x_perm, ws, s)) != MOE_OK)
     return st;
   if (!mk.rec(2)) return MOE_ERR_CUDA;
-  if ((st = run_experts(cfg, x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk)) != MOE_OK)
+  if ((st = run_experts(cfg, gather ? nullptr : x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk,
+                        perm_src)) != MOE_OK)
     return st;
   MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_sh, out, cfg->T,
                        cfg->d_model, cfg->top_k, s));

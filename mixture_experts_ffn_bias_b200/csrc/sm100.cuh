@@ -89,6 +89,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (L2 only, no L1 allocation).
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+               ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// Arrive on `bar` once all prior cp.async of this thread have completed; the
+// pending count is raised now, so the phase cannot complete before that.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // 2-D tiled store shared -> global (bulk-group completion).  Rows or columns
 // of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int32_t x,

@@ -87,6 +87,16 @@ def test_forward_full_size_sampled(name):
     torch.cuda.empty_cache()
 
 
+@pytest.mark.parametrize("name", ["page2_small", "qwen3_small", "skew_small"])
+def test_forward_with_gathered_gate_up_rows(name, monkeypatch):
+    """The alternative expert path that skips the permuted copy of x and
+    gathers the gate/up GEMM's rows from x (MOE_B200_GATHER_A=1)."""
+    monkeypatch.setenv("MOE_B200_GATHER_A", "1")
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
 def test_skew_bias_update_then_deferred_forward():
     """Skewed workload: forward, bias update from its counts (bit-exact), then a
     second forward routes with the new bias (the update lands on the next
