@@ -68,6 +68,7 @@ struct GemmArgs {
   uint32_t* status;
   const int32_t* gather_rows;  // GATHER: A row of output row r is gather_src[gather_rows[r]]
   const void* gather_src;      // GATHER: [rows, K] bf16
+  int m_fastest;               // tile order inside a group: 1 = m-tiles fastest
 };
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
@@ -114,6 +115,23 @@ __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, in
   }
   if (lane == 31) s_prefix[G] = incl;
   __syncwarp();
+}
+
+// Tile order inside a group.  n fastest (default): the CTAs running at the
+// same time share A tiles and one expert's weights, which suits experts whose
+// weights fit in L2 many times over.  m fastest: they share B tiles instead,
+// so an expert whose weights are a large part of L2 is streamed from HBM
+// once while its (smaller) rows are re-read from L2.
+__device__ __forceinline__ void tile_mn(int local, int rows_g, int n_tiles, int m_fastest,
+                                        int& m, int& n) {
+  if (m_fastest) {
+    const int mt = (rows_g + BM - 1) / BM;
+    n = local / mt;
+    m = local - n * mt;
+  } else {
+    m = local / n_tiles;
+    n = local - m * n_tiles;
+  }
 }
 
 // Largest g with prefix[g] <= tile (groups with no tiles are skipped).
@@ -209,9 +227,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
       const int g = find_group(s_prefix, G, tile);
-      const int local = tile - s_prefix[g];
-      const int m = local / n_tiles;
-      const int n = local - m * n_tiles;
+      int m, n;
+      tile_mn(tile - s_prefix[g], s_off[g + 1] - s_off[g], n_tiles, args.m_fastest, m, n);
       const int arow = s_off[g] + m * BM;
       const int brow = g * args.n_per_group + n * BN_OUT;
       int tok[GATHER ? 32 : 1];
@@ -331,10 +348,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       if (!ok) break;
       tc_fence_after();
       const int g = find_group(s_prefix, G, tile);
-      const int local = tile - s_prefix[g];
-      const int m = local / n_tiles;
-      const int n = local - m * n_tiles;
       const int rows_g = s_off[g + 1] - s_off[g];
+      int m, n;
+      tile_mn(tile - s_prefix[g], rows_g, n_tiles, args.m_fastest, m, n);
       const bool valid = (m * BM + row) < rows_g;
       // a warp whose 32 rows all belong to this group stages its rows in
       // shared memory and writes them with one TMA store per 64 columns;
@@ -478,11 +494,18 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
     attr_done |= bit;
   }
   const int G = args.offsets == nullptr ? 1 : args.num_groups;
+  // m-fastest order once one group's weights (B rows x K, both halves for
+  // SwiGLU) exceed 32 MB, a quarter of the L2
+  GemmArgs a2 = args;
+  const double b_bytes = static_cast<double>(BN_OUT == BN_ACC ? args.n_per_group
+                                                              : 2 * args.n_per_group) *
+                         args.K * 2.0;
+  a2.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
   const long long m_tiles_upper = (rows_upper + BM - 1) / BM + (G > 1 ? G : 0);
   const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
   if (tiles_upper <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles_upper < num_sms() ? tiles_upper : num_sms());
-  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, args);
+  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, a2);
   return cudaGetLastError();
 }
 
@@ -499,7 +522,7 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
       !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr};
+  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
 }
@@ -516,7 +539,7 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
   if (!make_map(&tb0, W1, b_rows, K, 128) || !make_map(&tb1, W3, b_rows, K, 128) ||
       !make_map(&tc, H, R, F, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X};
+  GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0};
   // tmA is unused in gather mode (A comes through cp.async)
   return launch<256, MODE_SWIGLU_BF16, true>(tb0, tb0, tb1, tc, args, static_cast<int>(R), stream);
 }
@@ -532,7 +555,7 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr};
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
   return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);

@@ -141,6 +141,15 @@ def test_zero_tokens_is_a_noop():
     assert int(counts.abs().sum()) == 0
 
 
+def test_large_experts_use_m_fastest_tile_order():
+    """Experts whose weights exceed a quarter of L2 are tiled m-fastest; check
+    that order element-wise (two 5120 x 4352 experts, ragged rows)."""
+    shape = I.MoEShape("big_experts", 333, 5120, 2, 4352, 1, 0, 0, I.GATE_SOFTMAX, 1,
+                       I.DTYPE_BF16, "uniform", 0.0, 10)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
 def test_one_expert_top1_is_dense_ffn():
     shape = I.MoEShape("one", 300, 256, 1, 256, 1, 0, 0, I.GATE_SOFTMAX, 1, I.DTYPE_BF16,
                        "none", 0.0, 7)
