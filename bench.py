@@ -329,7 +329,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         t_gemm = (phases[2] + phases[3] + phases[4]) * 1e-3
         achieved = fl["gate_up"] / t_gateup / 1e12
         gemm_tflops = (fl["gate_up"] + fl["down"] + fl["shared"]) / t_gemm / 1e12
-        router_launches = 3 if shape.dtype == I.DTYPE_BF16 else 2   # fused TC router + refine logits + refine select
+        router_launches = 2   # bf16: fused TC router + refine; fp32: logits + select
         per_step_launches = router_launches + 3 + 2 + 2 * shape.n_shared + 1 + 1
         line = {
             "metric": METRIC, "value": shape.T * world / (ms * 1e-3), "unit": UNIT,

@@ -55,12 +55,15 @@ struct Vec<false> {
   }
 };
 
-template <bool BF16>
+// KT > 0: k == KT known at compile time, so each lane issues the loads of all
+// k rows (and the shared row) before it accumulates; KT == 0: any k.
+template <bool BF16, int KT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
                const float* __restrict__ topk_w, const uint4* __restrict__ y_shared,
-               uint4* __restrict__ out, int T, int vecs, int k) {
+               uint4* __restrict__ out, int T, int vecs, int k_rt) {
   using V = Vec<BF16>;
+  const int k = KT > 0 ? KT : k_rt;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -69,6 +72,40 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slo
   if (lane < k) {
     my_slot = slot_pos[static_cast<size_t>(t) * k + lane];
     my_w = topk_w[static_cast<size_t>(t) * k + lane];
+  }
+  if (KT > 0) {
+    int sl[KT > 0 ? KT : 1];
+    float wj[KT > 0 ? KT : 1];
+#pragma unroll
+    for (int j = 0; j < KT; ++j) {
+      sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
+      wj[j] = __shfl_sync(0xffffffffu, my_w, j);
+    }
+    for (int c = lane; c < vecs; c += 32) {
+      uint4 v[KT > 0 ? KT : 1];
+      uint4 vs = make_uint4(0u, 0u, 0u, 0u);
+      if (y_shared) vs = __ldcs(y_shared + static_cast<size_t>(t) * vecs + c);
+#pragma unroll
+      for (int j = 0; j < KT; ++j)
+        v[j] = sl[j] >= 0 ? __ldcs(y_perm + static_cast<size_t>(sl[j]) * vecs + c)
+                          : make_uint4(0u, 0u, 0u, 0u);
+      float acc[V::N];
+      if (y_shared) {
+        V::load(vs, acc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < KT; ++j) {
+        float f[V::N];
+        V::load(v[j], f);
+#pragma unroll
+        for (int i = 0; i < V::N; ++i) acc[i] = fmaf(wj[j], f[i], acc[i]);
+      }
+      out[static_cast<size_t>(t) * vecs + c] = V::store(acc);
+    }
+    return;
   }
   for (int c = lane; c < vecs; c += 32) {
     float acc[V::N];
@@ -118,19 +155,31 @@ bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias,
 
 }  // namespace
 
+template <bool BF16>
+void launch_combine(dim3 grid, int threads, cudaStream_t stream, const uint4* y, const int32_t* sp,
+                    const float* w, const uint4* ysh, uint4* out, int T, int vecs, int k) {
+  switch (k) {
+    case 1: combine_kernel<BF16, 1><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
+    case 2: combine_kernel<BF16, 2><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
+    case 4: combine_kernel<BF16, 4><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
+    case 6: combine_kernel<BF16, 6><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
+    case 8: combine_kernel<BF16, 8><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
+    default: combine_kernel<BF16, 0><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k);
+  }
+}
+
 cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
                     const void* y_shared, void* out, int T, int d, int k, cudaStream_t stream) {
   const int vecs = d * (bf16 ? 2 : 4) / 16;
   const int warps = 8;
   const dim3 grid((T + warps - 1) / warps);
+  const uint4* y = static_cast<const uint4*>(y_perm);
+  const uint4* ysh = static_cast<const uint4*>(y_shared);
+  uint4* o = static_cast<uint4*>(out);
   if (bf16)
-    combine_kernel<true><<<grid, warps * 32, 0, stream>>>(
-        static_cast<const uint4*>(y_perm), slot_pos, topk_w,
-        static_cast<const uint4*>(y_shared), static_cast<uint4*>(out), T, vecs, k);
+    launch_combine<true>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
   else
-    combine_kernel<false><<<grid, warps * 32, 0, stream>>>(
-        static_cast<const uint4*>(y_perm), slot_pos, topk_w,
-        static_cast<const uint4*>(y_shared), static_cast<uint4*>(out), T, vecs, k);
+    launch_combine<false>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
   return cudaGetLastError();
 }
 

@@ -28,22 +28,29 @@ cudaError_t router_select(const double* logits, const float* sel_bias, int T, in
 // exact ones (measured on every logit of the full workloads), so a key gap
 // above the margin cannot change order.
 constexpr float kRefineMargin = 1e-4f;
+// A listed token carries up to kRefineCand candidate experts (the experts
+// whose key is within the margin of its (k+1)-th pick); -2 in slot 0 means
+// "re-decide over all experts".
+constexpr int kRefineCand = 16;
 bool router_fused_supported(int E, int k);
 cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, int K,
                            const float* logit_offset, const float* sel_bias, int k, int gate,
                            int renorm, int32_t* topk_idx, float* topk_w, int32_t* refine_count,
-                           int32_t* refine_list, uint32_t* status, cudaStream_t stream);
+                           int32_t* refine_list, int32_t* refine_cand, uint32_t* status,
+                           cudaStream_t stream);
 cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
                              float* logits, uint32_t* status, cudaStream_t stream);
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
                                int32_t* topk_idx, float* topk_w, int32_t* refine_count,
                                int32_t* refine_list, cudaStream_t stream);
-// exact_scratch: fp64 [T, E] (rows indexed by position in the refine list).
+// Exact re-decision of the listed tokens.  refine_cand null: every listed
+// token is re-decided over all experts (the unfused path lists no
+// candidates).
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
                           int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          double* exact_scratch, int32_t* topk_idx, float* topk_w, int sms,
+                          const int32_t* refine_cand, int32_t* topk_idx, float* topk_w, int sms,
                           cudaStream_t stream);
 
 // logits[t, e] += offset[e]

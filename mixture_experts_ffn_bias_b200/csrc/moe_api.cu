@@ -16,8 +16,8 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
-  size_t status, blk, offsets, slot_pos, perm_src, refine, logits, x_perm, h, y_perm, h_sh, y_sh,
-      total;
+  size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, logits, x_perm, h,
+      y_perm, h_sh, y_sh, total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -34,6 +34,7 @@ Layout layout(const moe_config& c) {
   L.slot_pos = o; o += up(R * 4);
   L.perm_src = o; o += up(R * 4);
   L.refine = o;   o += up(T * 4);
+  L.refine_cand = o; o += up(T * moe::kRefineCand * 4);
   L.logits = o;   o += up(T * E * 8);
   L.x_perm = o;   o += up(R * d * es);
   L.h = o;        o += up(R * F * es);
@@ -109,10 +110,12 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
     float* logits = at<float>(ws, L.logits);
     int32_t* count = at<int32_t>(ws, L.status) + 1;
     int32_t* list = at<int32_t>(ws, L.refine);
-    if (moe::router_fused_supported(c->n_experts, c->top_k)) {
+    const bool fused = moe::router_fused_supported(c->n_experts, c->top_k);
+    int32_t* cand = at<int32_t>(ws, L.refine_cand);
+    if (fused) {
       MOE_TRY(moe::router_topk_tc(x, c->T, w_router, c->n_experts, c->d_model, logit_offset,
                                   sel_bias, c->top_k, c->gate, c->norm_topk_prob, topk_idx,
-                                  topk_w, count, list, at<uint32_t>(ws, L.status), s));
+                                  topk_w, count, list, cand, at<uint32_t>(ws, L.status), s));
     } else {
       MOE_TRY(moe::router_logits_tc(x, c->T, w_router, c->n_experts, c->d_model, logits,
                                     at<uint32_t>(ws, L.status), s));
@@ -120,11 +123,9 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
                                       c->top_k, c->gate, c->norm_topk_prob, topk_idx, topk_w,
                                       count, list, s));
     }
-    // the fp32 logits (unfused path) are consumed before the exact logits of
-    // the listed tokens reuse the same scratch region
     MOE_TRY(moe::router_refine(x, w_router, logit_offset, sel_bias, c->T, c->d_model,
                                c->n_experts, c->top_k, c->gate, c->norm_topk_prob, count, list,
-                               at<double>(ws, L.logits), topk_idx, topk_w, device_sms(), s));
+                               fused ? cand : nullptr, topk_idx, topk_w, device_sms(), s));
     return MOE_OK;
   }
   double* logits = at<double>(ws, L.logits);

@@ -307,90 +307,163 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
   }
 }
 
-// Exact re-decision of the listed tokens, in two kernels.
-// router_refine_logits_kernel: blocks are (listed token, chunk of 16
-// experts); the token's x row is staged in shared memory as fp32, each warp
-// computes two experts' exact logits (bf16 x bf16 products are exact in fp32,
-// the sums run in fp64) from coalesced 16-byte reads of the router rows, and
-// writes them to exact[i, e] (fp64 scratch, i = position in the list).
-// Spreading one token's experts over several blocks keeps the per-token
-// latency low when only a handful of tokens are listed.
-constexpr int kRefineExperts = 16;
-
-__global__ void __launch_bounds__(256)
-router_refine_logits_kernel(const __nv_bfloat16* __restrict__ x,
-                            const __nv_bfloat16* __restrict__ wr,
-                            const float* __restrict__ offset, int d, int E,
-                            const int32_t* __restrict__ refine_count,
-                            const int32_t* __restrict__ refine_list,
-                            double* __restrict__ exact) {
-  extern __shared__ float4 s_x4[];           // d floats
-  const float* s_x = reinterpret_cast<const float*>(s_x4);
-  const int n = *refine_count;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int e0 = blockIdx.y * kRefineExperts + warp;
-  const int e1 = e0 + 8;
-  for (int i = blockIdx.x; i < n; i += gridDim.x) {
-    const int t = refine_list[i];
-    __syncthreads();
-    for (int c = threadIdx.x; c < d; c += blockDim.x)
-      reinterpret_cast<float*>(s_x4)[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
-    __syncthreads();
-    if (e0 >= E) continue;
-    const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
-    const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1 < E ? e1 : e0) * d);
-    const float4* sx4 = reinterpret_cast<const float4*>(s_x);
-    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-    for (int c0 = lane * 8; c0 < d; c0 += 256) {
-      const uint4 u0 = __ldg(r0 + c0 / 8), u1 = __ldg(r1 + c0 / 8);
-      const float4 xa = sx4[c0 / 4], xb = sx4[c0 / 4 + 1];
-      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-      const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
-      const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+// Exact re-decision of a listed token: one block per listed token.  The
+// experts to decide over are the token's candidates (the experts whose fp32
+// key was within the margin of its (k+1)-th pick, which must contain the
+// exact top-k) or all experts.  Their exact logits are fp64 sums of exact
+// bf16 x bf16 products (x staged in shared memory as fp32, each warp reads
+// two router rows at a time with coalesced 16-byte loads).  Selection uses
+// the fp64 keys (ties to the lower expert id); the weights are formed in fp32
+// from the exact logits.
+__device__ void refine_select(const double* s_l, const int* s_e, int n, const float* bias,
+                              int k, int gate, int renorm, bool all_experts,
+                              int32_t* idx_row, float* w_row) {
+  const int lane = threadIdx.x & 31;
+  double key[kMaxPerLane];
+  float lf[kMaxPerLane];
+  int ex[kMaxPerLane];
+  bool taken[kMaxPerLane];
+  float m = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
-        b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    const int c = lane + 32 * j;
+    taken[j] = c >= n;
+    ex[j] = c < n ? s_e[c] : 0x7fffffff;
+    const double l = c < n ? s_l[c] : -INFINITY;
+    lf[j] = static_cast<float>(l);
+    key[j] = c < n ? l + (bias ? static_cast<double>(bias[ex[j]]) : 0.0) : -INFINITY;
+    m = fmaxf(m, lf[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float S = 1.0f;
+  if (gate == 0 && all_experts) {
+    S = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxPerLane; ++j)
+      if (lane + 32 * j < n) S += expf(lf[j] - m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  }
+  int my_idx = 0;
+  float my_s = 0.f, ssum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    double bk = -INFINITY;
+    int be = 0x7fffffff, bslot = 0;
+#pragma unroll
+    for (int q = 0; q < kMaxPerLane; ++q) {
+      if (!taken[q] && (key[q] > bk || (key[q] == bk && ex[q] < be))) {
+        bk = key[q];
+        be = ex[q];
+        bslot = q;
       }
     }
-    double s0 = (a[0] + a[1]) + (a[2] + a[3]);
-    double s1 = (b[0] + b[1]) + (b[2] + b[3]);
+    int owner = lane;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      const double ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const int ow = __shfl_xor_sync(0xffffffffu, owner, o);
+      const int os = __shfl_xor_sync(0xffffffffu, bslot, o);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+        owner = ow;
+        bslot = os;
+      }
     }
-    if (lane == 0) {
-      exact[static_cast<size_t>(i) * E + e0] = s0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
-      if (e1 < E)
-        exact[static_cast<size_t>(i) * E + e1] =
-            s1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+    float l = 0.f;
+#pragma unroll
+    for (int q = 0; q < kMaxPerLane; ++q) {
+      if (lane == owner && q == bslot) {
+        taken[q] = true;
+        l = lf[q];
+      }
     }
+    l = __shfl_sync(0xffffffffu, l, owner);
+    const float sc = gate == 1 ? 1.0f / (1.0f + expf(-l)) : expf(l - m) / S;
+    if (lane == j) {
+      my_idx = be;
+      my_s = sc;
+    }
+    ssum += sc;
+  }
+  if (lane < k) {
+    idx_row[lane] = my_idx;
+    w_row[lane] = renorm ? my_s / (ssum + 1e-9f) : my_s;
   }
 }
 
-// router_refine_select_kernel: one warp per listed token, fp64 selection on
-// the exact logits.
 __global__ void __launch_bounds__(256)
-router_refine_select_kernel(const double* __restrict__ exact, const float* __restrict__ bias,
-                            int E, int k, int gate, int renorm,
-                            const int32_t* __restrict__ refine_count,
-                            const int32_t* __restrict__ refine_list,
-                            int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  const int n = *refine_count;
-  const int lane = threadIdx.x & 31;
-  const int wpb = blockDim.x >> 5;
-  for (int i = blockIdx.x * wpb + (threadIdx.x >> 5); i < n; i += gridDim.x * wpb) {
+router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
+                     const float* __restrict__ offset, const float* __restrict__ bias, int d,
+                     int E, int k, int gate, int renorm, const int32_t* __restrict__ refine_count,
+                     const int32_t* __restrict__ refine_list,
+                     const int32_t* __restrict__ refine_cand, int32_t* __restrict__ topk_idx,
+                     float* __restrict__ topk_w) {
+  extern __shared__ float4 s_x4[];          // d floats
+  float* s_x = reinterpret_cast<float*>(s_x4);
+  __shared__ double s_l[256];
+  __shared__ int s_e[256];
+  __shared__ int s_n;
+  const int n_list = *refine_count;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = blockIdx.x; i < n_list; i += gridDim.x) {
     const int t = refine_list[i];
-    double l[kMaxPerLane];
-#pragma unroll
-    for (int j = 0; j < kMaxPerLane; ++j) {
-      const int e = lane + 32 * j;
-      l[j] = e < E ? exact[static_cast<size_t>(i) * E + e] : -INFINITY;
+    const int32_t* cand = refine_cand ? refine_cand + static_cast<size_t>(i) * kRefineCand : nullptr;
+    const bool all = cand == nullptr || cand[0] == -2;
+    if (threadIdx.x == 0) {
+      int n = E;
+      if (!all) {
+        n = 0;
+        while (n < kRefineCand && cand[n] >= 0) ++n;
+      }
+      s_n = n;
     }
-    warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
-                     topk_w + static_cast<size_t>(t) * k);
+    for (int c = threadIdx.x; c < 256; c += blockDim.x)
+      s_e[c] = all ? c : (c < kRefineCand ? cand[c] : -1);
+    for (int c = threadIdx.x; c < d; c += blockDim.x)
+      s_x[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
+    __syncthreads();
+    const int n = s_n;
+    const float4* sx4 = reinterpret_cast<const float4*>(s_x);
+    for (int c0 = warp; c0 < n; c0 += 16) {
+      const int c1 = c0 + 8;
+      const int e0 = s_e[c0], e1 = c1 < n ? s_e[c1] : e0;
+      const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
+      const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1) * d);
+      double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+      for (int col = lane * 8; col < d; col += 256) {
+        const uint4 u0 = __ldg(r0 + col / 8), u1 = __ldg(r1 + col / 8);
+        const float4 xa = sx4[col / 4], xb = sx4[col / 4 + 1];
+        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
+        const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          // bf16 x bf16 products are exact in fp32; the sums run in fp64
+          a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
+          b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
+        }
+      }
+      double s0 = (a[0] + a[1]) + (a[2] + a[3]);
+      double s1 = (b[0] + b[1]) + (b[2] + b[3]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      }
+      if (lane == 0) {
+        s_l[c0] = s0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
+        if (c1 < n) s_l[c1] = s1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+      }
+    }
+    __syncthreads();
+    if (warp == 0)
+      refine_select(s_l, s_e, n, bias, k, gate, renorm, all, topk_idx + static_cast<size_t>(t) * k,
+                    topk_w + static_cast<size_t>(t) * k);
+    __syncthreads();
   }
 }
 
@@ -448,27 +521,22 @@ cudaError_t router_select_fast(const float* logits, const float* logit_offset,
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
                           int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          double* exact_scratch, int32_t* topk_idx, float* topk_w, int sms,
+                          const int32_t* refine_cand, int32_t* topk_idx, float* topk_w, int sms,
                           cudaStream_t stream) {
-  const int gx = sms < T ? sms : T;
-  const dim3 grid(gx > 0 ? gx : 1, (E + kRefineExperts - 1) / kRefineExperts);
+  int grid = 2 * sms;
+  if (grid > T) grid = T;
+  if (grid < 1) grid = 1;
   const size_t smem = static_cast<size_t>(d) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_refine_logits_kernel,
+    cudaError_t e = cudaFuncSetAttribute(router_refine_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  router_refine_logits_kernel<<<grid, 256, smem, stream>>>(
+  router_refine_kernel<<<grid, 256, smem, stream>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
-      logit_offset, d, E, refine_count, refine_list, exact_scratch);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int warps = 8;
-  int gs = (T + warps - 1) / warps;
-  if (gs > sms) gs = sms > 0 ? sms : 1;
-  router_refine_select_kernel<<<gs, warps * 32, 0, stream>>>(
-      exact_scratch, sel_bias, E, k, gate, renorm, refine_count, refine_list, topk_idx, topk_w);
+      logit_offset, sel_bias, d, E, k, gate, renorm, refine_count, refine_list, refine_cand,
+      topk_idx, topk_w);
   return cudaGetLastError();
 }
 

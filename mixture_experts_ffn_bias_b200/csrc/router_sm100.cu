@@ -11,18 +11,20 @@
 // registers while the MMAs of the next chunks run.  This keeps the logit
 // error in the low 1e-6 range, far inside the router's re-decision margin.
 //
-// With up to 128 experts and top-k <= 8 the epilogue thread that owns a
-// token's row also takes the routing decision (fused select): it holds all of
-// the token's logits in registers, forms the gate statistics and the
-// selection keys, picks the top-(k+1) keys (descending, ties to the lower
-// expert id) and either writes the token's experts and weights or, when two
-// of those keys lie within kRefineMargin of each other, lists the token for
-// the exact re-decision kernel.  Otherwise the logits are written out and
-// router_select_fast_kernel decides.
+// With up to 128 experts and top-k <= 8 the routing decision is taken in the
+// same kernel (fused select): the epilogue thread that owns a token's row holds
+// all of its logits in registers, forms the gate statistics and the selection
+// keys and picks the top-(k+1) keys (descending, ties to the lower expert id;
+// a rolled round loop with four independent arg-max chains, the logits kept
+// in the thread's shared-memory column).  A token whose picked keys hold two keys
+// closer than kRefineMargin is not decided here: it is listed together with
+// its candidate experts (every expert whose key is within the margin of the
+// (k+1)-th pick), and router_refine_kernel decides it on exact logits.
+// Otherwise the logits are written out and router_select_fast_kernel decides.
 //
-// Warp roles (one 128-token tile at a time, persistent over tiles):
+// Warp roles (persistent over 128-token tiles):
 //   warp 0        TMA: x tile 128 x 64 and Wr tile NPAD x 64 per stage
-//   warp 1        TMEM allocation, one lane issues tcgen05.mma into a ring of
+//   warp 1        TMEM allocation; one lane issues tcgen05.mma into a ring of
 //                 NSLOT accumulator slots (one slot per K chunk)
 //   warps 2..     epilogue: one accumulator row per thread, NPAD <= 128
 //                 columns per warpgroup (two warpgroups for NPAD = 256)
@@ -52,7 +54,7 @@ struct RCfg {
   static constexpr int STAGE_BYTES = R_A_BYTES + B_BYTES;
   // fused select keeps each token's logits in a shared-memory column
   static constexpr int LOGIT_BYTES = FUSED ? NPAD * 128 * 4 : 0;
-  static constexpr int STAGE_BUDGET = 196608 - LOGIT_BYTES;
+  static constexpr int STAGE_BUDGET = 212992 - LOGIT_BYTES;   // 208 KB of stages + logit column
   static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
   static constexpr int NSLOT = (512 / NPAD) > 8 ? 8 : (512 / NPAD);
   static constexpr int TMEM_RAW = NSLOT * NPAD;
@@ -71,7 +73,8 @@ struct RouterOut {
   int32_t* topk_idx;             // fused outputs
   float* topk_w;
   int32_t* refine_count;
-  int32_t* refine_list;
+  int32_t* refine_list;          // [T] listed tokens
+  int32_t* refine_cand;          // [T, kRefineCand] candidate experts (-1 pad, -2 = all)
   uint32_t* status;
 };
 
@@ -141,7 +144,26 @@ __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int*
     s_seli[j * 128] = bi[0];
   }
   if (min_gap < kRefineMargin) {
-    o.refine_list[atomicAdd(o.refine_count, 1)] = t;
+    // list the token with its candidate experts: every expert whose key is
+    // within the margin of the last pick (the exact top-k is among them);
+    // softmax without renormalisation needs all exact logits
+    const int slot = atomicAdd(o.refine_count, 1);
+    o.refine_list[slot] = t;
+    int32_t* cand = o.refine_cand + static_cast<size_t>(slot) * kRefineCand;
+    const float lo = pv - kRefineMargin;
+    int n = (o.gate == 0 && !o.renorm) ? kRefineCand + 1 : 0;
+#pragma unroll
+    for (int i = 0; i < COLS; ++i) {
+      if (acc[i] >= lo) {
+        if (n < kRefineCand) cand[n] = i;
+        ++n;
+      }
+    }
+    if (n > kRefineCand) {
+      cand[0] = -2;
+      n = 1;
+    }
+    for (int c = n; c < kRefineCand; ++c) cand[c] = -1;
     return;
   }
   float sc[KMAX_FUSED];
@@ -433,7 +455,8 @@ cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, 
   if (npad > 256) return cudaErrorInvalidValue;
   CUtensorMap mx, mw;
   if (!maps(x, T, w_router, E, K, &mx, &mw)) return cudaErrorInvalidValue;
-  RouterOut o{logits, nullptr, nullptr, 0, 0, 0, nullptr, nullptr, nullptr, nullptr, status};
+  RouterOut o{logits, nullptr, nullptr, 0, 0, 0, nullptr, nullptr, nullptr, nullptr, nullptr,
+              status};
   switch (npad) {
     case 16: return launch_router<16, false>(mx, mw, T, K, E, o, stream);
     case 32: return launch_router<32, false>(mx, mw, T, K, E, o, stream);
@@ -446,13 +469,14 @@ cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, 
 cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, int K,
                            const float* logit_offset, const float* sel_bias, int k, int gate,
                            int renorm, int32_t* topk_idx, float* topk_w, int32_t* refine_count,
-                           int32_t* refine_list, uint32_t* status, cudaStream_t stream) {
+                           int32_t* refine_list, int32_t* refine_cand, uint32_t* status,
+                           cudaStream_t stream) {
   if (T <= 0) return cudaSuccess;
   if (!router_fused_supported(E, k)) return cudaErrorInvalidValue;
   CUtensorMap mx, mw;
   if (!maps(x, T, w_router, E, K, &mx, &mw)) return cudaErrorInvalidValue;
   RouterOut o{nullptr, logit_offset, sel_bias, k, gate, renorm, topk_idx, topk_w,
-              refine_count, refine_list, status};
+              refine_count, refine_list, refine_cand, status};
   switch (npad_for(E)) {
     case 16: return launch_router<16, true>(mx, mw, T, K, E, o, stream);
     case 32: return launch_router<32, true>(mx, mw, T, K, E, o, stream);
