@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -78,7 +79,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// One warp computes per-group tile prefixes: prefix[g] = sum_{g' < g} m_tiles(g') * n_tiles.
+// One warp computes per-group tile prefixes: prefix[g] = sum_{g' < g} m_tiles(g') * n_tiles,
+// with m-tiles of TM rows.
+template <int TM = BM>
 __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, int* s_prefix) {
   const int lane = threadIdx.x & 31;
   const int G = a.num_groups;
@@ -87,7 +90,7 @@ __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, in
       s_off[0] = 0;
       s_off[1] = a.rows_single;
       s_prefix[0] = 0;
-      s_prefix[1] = ((a.rows_single + BM - 1) / BM) * n_tiles;
+      s_prefix[1] = ((a.rows_single + TM - 1) / TM) * n_tiles;
     }
     __syncwarp();
     return;
@@ -99,7 +102,7 @@ __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, in
   int local = 0;
   for (int g = g0; g < g0 + per && g < G; ++g) {
     const int rows = s_off[g + 1] - s_off[g];
-    local += ((rows > 0 ? rows : 0) + BM - 1) / BM * n_tiles;
+    local += ((rows > 0 ? rows : 0) + TM - 1) / TM * n_tiles;
   }
   int incl = local;
 #pragma unroll
@@ -111,7 +114,7 @@ __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, in
   for (int g = g0; g < g0 + per && g < G; ++g) {
     s_prefix[g] = run;
     const int rows = s_off[g + 1] - s_off[g];
-    run += ((rows > 0 ? rows : 0) + BM - 1) / BM * n_tiles;
+    run += ((rows > 0 ? rows : 0) + TM - 1) / TM * n_tiles;
   }
   if (lane == 31) s_prefix[G] = incl;
   __syncwarp();
@@ -122,10 +125,11 @@ __device__ void build_tile_prefix(const GemmArgs& a, int n_tiles, int* s_off, in
 // weights fit in L2 many times over.  m fastest: they share B tiles instead,
 // so an expert whose weights are a large part of L2 is streamed from HBM
 // once while its (smaller) rows are re-read from L2.
+template <int TM = BM>
 __device__ __forceinline__ void tile_mn(int local, int rows_g, int n_tiles, int m_fastest,
                                         int& m, int& n) {
   if (m_fastest) {
-    const int mt = (rows_g + BM - 1) / BM;
+    const int mt = (rows_g + TM - 1) / TM;
     n = local / mt;
     m = local - n * mt;
   } else {
@@ -435,6 +439,266 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   }
 }
 
+// --------------------------------------------------- CTA-pair (2-SM) kernel
+// The same grouped GEMM with a cluster of two CTAs per 256 x BN_ACC tile:
+// rank r holds rows [128 r, 128 r + 128) of the A tile and half of the B tile
+// (SwiGLU: rank 0 the W1 rows, rank 1 the W3 rows; plain: rows
+// [r BN_ACC/2, (r+1) BN_ACC/2)), so each SM stages half the B bytes of the
+// single-CTA kernel per MMA flop.  Rank 0 issues tcgen05.mma.cta_group::2
+// (M = 256), which reads both CTAs' shared memory and writes each CTA's 128
+// accumulator rows into its own TMEM; commits arrive on both CTAs'
+// barriers.  Both CTAs' TMA completions are counted on rank 0's stage
+// barrier.  No load uses cluster multicast.
+constexpr int BM2 = 256;
+
+template <int BN_ACC>
+struct PairCfg {
+  static constexpr int B_HALF_BYTES = (BN_ACC / 2) * BK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_HALF_BYTES;
+  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+  static constexpr int TMEM_COLS = 2 * BN_ACC;
+  static constexpr int EPI_BYTES = 4 * 32 * 128;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+};
+
+template <int BN_ACC, int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmB1,
+                         const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using Cfg = PairCfg<BN_ACC>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
+  constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM2, BN_ACC);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smemA = smem;
+  uint8_t* smemB = smem + STAGES * A_STAGE_BYTES;
+  uint8_t* smemEpi = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smemEpi + Cfg::EPI_BYTES);
+  uint64_t* full_bar = bars;                   // rank 0's copy is used
+  uint64_t* empty_bar = bars + STAGES;         // both copies
+  uint64_t* tfull_bar = bars + 2 * STAGES;     // both copies
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;  // rank 0's copy (8 arrivals)
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+
+  __shared__ int s_off[MAX_GROUPS + 1];
+  __shared__ int s_prefix[MAX_GROUPS + 1];
+  __shared__ uint32_t s_tmem_base;
+  __shared__ int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+  const int n_tiles = args.n_per_group / BN_OUT;
+  const int G = args.offsets == nullptr ? 1 : args.num_groups;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);
+    }
+    mbar_init(drain_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (SWIGLU) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(&s_tmem_base, Cfg::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 2) build_tile_prefix<BM2>(args, n_tiles, s_off, s_prefix);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();        // both CTAs' barriers are initialised
+  tc_fence_after();
+
+  const uint32_t tmem_base = s_tmem_base;
+  const int total_tiles = s_prefix[G];
+  volatile int* abort_flag = &s_abort;
+  const int kblocks = args.K / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += npairs) {
+        const int g = find_group(s_prefix, G, tile);
+        int m, n;
+        tile_mn<BM2>(tile - s_prefix[g], s_off[g + 1] - s_off[g], n_tiles, args.m_fastest, m, n);
+        const int arow = s_off[g] + m * BM2 + static_cast<int>(rank) * BM;
+        const int brow = SWIGLU ? g * args.n_per_group + n * BN_OUT
+                                : g * args.n_per_group + n * BN_OUT + static_cast<int>(rank) * (BN_ACC / 2);
+        const CUtensorMap* mb = (SWIGLU && rank == 1) ? &tmB1 : &tmB0;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
+          tma_load_2d_pair(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
+          tma_load_2d_pair(smemB + stage * Cfg::B_HALF_BYTES, mb, &full_bar[stage], kb * BK, brow);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        // rank 0's stage barriers count both CTAs' copies: let them all land
+        for (int s = 0; s < STAGES; ++s) {
+          if (!(issued_mask & (1u << s))) continue;
+          const uint32_t par = (issued_phase >> s) & 1u;
+          const unsigned long long t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full_bar[s], par))
+            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer (rank 0)
+    if (lane == 0 && rank == 0) {
+      int stage = 0, it = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued_any = false;
+      for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN_ACC;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smemA + stage * A_STAGE_BYTES);
+          const uint32_t b_addr = smem_u32(smemB + stage * Cfg::B_HALF_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc_mma_f16_pair(d_tmem, smem_desc_sw128(a_addr + kk * 32),
+                            smem_desc_sw128(b_addr + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
+          issued_any = true;
+          tc_commit_pair(&empty_bar[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(&tfull_bar[acc]);
+      }
+      if (!ok && issued_any) {
+        tc_commit_pair(drain_bar);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int g = find_group(s_prefix, G, tile);
+      const int rows_g = s_off[g + 1] - s_off[g];
+      int m, n;
+      tile_mn<BM2>(tile - s_prefix[g], rows_g, n_tiles, args.m_fastest, m, n);
+      const int r0 = m * BM2 + static_cast<int>(rank) * BM;   // first row (in group) of this CTA
+      const bool valid = (r0 + row) < rows_g;
+      const bool warp_full = (r0 + q * 32 + 32) <= rows_g;
+      const int warp_row0 = s_off[g] + r0 + q * 32;
+      uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
+      const size_t crow_off = static_cast<size_t>(s_off[g] + r0 + row) * args.ldc +
+                              static_cast<size_t>(n) * BN_OUT;
+      const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int cb = 0; cb < BN_OUT / 64; ++cb) {
+        uint32_t packed[32];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int c0 = cb * 64 + half * 32;
+          uint32_t v[32];
+          if (SWIGLU) {
+            uint32_t u[32];
+            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_ld16(t_addr + BN_OUT + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+            tmem_ld16(t_addr + BN_OUT + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 =
+                  silu_f32(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              packed[half * 16 + i] = pack_bf16x2(h0, h1);
+            }
+          } else {
+            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[half * 16 + i] =
+                  pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          }
+        }
+        if (warp_full) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stage_buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                           packed[4 * c + 3]);
+          fence_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, stage_buf, n * BN_OUT + cb * 64, warp_row0);
+            bulk_commit();
+          }
+        } else if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
+                                                cb * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
+                                packed[4 * c + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_rank0(&tempty_bar[acc]);
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();        // neither CTA leaves while the other still uses the pair
+  if (threadIdx.x == 0 && s_abort) atomicOr(args.status, kDevTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
 // ----------------------------------------------------------------- host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -509,6 +773,45 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   return cudaGetLastError();
 }
 
+template <int BN_ACC, int MODE>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const CUtensorMap& c, const GemmArgs& args, int rows_upper,
+                        cudaStream_t stream) {
+  using Cfg = PairCfg<BN_ACC>;
+  constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
+  auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE>;
+  static unsigned long long attr_done = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(attr_done & bit)) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done |= bit;
+  }
+  const int G = args.offsets == nullptr ? 1 : args.num_groups;
+  GemmArgs a2 = args;
+  const double b_bytes = static_cast<double>(BN_OUT == BN_ACC ? args.n_per_group
+                                                              : 2 * args.n_per_group) *
+                         args.K * 2.0;
+  a2.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
+  const long long m_tiles_upper = (rows_upper + BM2 - 1) / BM2 + (G > 1 ? G : 0);
+  const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
+  if (tiles_upper <= 0) return cudaSuccess;
+  const int max_pairs = num_sms() / 2;
+  const int pairs = static_cast<int>(tiles_upper < max_pairs ? tiles_upper : max_pairs);
+  kern<<<2 * pairs, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, a2);
+  return cudaGetLastError();
+}
+
+// The CTA-pair kernel is the default; MOE_B200_GEMM_1SM=1 selects the
+// single-CTA kernel.
+bool use_pair() {
+  const char* v = std::getenv("MOE_B200_GEMM_1SM");
+  return !(v != nullptr && v[0] == '1');
+}
+
 }  // namespace
 
 // h[r] = silu(A[r] W1[g]^T) * (A[r] W3[g]^T), bf16 out.
@@ -524,6 +827,8 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (use_pair())
+    return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
   return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
 }
 
@@ -552,11 +857,18 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
   const int64_t c_rows = offsets ? a_rows : rows_single;
   const int bn = (N % 256 == 0) ? 256 : 128;
-  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn) ||
+  const bool pair = use_pair();
+  // the pair kernel's CTAs each load half of the B tile
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, pair ? bn / 2 : bn) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (pair) {
+    if (bn == 256)
+      return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+    return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+  }
   if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
   return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
 }

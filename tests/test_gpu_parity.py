@@ -97,6 +97,16 @@ def test_forward_with_gathered_gate_up_rows(name, monkeypatch):
     _check_layer(shape, host, _run(shape, host))
 
 
+@pytest.mark.parametrize("name", ["page2_small", "qwen3_small", "wide_small"])
+def test_forward_with_single_cta_gemm(name, monkeypatch):
+    """The single-CTA grouped GEMM (MOE_B200_GEMM_1SM=1) beside the default
+    CTA-pair kernel."""
+    monkeypatch.setenv("MOE_B200_GEMM_1SM", "1")
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
+
+
 def test_skew_bias_update_then_deferred_forward():
     """Skewed workload: forward, bias update from its counts (bit-exact), then a
     second forward routes with the new bias (the update lands on the next
