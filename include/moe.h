@@ -241,6 +241,15 @@ moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
  * Diagnostic only; 0 for fp32 layers. */
 moe_status moe_router_refined_tokens(void* ws, size_t ws_bytes, void* stream, int32_t* count);
 
+/* Diagnostic: launch a kernel that waits on a barrier phase nothing
+ * completes, using the same bounded wait as the tensor-core kernels, with a
+ * limit of limit_seconds (0 < limit <= 2).  The wait gives up, the kernel
+ * records the timeout in the status word of ws (>= 256 bytes, 256-byte
+ * aligned) and returns; moe_device_status then reports MOE_ERR_TIMEOUT and
+ * the context stays usable.  Has no counterpart on the pages. */
+moe_status moe_selftest_bounded_wait(void* ws, size_t ws_bytes, double limit_seconds,
+                                     void* stream);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status s);
 

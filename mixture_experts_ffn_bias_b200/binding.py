@@ -66,6 +66,7 @@ _SIGNATURES = {
     "moe_permute_noalloc": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_device_status": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_router_refined_tokens": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_int32)]),
+    "moe_selftest_bounded_wait": (_I32, [_VP, _SZ, _F64, _VP]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
 }
 
@@ -241,3 +242,9 @@ def moe_router_refined_tokens(ws, stream=None) -> int:
     c = ctypes.c_int32(0)
     _check(lib().moe_router_refined_tokens(_p(ws), _nbytes(ws), _s(stream), ctypes.byref(c)), True)
     return int(c.value)
+
+
+def moe_selftest_bounded_wait(ws, limit_seconds=0.05, stream=None, check=True) -> int:
+    """Run the bounded-wait self-test kernel (returns after limit_seconds)."""
+    st = lib().moe_selftest_bounded_wait(_p(ws), _nbytes(ws), float(limit_seconds), _s(stream))
+    return _check(st, check)

@@ -398,3 +398,16 @@ def test_bias_update_call_bit_exact(E):
         B.moe_bias_update(cfg, c_d, b_d, rate, 0.1, 0.5, 10.0)
         torch.cuda.synchronize()
         np.testing.assert_array_equal(_np(b_d), O.bias_update(counts, bias, rate, 0.1, 0.5, 10.0))
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """A wait on a barrier nothing completes runs out after 50 ms; the host
+    reads MOE_ERR_TIMEOUT from the status word and the context still works."""
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    B.moe_selftest_bounded_wait(ws, 0.05)
+    st, flags = B.moe_device_status(ws)
+    assert st == B.MOE_ERR_TIMEOUT and flags & 2
+    assert B.moe_device_status(ws)[0] == B.MOE_OK      # read clears the word
+    shape = SMALL["qwen3_small"].replace(T=64)
+    host = I.make_inputs(shape)
+    _check_layer(shape, host, _run(shape, host))
