@@ -126,6 +126,22 @@ moe_status moe_router_logits(const moe_config* cfg, const void* x, const void* w
                              const float* logit_offset, float* logits,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* Router losses and health metrics for a batch and its routing (the aux
+ * dict of SigmoidRouter.forward, "moe-200m-qwen3-100b" README; load metrics
+ * of SpecForge PR #931, "What to watch").  Recomputes the logits
+ * (tensor cores for bf16) and reads topk_idx [T, k] (e.g. from
+ * moe_router_topk).  stats: 8 floats on the device:
+ *   [0] z_loss = mean_t logsumexp_e(logits)^2
+ *   [1] aux_loss = E * sum_e (fraction of tokens choosing e) * (mean score of e)
+ *   [2] cv = std(counts, Bessel) / max(mean(counts), 1)   (NaN for E = 1)
+ *   [3] entropy of the normalised mean scores, in bits
+ *   [4] load_max_ratio = max(counts) / mean(counts)   (ceiling E / k)
+ *   [5] fraction of experts with no tokens;  [6], [7] = 0.
+ * Deterministic (fixed reduction order). */
+moe_status moe_router_stats(const moe_config* cfg, const void* x, const void* w_router,
+                            const float* logit_offset, const int32_t* topk_idx, float* stats,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /* Dispatch: per-expert counts, offsets, and the stable expert-contiguous
  * permutation of the T*k routed rows, with x gathered into that order.
  * (Grouped-GEMM dispatch, SpecForge PR #930 "Why FSDP is enough here" and
@@ -177,6 +193,14 @@ moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t*
 moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* sel_bias,
                            double rate, double starved_frac, double starved_add,
                            double clamp, void* stream);
+
+/* Selection-bias update of the noaux_tc kind: one fixed step per call
+ * (micro-batch) toward balance, fp32, in place, no clamp:
+ *   bias_e += fp32(rate) * sign(fp32(sum c) / E - c_e)      (sign(0) = 0).
+ * SpecForge PR #931, "What to watch": at rate 0.001 and 64 accumulation
+ * steps a starved expert's bias grows 0.064 per optimizer step. */
+moe_status moe_bias_update_sign(const moe_config* cfg, const int32_t* counts, float* sel_bias,
+                                double rate, void* stream);
 
 /* The whole layer forward: router, dispatch, grouped SwiGLU experts (+ shared
  * expert), combine.  Inputs as above; out [T, d] act.  Also returns the

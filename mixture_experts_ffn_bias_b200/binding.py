@@ -56,10 +56,12 @@ _SIGNATURES = {
     "moe_check_config": (_I32, [_CFG]),
     "moe_router_topk": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_router_logits": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_router_stats": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_swiglu": (_I32, [_CFG, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_bias_update": (_I32, [_CFG, _VP, _VP, _F64, _F64, _F64, _F64, _VP]),
+    "moe_bias_update_sign": (_I32, [_CFG, _VP, _VP, _F64, _VP]),
     "moe_forward": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_forward_profiled": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ,
                                      _VP, ctypes.POINTER(ctypes.c_void_p)]),
@@ -163,6 +165,17 @@ def moe_router_logits(cfg, x, w_router, logit_offset, logits, ws, stream=None, c
     return _check(st, check)
 
 
+def moe_router_stats(cfg, x, w_router, logit_offset, topk_idx, stats, ws, stream=None,
+                     check=True) -> int:
+    st = lib().moe_router_stats(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_offset),
+                                _p(topk_idx), _p(stats), _p(ws),
+                                _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+STAT_NAMES = ("z_loss", "aux_loss", "cv", "entropy_bits", "load_max_ratio", "unused_frac")
+
+
 def moe_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src, x_perm, ws,
                 stream=None, check=True) -> int:
     st = lib().moe_permute(ctypes.byref(cfg), _p(topk_idx), _p(x), _p(counts), _p(offsets),
@@ -199,6 +212,11 @@ def moe_bias_update(cfg, counts, sel_bias, rate=1e-3, starved_frac=0.1, starved_
                     clamp=10.0, stream=None, check=True) -> int:
     st = lib().moe_bias_update(ctypes.byref(cfg), _p(counts), _p(sel_bias), rate,
                                starved_frac, starved_add, clamp, _s(stream))
+    return _check(st, check)
+
+
+def moe_bias_update_sign(cfg, counts, sel_bias, rate=1e-3, stream=None, check=True) -> int:
+    st = lib().moe_bias_update_sign(ctypes.byref(cfg), _p(counts), _p(sel_bias), rate, _s(stream))
     return _check(st, check)
 
 

@@ -153,6 +153,30 @@ bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias,
   }
 }
 
+// noaux_tc-style update (SpecForge PR #931, "What to watch": a fixed step
+// per micro-batch): bias_e += rate * sign(mean(c) - c_e), fp32.
+__global__ void __launch_bounds__(256)
+bias_update_sign_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias, int E,
+                        float rate) {
+  __shared__ long long s_part[8];
+  const int tid = threadIdx.x;
+  long long c_sum = 0;
+  for (int e = tid; e < E; e += 256) c_sum += counts[e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c_sum += __shfl_xor_sync(0xffffffffu, c_sum, o);
+  if ((tid & 31) == 0) s_part[tid >> 5] = c_sum;
+  __syncthreads();
+  long long total_i = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) total_i += s_part[w];
+  const float mean = __fdiv_rn(__ll2float_rn(total_i), __int2float_rn(E));
+  for (int e = tid; e < E; e += 256) {
+    const float d = __fsub_rn(mean, __int2float_rn(counts[e]));
+    const float step = d > 0.f ? rate : (d < 0.f ? -rate : 0.f);
+    bias[e] = __fadd_rn(bias[e], step);
+  }
+}
+
 }  // namespace
 
 template <bool BF16>
@@ -187,6 +211,12 @@ cudaError_t bias_update(const int32_t* counts, float* bias, int E, float target,
                         float starved_add, float rate, float clamp, cudaStream_t stream) {
   bias_update_kernel<<<1, 256, 0, stream>>>(counts, bias, E, target, thresh, starved_add, rate,
                                             clamp);
+  return cudaGetLastError();
+}
+
+cudaError_t bias_update_sign(const int32_t* counts, float* bias, int E, float rate,
+                             cudaStream_t stream) {
+  bias_update_sign_kernel<<<1, 256, 0, stream>>>(counts, bias, E, rate);
   return cudaGetLastError();
 }
 

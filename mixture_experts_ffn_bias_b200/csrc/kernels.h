@@ -56,6 +56,13 @@ cudaError_t router_refine(const void* x, const void* w_router, const float* logi
 // logits[t, e] += offset[e]
 cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream);
 
+// Router statistics --------------------------------------------------------
+int stats_blocks(int T);
+// partials: fp64 [stats_blocks(T), 2E+1]; out: float[8] on the device.
+cudaError_t router_stats(bool fp64_logits, const void* logits, int T, int E, int gate,
+                         const int32_t* topk_idx, int k, double* partials, float* out,
+                         cudaStream_t stream);
+
 // Dispatch -------------------------------------------------------------------
 constexpr int kRankBlock = 256;   // tokens per histogram block
 inline int rank_blocks(int T) { return (T + kRankBlock - 1) / kRankBlock; }
@@ -96,5 +103,7 @@ cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, cons
                     const void* y_shared, void* out, int T, int d, int k, cudaStream_t stream);
 cudaError_t bias_update(const int32_t* counts, float* bias, int E, float target, float thresh,
                         float starved_add, float rate, float clamp, cudaStream_t stream);
+cudaError_t bias_update_sign(const int32_t* counts, float* bias, int E, float rate,
+                             cudaStream_t stream);
 
 }  // namespace moe

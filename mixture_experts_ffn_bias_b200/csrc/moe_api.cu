@@ -16,8 +16,8 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
-  size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, logits, x_perm, h,
-      y_perm, h_sh, y_sh, total;
+  size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, stats, logits, x_perm,
+      h, y_perm, h_sh, y_sh, total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -35,6 +35,7 @@ Layout layout(const moe_config& c) {
   L.perm_src = o; o += up(R * 4);
   L.refine = o;   o += up(T * 4);
   L.refine_cand = o; o += up(T * moe::kRefineCand * 4);
+  L.stats = o;    o += up(static_cast<size_t>(moe::stats_blocks(c.T)) * (2 * E + 1) * 8);
   L.logits = o;   o += up(T * E * 8);
   L.x_perm = o;   o += up(R * d * es);
   L.h = o;        o += up(R * F * es);
@@ -329,6 +330,40 @@ moe_status moe_router_logits(const moe_config* cfg, const void* x, const void* w
   return MOE_OK;
 }
 
+moe_status moe_router_stats(const moe_config* cfg, const void* x, const void* w_router,
+                            const float* logit_offset, const int32_t* topk_idx, float* stats,
+                            void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!stats || !aligned4(stats)) return MOE_ERR_INVALID;
+  if (cfg->T == 0) {
+    MOE_TRY(cudaMemsetAsync(stats, 0, 8 * sizeof(float), S(stream)));
+    return MOE_OK;
+  }
+  if (!x || !w_router || !topk_idx || !aligned16(x) || !aligned16(w_router) ||
+      !aligned4(topk_idx) || (logit_offset && !aligned4(logit_offset)))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  const Layout L = layout(*cfg);
+  cudaStream_t s = S(stream);
+  if ((st = clear_status(ws, s)) != MOE_OK) return st;
+  void* logits = at<void>(ws, L.logits);
+  const bool bf16 = cfg->dtype == MOE_BF16;
+  if (bf16) {
+    MOE_TRY(moe::router_logits_tc(x, cfg->T, w_router, cfg->n_experts, cfg->d_model,
+                                  static_cast<float*>(logits), at<uint32_t>(ws, 0), s));
+    if (logit_offset)
+      MOE_TRY(moe::add_row_offset(static_cast<float*>(logits), logit_offset, cfg->T,
+                                  cfg->n_experts, s));
+  } else {
+    MOE_TRY(moe::router_logits(false, x, w_router, logit_offset, cfg->T, cfg->d_model,
+                               cfg->n_experts, static_cast<double*>(logits), s));
+  }
+  MOE_TRY(moe::router_stats(!bf16, logits, cfg->T, cfg->n_experts, cfg->gate, topk_idx,
+                            cfg->top_k, at<double>(ws, L.stats), stats, s));
+  return MOE_OK;
+}
+
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* x,
                        int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_src,
                        void* x_perm, void* ws, size_t ws_bytes, void* stream) {
@@ -397,6 +432,16 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* 
                            static_cast<float>(starved_frac * inv_e),
                            static_cast<float>(starved_add), static_cast<float>(rate),
                            static_cast<float>(clamp), S(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_bias_update_sign(const moe_config* cfg, const int32_t* counts, float* sel_bias,
+                                double rate, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!counts || !sel_bias || !aligned4(counts) || !aligned4(sel_bias)) return MOE_ERR_INVALID;
+  MOE_TRY(moe::bias_update_sign(counts, sel_bias, cfg->n_experts, static_cast<float>(rate),
+                                S(stream)));
   return MOE_OK;
 }
 

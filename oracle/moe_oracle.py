@@ -271,3 +271,58 @@ def bias_update(counts, sel_bias, rate: float = 1e-3, starved_frac: float = 0.1,
     b = (b + step).astype(f32)
     b = np.minimum(np.maximum(b, f32(-clamp)), f32(clamp)).astype(f32)
     return b
+
+
+def bias_update_sign(counts, sel_bias, rate: float = 1e-3) -> np.ndarray:
+    """Aux-loss-free bias update of the noaux_tc kind, one micro-batch, float32.
+
+    SpecForge PR #931, "What to watch": with rate 0.001 and 64 accumulation
+    steps per optimizer step (its setup) the selection bias "grows linearly
+    (0.064/step at this accumulation)", i.e. every micro-batch moves a bias
+    by a fixed step toward balance:
+        bias_e += rate * sign(mean(c) - c_e)      (sign(0) = 0, no clamp)
+    mean(c) = fp32(sum c) / fp32(E), one fp32 operation per step.
+    """
+    f32 = np.float32
+    c = np.asarray(counts).astype(f32)
+    b = np.asarray(sel_bias, dtype=f32).copy()
+    mean = (f32(c.sum(dtype=f32)) / f32(c.size)).astype(f32)
+    d = (mean - c).astype(f32)
+    step = np.sign(d).astype(f32) * f32(rate)
+    return (b + step.astype(f32)).astype(f32)
+
+
+def router_stats(routing: Routing) -> dict:
+    """Router losses and health metrics, fp64.
+
+    "moe-200m-qwen3-100b" README, SigmoidRouter forward ("ST-MoE z-loss +
+    DeepSeek aux loss" and "Routing health metrics"):
+      z_loss       = mean_t (logsumexp_e logits[t, e])^2
+      aux_loss     = E * sum_e (one_hot.mean over tokens)_e * (scores.mean over tokens)_e
+      counts       = one_hot summed over tokens
+      cv           = std(counts) / max(mean(counts), 1)   (std with Bessel's correction,
+                                                          torch's default)
+      entropy_bits = -sum p log p / log 2 with p = max(mean scores, 1e-9), normalised
+    and SpecForge PR #931 ("What to watch"): load_max_ratio = max(counts) /
+    (mean counts) (ceiling E / k) and the fraction of experts with no tokens.
+    """
+    lg = routing.logits
+    T, E = lg.shape
+    m = lg.max(axis=1, keepdims=True)
+    lse = (m + np.log(np.exp(lg - m).sum(axis=1, keepdims=True)))[:, 0]
+    z_loss = float(np.mean(lse ** 2))
+    one_hot = np.zeros((T, E))
+    for j in range(routing.topk_idx.shape[1]):
+        one_hot[np.arange(T), routing.topk_idx[:, j]] += 1.0
+    p = routing.scores.mean(axis=0)
+    aux_loss = float(E * np.sum(one_hot.mean(axis=0) * p))
+    counts = one_hot.sum(axis=0)
+    cv = float(np.std(counts, ddof=1) / max(counts.mean(), 1.0)) if E > 1 else float("nan")
+    pa = np.maximum(p, 1e-9)
+    pa = pa / pa.sum()
+    entropy_bits = float(-np.sum(pa * np.log(pa)) / np.log(2.0))
+    mean_c = counts.sum() / E
+    load_max_ratio = float(counts.max() / mean_c) if mean_c > 0 else 0.0
+    unused = float(np.mean(counts == 0))
+    return {"z_loss": z_loss, "aux_loss": aux_loss, "cv": cv, "entropy_bits": entropy_bits,
+            "load_max_ratio": load_max_ratio, "unused_frac": unused, "counts": counts}

@@ -400,6 +400,45 @@ def test_bias_update_call_bit_exact(E):
         np.testing.assert_array_equal(_np(b_d), O.bias_update(counts, bias, rate, 0.1, 0.5, 10.0))
 
 
+@pytest.mark.parametrize("E", [16, 64, 128])
+def test_bias_update_sign_call_bit_exact(E):
+    """noaux_tc-style update: 64 calls on the GPU equal 64 oracle steps bitwise."""
+    rng = np.random.default_rng(100 + E)
+    counts = rng.integers(0, 900, E).astype(np.int32)
+    counts[:3] = [0, int(counts.mean()), 5000]
+    cfg = B.make_config(16, 128, E, 128, 1)
+    bias = rng.uniform(-1, 1, E).astype(np.float32)
+    c_d = torch.from_numpy(counts).cuda()
+    b_d = torch.from_numpy(bias.copy()).cuda()
+    ref = bias.copy()
+    for _ in range(64):
+        B.moe_bias_update_sign(cfg, c_d, b_d, 1e-3)
+        ref = O.bias_update_sign(counts, ref, 1e-3)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(_np(b_d), ref)
+
+
+@pytest.mark.parametrize("name", ["tiny", "page2_small", "qwen3_small", "skew_small"])
+def test_router_stats_call(name):
+    """Router losses and health metrics on the GPU vs the oracle (same routing)."""
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    r = P.oracle_routing(shape, host)
+    cfg, ws = _buffers(shape)
+    dt = torch.bfloat16 if shape.dtype == I.DTYPE_BF16 else torch.float32
+    x = to_device(host["x"], dt, "cuda")
+    wr = to_device(host["w_router"], dt, "cuda")
+    off = (to_device(host["logit_offset"], torch.float32, "cuda")
+           if "logit_offset" in host else None)
+    idx = torch.from_numpy(r.topk_idx.astype(np.int32)).cuda()
+    stats = torch.zeros(8, dtype=torch.float32, device="cuda")
+    B.moe_router_stats(cfg, x, wr, off, idx, stats, ws)
+    got = _np(stats)
+    ref = O.router_stats(r)
+    for i, key in enumerate(B.STAT_NAMES):
+        assert abs(got[i] - ref[key]) <= 1e-5 * max(1.0, abs(ref[key])), (key, got[i], ref[key])
+
+
 def test_bounded_wait_gives_up_and_reports_timeout():
     """A wait on a barrier nothing completes runs out after 50 ms; the host
     reads MOE_ERR_TIMEOUT from the status word and the context still works."""

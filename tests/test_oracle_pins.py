@@ -430,3 +430,74 @@ def test_input_generator_is_bf16_exact_and_seeded():
     for key in ("x", "w_router", "w1", "w3", "w2", "ws1", "ws3", "ws2"):
         np.testing.assert_array_equal(I.round_to_bf16(a[key]), a[key])
     assert a["sel_bias"].min() >= -0.5 and a["sel_bias"].max() < 0.5
+
+
+# --------------------------------------------------------------------------- #
+# noaux_tc sign-style bias update (NEXT row: bias-rule variant)               #
+# --------------------------------------------------------------------------- #
+def test_sign_update_growth_matches_page_figure(figures):
+    """64 micro-batch updates at rate 0.001 move a starved expert's bias by the
+    page's 0.064 per optimizer step (and an overloaded one by -0.064)."""
+    f = figures["noaux_tc_bias_growth"]
+    counts = np.array([0, 500, 500, 1000])            # mean 500
+    b = np.zeros(4, np.float32)
+    for _ in range(f["accumulation_steps"]):
+        b = O.bias_update_sign(counts, b, f["rate"])
+    assert abs(b[0] - f["growth_per_optimizer_step"]) < 1e-6
+    assert abs(b[3] + f["growth_per_optimizer_step"]) < 1e-6
+    assert b[1] == 0.0 and b[2] == 0.0                # at the mean: no move
+
+
+def test_sign_update_uniform_and_direction():
+    b0 = np.array([0.5, -0.25, 0.0], np.float32)
+    np.testing.assert_array_equal(O.bias_update_sign(np.array([7, 7, 7]), b0, 0.01), b0)
+    out = O.bias_update_sign(np.array([1, 2, 9]), np.zeros(3, np.float32), 0.01)
+    assert out[0] > 0 and out[1] > 0 and out[2] < 0
+    np.testing.assert_allclose(np.abs(out), 0.01, rtol=1e-7)
+
+
+# --------------------------------------------------------------------------- #
+# router statistics (NEXT row)                                                #
+# --------------------------------------------------------------------------- #
+def _balanced_routing(T, E, k, logit=0.0, gate=O.GATE_SOFTMAX):
+    """Token t picks experts (t*k + j) mod E: perfectly balanced counts."""
+    x = np.zeros((T, 1))
+    r = O.router(x, np.zeros((E, 1)), k, gate, True)
+    r.logits[:] = logit
+    r.scores[:] = (1.0 / E) if gate == O.GATE_SOFTMAX else 1.0 / (1.0 + math.exp(-logit))
+    r.topk_idx[:] = (np.arange(T)[:, None] * k + np.arange(k)[None, :]) % E
+    return r
+
+
+def test_stats_closed_forms_balanced():
+    T, E, k = 64, 8, 2
+    st = O.router_stats(_balanced_routing(T, E, k))
+    assert abs(st["z_loss"] - math.log(E) ** 2) < 1e-12      # lse of E zeros = ln E
+    assert abs(st["aux_loss"] - k) < 1e-12                    # E * E * (k/E) * (1/E)
+    assert st["cv"] == 0.0 and st["load_max_ratio"] == 1.0 and st["unused_frac"] == 0.0
+    assert abs(st["entropy_bits"] - math.log2(E)) < 1e-12
+    sg = O.router_stats(_balanced_routing(T, E, k, gate=O.GATE_SIGMOID))
+    assert abs(sg["aux_loss"] - E * k / 2) < 1e-12            # sigmoid(0) = 1/2
+
+
+def test_stats_collapse_hits_page_ceiling(figures):
+    """Every token on the same k experts: load_max_ratio = E/k (64/6 = 10.67)."""
+    f = figures["load_max_ratio_ceiling"]
+    T, E, k = 30, f["n_experts"], f["top_k"]
+    r = _balanced_routing(T, E, k)
+    r.topk_idx[:] = np.arange(k)[None, :]
+    st = O.router_stats(r)
+    assert abs(st["load_max_ratio"] - E / k) < 1e-12 and abs(E / k - f["ceiling"]) < 0.005
+    assert abs(st["unused_frac"] - (E - k) / E) < 1e-12
+
+
+def test_stats_cv_uses_bessel_and_lse_matches_scipy():
+    """cv of counts (1, 2, 3, 6): mean 3, unbiased std sqrt(14/3)."""
+    r = _balanced_routing(12, 4, 1)
+    r.topk_idx[:, 0] = np.array([0] + [1] * 2 + [2] * 3 + [3] * 6)
+    assert abs(O.router_stats(r)["cv"] - math.sqrt(14 / 3) / 3) < 1e-12
+    rng = np.random.default_rng(3)
+    inp = _random_layer(rng, 50, 12, 7, 4, 2)
+    rr = O.router(inp["x"], inp["w_router"], 2, O.GATE_SIGMOID, True)
+    lse = scipy.special.logsumexp(rr.logits, axis=1)
+    assert abs(O.router_stats(rr)["z_loss"] - np.mean(lse ** 2)) < 1e-12
