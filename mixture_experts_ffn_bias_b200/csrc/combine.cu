@@ -14,6 +14,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -62,6 +63,8 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
                const float* __restrict__ topk_w, const uint4* __restrict__ y_shared,
                uint4* __restrict__ out, int T, int vecs, int k_rt) {
+  pdl_trigger();
+  pdl_wait();
   using V = Vec<BF16>;
   const int k = KT > 0 ? KT : k_rt;
   const int lane = threadIdx.x & 31;
@@ -131,6 +134,8 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slo
 __global__ void __launch_bounds__(256)
 bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias, int E,
                    float target, float thresh, float starved_add, float rate, float clampv) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ long long s_part[8];
   const int tid = threadIdx.x;
   long long c_sum = 0;
@@ -158,6 +163,8 @@ bias_update_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias,
 __global__ void __launch_bounds__(256)
 bias_update_sign_kernel(const int32_t* __restrict__ counts, float* __restrict__ bias, int E,
                         float rate) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ long long s_part[8];
   const int tid = threadIdx.x;
   long long c_sum = 0;
@@ -180,15 +187,29 @@ bias_update_sign_kernel(const int32_t* __restrict__ counts, float* __restrict__ 
 }  // namespace
 
 template <bool BF16>
-void launch_combine(dim3 grid, int threads, cudaStream_t stream, const uint4* y, const int32_t* sp,
-                    const float* w, const uint4* ysh, uint4* out, int T, int vecs, int k) {
+cudaError_t launch_combine(dim3 grid, int threads, cudaStream_t stream, const uint4* y,
+                           const int32_t* sp, const float* w, const uint4* ysh, uint4* out, int T,
+                           int vecs, int k) {
+  const dim3 block(threads);
   switch (k) {
-    case 1: combine_kernel<BF16, 1><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
-    case 2: combine_kernel<BF16, 2><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
-    case 4: combine_kernel<BF16, 4><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
-    case 6: combine_kernel<BF16, 6><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
-    case 8: combine_kernel<BF16, 8><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k); break;
-    default: combine_kernel<BF16, 0><<<grid, threads, 0, stream>>>(y, sp, w, ysh, out, T, vecs, k);
+    case 1:
+      return launch_pdl(combine_kernel<BF16, 1>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
+    case 2:
+      return launch_pdl(combine_kernel<BF16, 2>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
+    case 4:
+      return launch_pdl(combine_kernel<BF16, 4>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
+    case 6:
+      return launch_pdl(combine_kernel<BF16, 6>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
+    case 8:
+      return launch_pdl(combine_kernel<BF16, 8>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
+    default:
+      return launch_pdl(combine_kernel<BF16, 0>, grid, block, 0, stream, y, sp, w, ysh, out, T,
+                        vecs, k);
   }
 }
 
@@ -201,23 +222,19 @@ cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, cons
   const uint4* ysh = static_cast<const uint4*>(y_shared);
   uint4* o = static_cast<uint4*>(out);
   if (bf16)
-    launch_combine<true>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
-  else
-    launch_combine<false>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
-  return cudaGetLastError();
+    return launch_combine<true>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
+  return launch_combine<false>(grid, warps * 32, stream, y, slot_pos, topk_w, ysh, o, T, vecs, k);
 }
 
 cudaError_t bias_update(const int32_t* counts, float* bias, int E, float target, float thresh,
                         float starved_add, float rate, float clamp, cudaStream_t stream) {
-  bias_update_kernel<<<1, 256, 0, stream>>>(counts, bias, E, target, thresh, starved_add, rate,
-                                            clamp);
-  return cudaGetLastError();
+  return launch_pdl(bias_update_kernel, dim3(1), dim3(256), 0, stream, counts, bias, E, target,
+                    thresh, starved_add, rate, clamp);
 }
 
 cudaError_t bias_update_sign(const int32_t* counts, float* bias, int E, float rate,
                              cudaStream_t stream) {
-  bias_update_sign_kernel<<<1, 256, 0, stream>>>(counts, bias, E, rate);
-  return cudaGetLastError();
+  return launch_pdl(bias_update_sign_kernel, dim3(1), dim3(256), 0, stream, counts, bias, E, rate);
 }
 
 }  // namespace moe

@@ -22,6 +22,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -42,6 +43,8 @@ __global__ void __launch_bounds__(kRankBlock)
 dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
                      int32_t* __restrict__ blk_counts, int32_t* __restrict__ rank_out,
                      uint32_t* __restrict__ status) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ uint32_t masks[kMaxE][kWords];
   const int tid = threadIdx.x;
   const int lane = tid & 31, word = tid >> 5;
@@ -88,6 +91,8 @@ constexpr int kScanSmemInts = 11776;   // 46 KB + the 1 KB scan array stay under
 __global__ void __launch_bounds__(kMaxE)
 dispatch_scan_kernel(int32_t* __restrict__ blk, int nblk, int E, int32_t* __restrict__ counts,
                      int32_t* __restrict__ offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s[kMaxE];
   __shared__ int sblk[kScanSmemInts];
   const int e = threadIdx.x;
@@ -135,6 +140,8 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
                         const int32_t* __restrict__ bases, int32_t* __restrict__ slot_pos,
                         int32_t* __restrict__ perm_src, uint4* __restrict__ x_perm, int T,
                         int vecs, int k, int E) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -175,6 +182,8 @@ __global__ void __launch_bounds__(256)
 dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ bases,
                           int32_t* __restrict__ slot_pos, int32_t* __restrict__ perm_src, int T,
                           int k, int E) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
   const int32_t* b = bases + static_cast<size_t>(t / kRankBlock) * E;
@@ -195,22 +204,20 @@ dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* _
 cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
                                int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
                                cudaStream_t stream) {
-  dispatch_positions_kernel<<<(T + 255) / 256, 256, 0, stream>>>(topk_idx, blk_bases, slot_pos,
-                                                                 perm_src, T, k, E);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_positions_kernel, dim3((T + 255) / 256), dim3(256), 0, stream,
+                    topk_idx, blk_bases, slot_pos, perm_src, T, k, E);
 }
 
 cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream) {
-  dispatch_rank_kernel<<<rank_blocks(T), kRankBlock, 0, stream>>>(topk_idx, T, k, E, blk_counts,
-                                                                   rank_out, status);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_rank_kernel, dim3(rank_blocks(T)), dim3(kRankBlock), 0, stream,
+                    topk_idx, T, k, E, blk_counts, rank_out, status);
 }
 
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream) {
-  dispatch_scan_kernel<<<1, kMaxE, 0, stream>>>(blk_counts, nblk, E, counts, offsets);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_scan_kernel, dim3(1), dim3(kMaxE), 0, stream, blk_counts, nblk, E,
+                    counts, offsets);
 }
 
 cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
@@ -218,10 +225,9 @@ cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              void* x_perm, int T, int d, int k, int E, cudaStream_t stream) {
   const int vecs = d * (bf16 ? 2 : 4) / 16;
   const int warps = 8;
-  dispatch_scatter_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-      static_cast<const uint4*>(x), topk_idx, blk_bases, slot_pos, perm_src,
-      static_cast<uint4*>(x_perm), T, vecs, k, E);
-  return cudaGetLastError();
+  return launch_pdl(dispatch_scatter_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
+                    stream, static_cast<const uint4*>(x), topk_idx, blk_bases, slot_pos, perm_src,
+                    static_cast<uint4*>(x_perm), T, vecs, k, E);
 }
 
 }  // namespace moe

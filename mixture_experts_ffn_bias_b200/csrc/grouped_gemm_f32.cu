@@ -11,6 +11,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -22,6 +23,8 @@ __global__ void __launch_bounds__(256)
 grouped_gemm_f32_kernel(const float* __restrict__ A, const int32_t* __restrict__ offsets, int G,
                         int rows_single, const float* __restrict__ B0,
                         const float* __restrict__ B1, int N, int K, float* __restrict__ C) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_off[MAXG + 1];
   __shared__ int s_pref[MAXG + 1];
   __shared__ float As[TK][TM + 1];
@@ -95,9 +98,8 @@ cudaError_t launch(const float* A, int64_t a_rows, const int32_t* offsets, int G
   const long long mt_upper = (rows + TM - 1) / TM + (g > 1 ? g : 0);
   if (mt_upper <= 0) return cudaSuccess;
   const dim3 grid(static_cast<unsigned>(mt_upper), (N + TN - 1) / TN);
-  grouped_gemm_f32_kernel<SWIGLU><<<grid, 256, 0, stream>>>(A, offsets, G, rows_single, B0, B1,
-                                                            N, K, C);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_f32_kernel<SWIGLU>, dim3(grid), dim3(256), 0, stream, A, offsets,
+                    G, rows_single, B0, B1, N, K, C);
 }
 
 }  // namespace

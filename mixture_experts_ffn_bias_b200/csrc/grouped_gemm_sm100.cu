@@ -31,6 +31,7 @@
 #include <cstdlib>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -207,6 +208,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc(&s_tmem_base, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  pdl_wait();   // everything above touches no global memory
   if (warp == 2) build_tile_prefix(args, n_tiles, s_off, s_prefix);
   tc_fence_before();
   __syncthreads();
@@ -283,6 +285,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
     }
+    if (lane == 0) pdl_trigger();   // all loads issued: the next kernel may launch
     if (!ok && lane == 0) {
       // Let every TMA copy this CTA started land before the CTA exits.
       for (int s = 0; s < STAGES; ++s) {
@@ -522,6 +525,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     tmem_alloc_pair(&s_tmem_base, Cfg::TMEM_COLS);
     tmem_relinquish_pair();
   }
+  pdl_wait();   // everything above touches no global memory
   if (warp == 2) build_tile_prefix<BM2>(args, n_tiles, s_off, s_prefix);
   tc_fence_before();
   __syncthreads();
@@ -557,6 +561,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      pdl_trigger();   // all loads issued: the next kernel may launch
       if (!ok && rank == 0) {
         // rank 0's stage barriers count both CTAs' copies: let them all land
         for (int s = 0; s < STAGES; ++s) {
@@ -769,8 +774,8 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
   if (tiles_upper <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles_upper < num_sms() ? tiles_upper : num_sms());
-  kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, a2);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(NUM_THREADS), Cfg::SMEM_BYTES, stream, a, b0, b1, c,
+                    a2);
 }
 
 template <int BN_ACC, int MODE>
@@ -801,8 +806,8 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   if (tiles_upper <= 0) return cudaSuccess;
   const int max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles_upper < max_pairs ? tiles_upper : max_pairs);
-  kern<<<2 * pairs, NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(a, b0, b1, c, a2);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), Cfg::SMEM_BYTES, stream, a, b0, b1,
+                    c, a2);
 }
 
 // The CTA-pair kernel is the default; MOE_B200_GEMM_1SM=1 selects the

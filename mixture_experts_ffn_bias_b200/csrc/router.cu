@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -43,6 +44,8 @@ __global__ void __launch_bounds__(256)
 router_logits_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
                      const float* __restrict__ offset, int T, int d, int E,
                      double* __restrict__ logits) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float xs[RT_KC][RT_TOK + 4];
   __shared__ float ws[RT_KC][RT_EXP + 4];
   const int tid = threadIdx.x;
@@ -191,6 +194,8 @@ __global__ void __launch_bounds__(256)
 router_select_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T,
                      int E, int k, int gate, int renorm, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -212,6 +217,8 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
                           int renorm, int32_t* __restrict__ topk_idx,
                           float* __restrict__ topk_w, int32_t* __restrict__ refine_count,
                           int32_t* __restrict__ refine_list) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -401,6 +408,8 @@ router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
                      const int32_t* __restrict__ refine_list,
                      const int32_t* __restrict__ refine_cand, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float4 s_x4[];          // d floats
   float* s_x = reinterpret_cast<float*>(s_x4);
   __shared__ double s_l[256];
@@ -469,6 +478,8 @@ router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
 
 __global__ void add_row_offset_kernel(float* __restrict__ logits, const float* __restrict__ off,
                                       long long n, int E) {
+  pdl_trigger();
+  pdl_wait();
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
     logits[i] += off[i % E];
@@ -479,8 +490,7 @@ __global__ void add_row_offset_kernel(float* __restrict__ logits, const float* _
 cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream) {
   const long long n = static_cast<long long>(T) * E;
   const int grid = static_cast<int>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  add_row_offset_kernel<<<grid, 256, 0, stream>>>(logits, offset, n, E);
-  return cudaGetLastError();
+  return launch_pdl(add_row_offset_kernel, dim3(grid), dim3(256), 0, stream, logits, offset, n, E);
 }
 
 cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
@@ -488,23 +498,21 @@ cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
                           cudaStream_t stream) {
   dim3 grid((T + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
   if (bf16)
-    router_logits_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
-        logit_offset, T, d, E, logits);
-  else
-    router_logits_kernel<float><<<grid, 256, 0, stream>>>(
-        static_cast<const float*>(x), static_cast<const float*>(w_router), logit_offset, T, d, E,
-        logits);
-  return cudaGetLastError();
+    return launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(256), 0, stream,
+                      static_cast<const __nv_bfloat16*>(x),
+                      static_cast<const __nv_bfloat16*>(w_router), logit_offset, T, d, E,
+                      logits);
+  return launch_pdl(router_logits_kernel<float>, grid, dim3(256), 0, stream,
+                    static_cast<const float*>(x), static_cast<const float*>(w_router),
+                    logit_offset, T, d, E, logits);
 }
 
 cudaError_t router_select(const double* logits, const float* sel_bias, int T, int E, int k,
                           int gate, int renorm, int32_t* topk_idx, float* topk_w,
                           cudaStream_t stream) {
   const int warps = 8;
-  router_select_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-      logits, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w);
-  return cudaGetLastError();
+  return launch_pdl(router_select_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
+                    stream, logits, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w);
 }
 
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
@@ -512,10 +520,9 @@ cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                int32_t* topk_idx, float* topk_w, int32_t* refine_count,
                                int32_t* refine_list, cudaStream_t stream) {
   const int warps = 8;
-  router_select_fast_kernel<<<(T + warps - 1) / warps, warps * 32, 0, stream>>>(
-      logits, logit_offset, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w, refine_count,
-      refine_list);
-  return cudaGetLastError();
+  return launch_pdl(router_select_fast_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
+                    stream, logits, logit_offset, sel_bias, T, E, k, gate, renorm, topk_idx,
+                    topk_w, refine_count, refine_list);
 }
 
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
@@ -533,11 +540,10 @@ cudaError_t router_refine(const void* x, const void* w_router, const float* logi
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  router_refine_kernel<<<grid, 256, smem, stream>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w_router),
-      logit_offset, sel_bias, d, E, k, gate, renorm, refine_count, refine_list, refine_cand,
-      topk_idx, topk_w);
-  return cudaGetLastError();
+  return launch_pdl(router_refine_kernel, dim3(grid), dim3(256), smem, stream,
+                    static_cast<const __nv_bfloat16*>(x),
+                    static_cast<const __nv_bfloat16*>(w_router), logit_offset, sel_bias, d, E, k,
+                    gate, renorm, refine_count, refine_list, refine_cand, topk_idx, topk_w);
 }
 
 }  // namespace moe

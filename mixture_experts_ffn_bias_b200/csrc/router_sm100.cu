@@ -35,6 +35,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -238,15 +239,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
   }
+  if (warp == 1) {
+    tmem_alloc(&s_tmem, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  pdl_wait();   // everything above touches no global memory
   if (FUSED && warp >= 2) {
     for (int e = threadIdx.x - 64; e < NPAD; e += 128) {
       s_off[e] = (e < E && out.offset) ? out.offset[e] : 0.f;
       s_bias[e] = (e < E && out.bias) ? out.bias[e] : 0.f;
     }
-  }
-  if (warp == 1) {
-    tmem_alloc(&s_tmem, C::TMEM_COLS);
-    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
@@ -270,6 +272,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      pdl_trigger();   // all loads issued: the next kernel may launch
       if (!ok) {
         for (int s = 0; s < C::STAGES; ++s) {
           if (!(issued_mask & (1u << s))) continue;
@@ -429,8 +432,8 @@ cudaError_t launch_router(const CUtensorMap& mx, const CUtensorMap& mw, int T, i
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int tiles = (T + RBM - 1) / RBM;
   const int grid = tiles < sms ? tiles : (sms > 0 ? sms : 148);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(mx, mw, T, K, E, out);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream, mx, mw, T, K, E,
+                    out);
 }
 
 int npad_for(int E) {

@@ -13,6 +13,7 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace moe {
 namespace {
@@ -25,6 +26,8 @@ __global__ void __launch_bounds__(256)
 stats_partial_kernel(const L* __restrict__ logits, int T, int E, int gate,
                      const int32_t* __restrict__ topk_idx, int k,
                      double* __restrict__ partials) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_sc[8][kMaxE];
   __shared__ int s_cnt[kMaxE];
   __shared__ double s_z[8];
@@ -99,6 +102,8 @@ __device__ double block_sum(double* s, double v) {
 __global__ void __launch_bounds__(256)
 stats_final_kernel(const double* __restrict__ partials, int nb, int T, int E,
                    float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ double s[256];
   const int e = threadIdx.x;
   double sc = 0.0, cnt = 0.0;
@@ -152,16 +157,14 @@ cudaError_t router_stats(bool fp64_logits, const void* logits, int T, int E, int
                          const int32_t* topk_idx, int k, double* partials, float* out,
                          cudaStream_t stream) {
   const int nb = stats_blocks(T);
-  if (fp64_logits)
-    stats_partial_kernel<double><<<nb, 256, 0, stream>>>(static_cast<const double*>(logits), T,
-                                                         E, gate, topk_idx, k, partials);
-  else
-    stats_partial_kernel<float><<<nb, 256, 0, stream>>>(static_cast<const float*>(logits), T, E,
-                                                        gate, topk_idx, k, partials);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e =
+      fp64_logits
+          ? launch_pdl(stats_partial_kernel<double>, dim3(nb), dim3(256), 0, stream,
+                       static_cast<const double*>(logits), T, E, gate, topk_idx, k, partials)
+          : launch_pdl(stats_partial_kernel<float>, dim3(nb), dim3(256), 0, stream,
+                       static_cast<const float*>(logits), T, E, gate, topk_idx, k, partials);
   if (e != cudaSuccess) return e;
-  stats_final_kernel<<<1, 256, 0, stream>>>(partials, nb, T, E, out);
-  return cudaGetLastError();
+  return launch_pdl(stats_final_kernel, dim3(1), dim3(256), 0, stream, partials, nb, T, E, out);
 }
 
 }  // namespace moe
