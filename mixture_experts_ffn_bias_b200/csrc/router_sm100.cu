@@ -14,9 +14,10 @@
 // With up to 128 experts and top-k <= 8 the routing decision is taken in the
 // same kernel (fused select): the epilogue thread that owns a token's row holds
 // all of its logits in registers, forms the gate statistics and the selection
-// keys and picks the top-(k+1) keys (descending, ties to the lower expert id;
-// a rolled round loop with four independent arg-max chains, the logits kept
-// in the thread's shared-memory column).  A token whose picked keys hold two keys
+// keys and picks the top-(k+1) keys (descending, ties to the lower expert id)
+// from per-group best keys, re-scanning only the winning group each round
+// (the logits kept in the thread's shared-memory column).  A token whose
+// picked keys hold two keys
 // closer than kRefineMargin is not decided here: it is listed together with
 // its candidate experts (every expert whose key is within the margin of the
 // (k+1)-th pick), and router_refine_kernel decides it on exact logits.
@@ -82,67 +83,115 @@ struct RouterOut {
 // Routing decision for one token from its logits held in registers (fused
 // select).  acc[i] = logit of expert i (i < E), overwritten with the
 // selection keys; the logits (with the per-expert offset) are kept in the
-// thread's shared-memory column s_log[i * 128] so the weights use them
-// exactly.
+// thread's shared-memory column s_log[i * 128], so the weights use them
+// exactly and the per-round re-scan can index them.  One thread owns a token
+// and only four warps run this per SM, so the code is written for
+// instruction-level parallelism: no branches inside the loops (even a
+// warp-uniform branch splits the unrolled loop into blocks that cannot be
+// interleaved), selects instead of short-circuit conditions, four partial
+// maxima and sums, and loads kept apart from stores.
 template <int COLS>
 __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int* s_seli,
                                           const float* s_off, const float* s_bias, int E, int t,
                                           const RouterOut& o) {
-  float m = -INFINITY;
+  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int i = 0; i < COLS; ++i) {
-    const float l = i < E ? acc[i] + s_off[i] : -INFINITY;
-    s_log[i * 128] = l;
-    acc[i] = i < E ? l + s_bias[i] : -INFINITY;
-    m = fmaxf(m, l);
+  for (int i = 0; i < COLS; i += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(s_off + i);
+    const float ov[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float l = i + q < E ? acc[i + q] + ov[q] : -INFINITY;
+      acc[i + q] = l;
+      mx[q] = fmaxf(mx[q], l);
+    }
   }
-  float S = 0.f;
-  if (o.gate == 0) {
-#pragma unroll 8
-    for (int i = 0; i < COLS; ++i)
-      if (i < E) S += expf(s_log[i * 128] - m);
+#pragma unroll
+  for (int i = 0; i < COLS; ++i) s_log[i * 128] = acc[i];
+#pragma unroll
+  for (int i = 0; i < COLS; i += 4) {
+    const float4 f = *reinterpret_cast<const float4*>(s_bias + i);
+    const float bv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[i + q] = i + q < E ? acc[i + q] + bv[q] : -INFINITY;
   }
-  // top-(k+1) keys: each round takes the largest key strictly after the
-  // previous pick in (descending key, ascending expert id) order.  The round
-  // loop stays rolled (an unrolled 9 x 128 body overflows the instruction
-  // cache); four independent arg-max chains per round give the scheduler
-  // independent work.  Picks go to the thread's shared-memory columns.
+  const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  // The softmax denominator is needed only without renormalisation: with
+  // it, the weights exp(l_j - m) / sum over the picks are the renormalised
+  // probabilities (the 1e-9 guard then scales with the denominator).
+  float S = 1.0f;
+  if (o.gate == 0 && !o.renorm) {
+    float sp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int i = 0; i < COLS; i += 4) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sp[q] += expf(s_log[(i + q) * 128] - m);   // exp(-inf) = 0 past E
+    }
+    S = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+  }
+  // top-(k+1) keys in (descending key, ascending expert id) order.  The
+  // experts are split into NG groups of GS consecutive ids; each group holds
+  // its best key not yet picked.  A round takes the best group head and
+  // re-scans only that group (keys re-formed from the shared-memory logit
+  // column and the bias: the same fp32 sums as acc[]) for its best key after
+  // the pick.  Picks go to the thread's shared-memory column s_seli.
+  constexpr int GS = COLS >= 64 ? 8 : 4;
+  constexpr int NG = COLS / GS;
+  constexpr int NONE = 0x7fffffff;
+  float gv[NG];
+  int gi[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    gv[g] = acc[g * GS];
+    gi[g] = g * GS;
+#pragma unroll
+    for (int s = 1; s < GS; ++s) {
+      const bool take = acc[g * GS + s] > gv[g];
+      gv[g] = take ? acc[g * GS + s] : gv[g];
+      gi[g] = take ? g * GS + s : gi[g];
+    }
+  }
   const int rounds = o.k < E ? o.k + 1 : o.k;
   float pv = INFINITY;
   int pi = -1;
   float min_gap = INFINITY;
 #pragma unroll 1
   for (int j = 0; j < rounds; ++j) {
-    float bv[4];
-    int bi[4];
+    // groups are in id order, so on equal heads the earlier group wins
+    float bv = gv[0];
+    int bi = gi[0], bg = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      bv[c] = -INFINITY;
-      bi[c] = 0x7fffffff;
+    for (int g = 1; g < NG; ++g) {
+      const bool take = (gi[g] != NONE) & ((bi == NONE) | (gv[g] > bv));
+      bv = take ? gv[g] : bv;
+      bi = take ? gi[g] : bi;
+      bg = take ? g : bg;
+    }
+    min_gap = j > 0 ? fminf(min_gap, pv - bv) : min_gap;
+    pv = bv;
+    pi = bi;
+    s_seli[j * 128] = bi;
+    float vv[GS];
+#pragma unroll
+    for (int s = 0; s < GS; ++s) {
+      const int i = bg * GS + s;
+      vv[s] = i < E ? s_log[i * 128] + s_bias[i] : -INFINITY;
+    }
+    float nv = -INFINITY;
+    int ni = NONE;
+#pragma unroll
+    for (int s = 0; s < GS; ++s) {
+      const int i = bg * GS + s;
+      const bool after = (vv[s] < pv) | ((vv[s] == pv) & (i > pi));
+      const bool take = after & ((vv[s] > nv) | (ni == NONE));
+      nv = take ? vv[s] : nv;
+      ni = take ? i : ni;
     }
 #pragma unroll
-    for (int i = 0; i < COLS; ++i) {
-      const int c = i & 3;
-      const float v = acc[i];
-      const bool after = v < pv || (v == pv && i > pi);
-      if (after && (v > bv[c] || bi[c] == 0x7fffffff)) {
-        bv[c] = v;
-        bi[c] = i;
-      }
+    for (int g = 0; g < NG; ++g) {
+      gv[g] = g == bg ? nv : gv[g];
+      gi[g] = g == bg ? ni : gi[g];
     }
-    // merge the chains: larger key wins, equal keys -> lower expert id
-#pragma unroll
-    for (int c = 1; c < 4; ++c) {
-      if (bi[c] != 0x7fffffff &&
-          (bi[0] == 0x7fffffff || bv[c] > bv[0] || (bv[c] == bv[0] && bi[c] < bi[0]))) {
-        bv[0] = bv[c];
-        bi[0] = bi[c];
-      }
-    }
-    if (j > 0) min_gap = fminf(min_gap, pv - bv[0]);
-    pv = bv[0];
-    pi = bi[0];
-    s_seli[j * 128] = bi[0];
   }
   if (min_gap < kRefineMargin) {
     // list the token with its candidate experts: every expert whose key is
@@ -153,9 +202,9 @@ __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int*
     int32_t* cand = o.refine_cand + static_cast<size_t>(slot) * kRefineCand;
     const float lo = pv - kRefineMargin;
     int n = (o.gate == 0 && !o.renorm) ? kRefineCand + 1 : 0;
-#pragma unroll
-    for (int i = 0; i < COLS; ++i) {
-      if (acc[i] >= lo) {
+#pragma unroll 1
+    for (int i = 0; i < E; ++i) {
+      if (s_log[i * 128] + s_bias[i] >= lo) {   // the key, as in acc[]
         if (n < kRefineCand) cand[n] = i;
         ++n;
       }
@@ -213,8 +262,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ float s_off[NPAD];
-  __shared__ float s_bias[NPAD];
+  __shared__ __align__(16) float s_off[NPAD];
+  __shared__ __align__(16) float s_bias[NPAD];
   __shared__ int s_sel[FUSED ? (KMAX_FUSED + 1) * 128 : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
