@@ -118,6 +118,36 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
                            int32_t* topk_idx, float* topk_w,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Selection-key variants of the router.
+ *   bias_space 0: key = logit + sel_bias (SigmoidRouter.forward of the
+ *     "moe-200m-qwen3-100b" README; what moe_router_topk does).
+ *   bias_space 1: key = gate score + sel_bias, the score being sigmoid(logit)
+ *     or the softmax probability over all E experts (the score-space
+ *     placement of the "noaux_tc" balance bias named on the page-3 model
+ *     card, which prints no code for it).
+ *   sel_noise: NULL, or [T, E] fp32 on the device, added to every key: the
+ *     training-time exploration noise of SigmoidRouter.forward
+ *     (sel_logits += randn * noise_std), drawn and scaled by the caller
+ *     (noise_std * standard-normal draws), so the library draws nothing.
+ * The noise and the bias move the selection only; the weights are the
+ * unbiased gate scores of the chosen experts, as in moe_router_topk. */
+typedef struct {
+  int32_t bias_space;        /* 0 or 1                                  */
+  int32_t reserved;          /* 0                                       */
+  const float* sel_noise;    /* [T, E] fp32 or NULL                     */
+} moe_router_opts;
+
+/* moe_router_topk with the key variants above (arguments and outputs as
+ * there; opts must not be NULL; bias_space outside {0, 1} or an unaligned
+ * sel_noise is MOE_ERR_INVALID).  Runs the unfused tensor-core path for
+ * bf16 layers: fp32 logits, fp32 keys, exact fp64 re-decision over all
+ * experts of every token with two of its top-(k+1) keys closer than 1e-4.
+ * With bias_space 0 and no noise it returns what moe_router_topk returns. */
+moe_status moe_router_topk_opts(const moe_config* cfg, const void* x, const void* w_router,
+                                const float* sel_bias, const float* logit_offset,
+                                const moe_router_opts* opts, int32_t* topk_idx, float* topk_w,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* Router GEMM alone: logits [T, E] fp32 = x . w_router^T (+ logit_offset),
  * for bf16 layers (fp32 layers return MOE_ERR_UNSUPPORTED).  Tensor cores,
  * exact bf16 products, fp32 accumulation: these are the logits moe_router_topk

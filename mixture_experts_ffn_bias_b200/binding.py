@@ -48,6 +48,11 @@ class MoEExpertWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2")]
 
 
+class MoERouterOpts(ctypes.Structure):
+    _fields_ = [("bias_space", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("sel_noise", ctypes.c_void_p)]
+
+
 _VP, _SZ, _I32, _F64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_double
 _CFG = ctypes.POINTER(MoEConfig)
 _WTS = ctypes.POINTER(MoEExpertWeights)
@@ -55,6 +60,8 @@ _SIGNATURES = {
     "moe_workspace_size": (_SZ, [_CFG]),
     "moe_check_config": (_I32, [_CFG]),
     "moe_router_topk": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_router_topk_opts": (_I32, [_CFG, _VP, _VP, _VP, _VP, ctypes.POINTER(MoERouterOpts),
+                                     _VP, _VP, _VP, _SZ, _VP]),
     "moe_router_logits": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_router_stats": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_permute": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -155,6 +162,19 @@ def moe_router_topk(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, 
     st = lib().moe_router_topk(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
                                _p(logit_offset), _p(topk_idx), _p(topk_w), _p(ws),
                                _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_router_topk_opts(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws,
+                         bias_space=0, sel_noise=None, stream=None, check=True) -> int:
+    """moe_router_topk with the key variants: bias_space 1 puts the bias on
+    the gate scores; sel_noise ([T, E] fp32, already scaled) is added to the
+    keys."""
+    opts = MoERouterOpts(int(bias_space), 0, _p(sel_noise))
+    st = lib().moe_router_topk_opts(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
+                                    _p(logit_offset), ctypes.byref(opts), _p(topk_idx),
+                                    _p(topk_w), _p(ws), _nbytes(ws) if ws is not None else 0,
+                                    _s(stream))
     return _check(st, check)
 
 

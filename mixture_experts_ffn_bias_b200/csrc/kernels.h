@@ -11,6 +11,14 @@ constexpr uint32_t kDevBadIndex = 1u;   // expert id outside [0, E) or repeated 
 constexpr uint32_t kDevTimeout = 2u;    // a bounded wait inside a kernel gave up
 
 // Router ---------------------------------------------------------------------
+// Selection-key variants: space 0: key = logit + bias (the default); space 1:
+// key = gate score + bias.  noise [T, E] fp32, already scaled by the caller,
+// is added to every key when non-null.
+struct KeyOpts {
+  int space = 0;
+  const float* noise = nullptr;
+  bool is_default() const { return space == 0 && noise == nullptr; }
+};
 // logits[T, E] (fp64 scratch) = x . w_router^T (+ logit_offset), exact products
 // with fp32 partial sums over 32-wide K chunks added in fp64.
 cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
@@ -18,8 +26,8 @@ cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
                           cudaStream_t stream);
 // gate scores, biased selection, top-k, combine weights from the logits.
 cudaError_t router_select(const double* logits, const float* sel_bias, int T, int E, int k,
-                          int gate, int renorm, int32_t* topk_idx, float* topk_w,
-                          cudaStream_t stream);
+                          int gate, int renorm, const KeyOpts& ko, int32_t* topk_idx,
+                          float* topk_w, cudaStream_t stream);
 
 // bf16 router: tensor-core fp32 logits, fast selection with near-tie
 // flagging, exact fp64 re-decision of the flagged tokens.  Tokens whose
@@ -42,16 +50,16 @@ cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, 
                              float* logits, uint32_t* status, cudaStream_t stream);
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
-                               int32_t* topk_idx, float* topk_w, int32_t* refine_count,
-                               int32_t* refine_list, cudaStream_t stream);
+                               const KeyOpts& ko, int32_t* topk_idx, float* topk_w,
+                               int32_t* refine_count, int32_t* refine_list, cudaStream_t stream);
 // Exact re-decision of the listed tokens.  refine_cand null: every listed
 // token is re-decided over all experts (the unfused path lists no
-// candidates).
+// candidates; score-space softmax keys need all of them).
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
-                          int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          const int32_t* refine_cand, int32_t* topk_idx, float* topk_w, int sms,
-                          cudaStream_t stream);
+                          int renorm, const KeyOpts& ko, const int32_t* refine_count,
+                          const int32_t* refine_list, const int32_t* refine_cand,
+                          int32_t* topk_idx, float* topk_w, int sms, cudaStream_t stream);
 
 // logits[t, e] += offset[e]
 cudaError_t add_row_offset(float* logits, const float* offset, int T, int E, cudaStream_t stream);

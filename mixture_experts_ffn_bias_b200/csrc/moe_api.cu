@@ -105,13 +105,16 @@ int device_sms() {
 // Router into caller buffers; logits scratch in ws.
 moe_status run_router(const moe_config* c, const void* x, const void* w_router,
                       const float* sel_bias, const float* logit_offset, int32_t* topk_idx,
-                      float* topk_w, void* ws, cudaStream_t s) {
+                      float* topk_w, void* ws, cudaStream_t s,
+                      const moe::KeyOpts& ko = moe::KeyOpts{}) {
   const Layout L = layout(*c);
   if (c->dtype == MOE_BF16) {
     float* logits = at<float>(ws, L.logits);
     int32_t* count = at<int32_t>(ws, L.status) + 1;
     int32_t* list = at<int32_t>(ws, L.refine);
-    const bool fused = moe::router_fused_supported(c->n_experts, c->top_k);
+    // the key variants take the unfused path: fp32 logits, a select kernel
+    // and exact re-decision over all experts
+    const bool fused = ko.is_default() && moe::router_fused_supported(c->n_experts, c->top_k);
     int32_t* cand = at<int32_t>(ws, L.refine_cand);
     if (fused) {
       MOE_TRY(moe::router_topk_tc(x, c->T, w_router, c->n_experts, c->d_model, logit_offset,
@@ -121,19 +124,19 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
       MOE_TRY(moe::router_logits_tc(x, c->T, w_router, c->n_experts, c->d_model, logits,
                                     at<uint32_t>(ws, L.status), s));
       MOE_TRY(moe::router_select_fast(logits, logit_offset, sel_bias, c->T, c->n_experts,
-                                      c->top_k, c->gate, c->norm_topk_prob, topk_idx, topk_w,
+                                      c->top_k, c->gate, c->norm_topk_prob, ko, topk_idx, topk_w,
                                       count, list, s));
     }
     MOE_TRY(moe::router_refine(x, w_router, logit_offset, sel_bias, c->T, c->d_model,
-                               c->n_experts, c->top_k, c->gate, c->norm_topk_prob, count, list,
-                               fused ? cand : nullptr, topk_idx, topk_w, device_sms(), s));
+                               c->n_experts, c->top_k, c->gate, c->norm_topk_prob, ko, count,
+                               list, fused ? cand : nullptr, topk_idx, topk_w, device_sms(), s));
     return MOE_OK;
   }
   double* logits = at<double>(ws, L.logits);
   MOE_TRY(moe::router_logits(false, x, w_router, logit_offset, c->T, c->d_model, c->n_experts,
                              logits, s));
   MOE_TRY(moe::router_select(logits, sel_bias, c->T, c->n_experts, c->top_k, c->gate,
-                             c->norm_topk_prob, topk_idx, topk_w, s));
+                             c->norm_topk_prob, ko, topk_idx, topk_w, s));
   return MOE_OK;
 }
 
@@ -309,6 +312,29 @@ moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_r
   if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
   if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
   return run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, S(stream));
+}
+
+moe_status moe_router_topk_opts(const moe_config* cfg, const void* x, const void* w_router,
+                                const float* sel_bias, const float* logit_offset,
+                                const moe_router_opts* opts, int32_t* topk_idx, float* topk_w,
+                                void* ws, size_t ws_bytes, void* stream) {
+  if (opts == nullptr || (opts->bias_space != 0 && opts->bias_space != 1) ||
+      (opts->sel_noise && !aligned4(opts->sel_noise)))
+    return MOE_ERR_INVALID;
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w) return MOE_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned4(topk_idx) || !aligned4(topk_w) ||
+      (sel_bias && !aligned4(sel_bias)) || (logit_offset && !aligned4(logit_offset)))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  if ((st = clear_status(ws, S(stream))) != MOE_OK) return st;
+  moe::KeyOpts ko;
+  ko.space = opts->bias_space;
+  ko.noise = opts->sel_noise;
+  return run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, S(stream),
+                    ko);
 }
 
 moe_status moe_router_logits(const moe_config* cfg, const void* x, const void* w_router,

@@ -19,6 +19,13 @@
 //   margin, so every token's decision equals the one taken on exact logits.
 // fp32 layers: logits on CUDA cores (fp32 products summed in fp32 over
 // 32-wide K chunks, chunk sums added in fp64), selection in fp64.
+//
+// Key variants (KeyOpts, moe_router_topk_opts): the bias added to the gate
+// score instead of the logit (the score-space placement of the "noaux_tc"
+// balance bias named on the page-3 model card), and a caller-drawn selection
+// noise [T, E] added to every key (the training-time exploration noise of
+// SigmoidRouter.forward).  Every select path forms the same keys; the
+// variants run the unfused bf16 path with re-decision over all experts.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -112,9 +119,11 @@ router_logits_kernel(const Tin* __restrict__ x, const Tin* __restrict__ wr,
 }
 
 // Selection, gate and weights for one token in fp64, done by one warp.  `l`
-// holds the logits of experts lane + 32 i (offset already added).
+// holds the logits of experts lane + 32 i (offset already added); keys are
+// (space ? score : logit) + bias (+ noise_row[e]).
 __device__ void warp_select_fp64(const double (&l)[kMaxPerLane], const float* __restrict__ bias,
-                                 int E, int k, int gate, int renorm,
+                                 int E, int k, int gate, int renorm, int space,
+                                 const float* __restrict__ noise_row,
                                  int32_t* __restrict__ idx_row, float* __restrict__ w_row) {
   const int lane = threadIdx.x & 31;
   double key[kMaxPerLane], s[kMaxPerLane];
@@ -124,7 +133,6 @@ __device__ void warp_select_fp64(const double (&l)[kMaxPerLane], const float* __
   for (int i = 0; i < kMaxPerLane; ++i) {
     const int e = lane + 32 * i;
     taken[i] = e >= E;
-    key[i] = e < E ? l[i] + (bias ? static_cast<double>(bias[e]) : 0.0) : -INFINITY;
     if (e < E) lmax = fmax(lmax, l[i]);
   }
   if (gate == 1) {  // sigmoid
@@ -143,6 +151,13 @@ __device__ void warp_select_fp64(const double (&l)[kMaxPerLane], const float* __
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
 #pragma unroll
     for (int i = 0; i < kMaxPerLane; ++i) s[i] = s[i] / sum;
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = e < E ? (space ? s[i] : l[i]) + (bias ? static_cast<double>(bias[e]) : 0.0) +
+                         (noise_row ? static_cast<double>(noise_row[e]) : 0.0)
+                   : -INFINITY;
   }
   int my_idx = 0;
   double my_w = 0.0, wsum = 0.0;
@@ -192,7 +207,8 @@ __device__ void warp_select_fp64(const double (&l)[kMaxPerLane], const float* __
 // One warp per token, fp64 logits.
 __global__ void __launch_bounds__(256)
 router_select_kernel(const double* __restrict__ logits, const float* __restrict__ bias, int T,
-                     int E, int k, int gate, int renorm, int32_t* __restrict__ topk_idx,
+                     int E, int k, int gate, int renorm, int space,
+                     const float* __restrict__ noise, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w) {
   pdl_trigger();
   pdl_wait();
@@ -205,8 +221,9 @@ router_select_kernel(const double* __restrict__ logits, const float* __restrict_
     const int e = lane + 32 * i;
     l[i] = e < E ? logits[static_cast<size_t>(t) * E + e] : -INFINITY;
   }
-  warp_select_fp64(l, bias, E, k, gate, renorm, topk_idx + static_cast<size_t>(t) * k,
-                   topk_w + static_cast<size_t>(t) * k);
+  warp_select_fp64(l, bias, E, k, gate, renorm, space,
+                   noise ? noise + static_cast<size_t>(t) * E : nullptr,
+                   topk_idx + static_cast<size_t>(t) * k, topk_w + static_cast<size_t>(t) * k);
 }
 
 // ---------------------------------------------------------------- bf16 layers
@@ -214,8 +231,9 @@ router_select_kernel(const double* __restrict__ logits, const float* __restrict_
 __global__ void __launch_bounds__(256)
 router_select_fast_kernel(const float* __restrict__ logits, const float* __restrict__ offset,
                           const float* __restrict__ bias, int T, int E, int k, int gate,
-                          int renorm, int32_t* __restrict__ topk_idx,
-                          float* __restrict__ topk_w, int32_t* __restrict__ refine_count,
+                          int renorm, int space, const float* __restrict__ noise,
+                          int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                          int32_t* __restrict__ refine_count,
                           int32_t* __restrict__ refine_list) {
   pdl_trigger();
   pdl_wait();
@@ -230,7 +248,7 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
     const int e = lane + 32 * i;
     if (e < E) {
       l[i] = logits[static_cast<size_t>(t) * E + e] + (offset ? offset[e] : 0.0f);
-      key[i] = l[i] + (bias ? bias[e] : 0.0f);
+      key[i] = l[i];
       taken[i] = false;
       lmax = fmaxf(lmax, l[i]);
     } else {
@@ -238,6 +256,39 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
       key[i] = -INFINITY;
       taken[i] = true;
     }
+  }
+  // Score-space softmax keys are probabilities: their error scales with the
+  // largest one (1 / sum), so the re-decision margin does too, with a floor
+  // for the rounding of the bias addition.
+  float margin = kRefineMargin;
+  if (space) {   // key base = the gate score
+    if (gate == 1) {
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i) key[i] = 1.0f / (1.0f + expf(-l[i]));
+    } else {
+      float mm = lmax;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i) {
+        key[i] = expf(l[i] - mm);   // 0 past E
+        sum += key[i];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+      for (int i = 0; i < kMaxPerLane; ++i) key[i] = key[i] / sum;
+      margin = fmaxf(kRefineMargin / sum, 1e-5f);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E)
+      key[i] += (bias ? bias[e] : 0.0f) + (noise ? noise[static_cast<size_t>(t) * E + e] : 0.0f);
+    else
+      key[i] = -INFINITY;
   }
   // top-(k+1) keys, descending, ties -> lower expert id
   const int rounds = k < E ? k + 1 : k;
@@ -285,7 +336,7 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
       my_l = lsel;
     }
   }
-  if (fminf(min_gap, edge_gap) < kRefineMargin) {
+  if (fminf(min_gap, edge_gap) < margin) {
     if (lane == 0) refine_list[atomicAdd(refine_count, 1)] = t;
     return;
   }
@@ -323,8 +374,8 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
 // the fp64 keys (ties to the lower expert id); the weights are formed in fp32
 // from the exact logits.
 __device__ void refine_select(const double* s_l, const int* s_e, int n, const float* bias,
-                              int k, int gate, int renorm, bool all_experts,
-                              int32_t* idx_row, float* w_row) {
+                              int k, int gate, int renorm, bool all_experts, int space,
+                              const float* noise_row, int32_t* idx_row, float* w_row) {
   const int lane = threadIdx.x & 31;
   double key[kMaxPerLane];
   float lf[kMaxPerLane];
@@ -338,8 +389,36 @@ __device__ void refine_select(const double* s_l, const int* s_e, int n, const fl
     ex[j] = c < n ? s_e[c] : 0x7fffffff;
     const double l = c < n ? s_l[c] : -INFINITY;
     lf[j] = static_cast<float>(l);
-    key[j] = c < n ? l + (bias ? static_cast<double>(bias[ex[j]]) : 0.0) : -INFINITY;
+    key[j] = l;
     m = fmaxf(m, lf[j]);
+  }
+  if (space) {   // key base = the exact gate score (softmax: all experts are here)
+    if (gate == 1) {
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) key[j] = 1.0 / (1.0 + exp(-key[j]));
+    } else {
+      double mm = -INFINITY, sum = 0.0;
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) mm = fmax(mm, key[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mm = fmax(mm, __shfl_xor_sync(0xffffffffu, mm, o));
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) {
+        key[j] = exp(key[j] - mm);   // 0 past n
+        sum += key[j];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+      for (int j = 0; j < kMaxPerLane; ++j) key[j] = key[j] / sum;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxPerLane; ++j) {
+    const int c = lane + 32 * j;
+    key[j] = c < n ? key[j] + (bias ? static_cast<double>(bias[ex[j]]) : 0.0) +
+                         (noise_row ? static_cast<double>(noise_row[ex[j]]) : 0.0)
+                   : -INFINITY;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -404,7 +483,8 @@ __device__ void refine_select(const double* s_l, const int* s_e, int n, const fl
 __global__ void __launch_bounds__(256)
 router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
                      const float* __restrict__ offset, const float* __restrict__ bias, int d,
-                     int E, int k, int gate, int renorm, const int32_t* __restrict__ refine_count,
+                     int E, int k, int gate, int renorm, int space,
+                     const float* __restrict__ noise, const int32_t* __restrict__ refine_count,
                      const int32_t* __restrict__ refine_list,
                      const int32_t* __restrict__ refine_cand, int32_t* __restrict__ topk_idx,
                      float* __restrict__ topk_w) {
@@ -470,8 +550,9 @@ router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
     }
     __syncthreads();
     if (warp == 0)
-      refine_select(s_l, s_e, n, bias, k, gate, renorm, all, topk_idx + static_cast<size_t>(t) * k,
-                    topk_w + static_cast<size_t>(t) * k);
+      refine_select(s_l, s_e, n, bias, k, gate, renorm, all, space,
+                    noise ? noise + static_cast<size_t>(t) * E : nullptr,
+                    topk_idx + static_cast<size_t>(t) * k, topk_w + static_cast<size_t>(t) * k);
     __syncthreads();
   }
 }
@@ -508,28 +589,29 @@ cudaError_t router_logits(bool bf16, const void* x, const void* w_router,
 }
 
 cudaError_t router_select(const double* logits, const float* sel_bias, int T, int E, int k,
-                          int gate, int renorm, int32_t* topk_idx, float* topk_w,
-                          cudaStream_t stream) {
+                          int gate, int renorm, const KeyOpts& ko, int32_t* topk_idx,
+                          float* topk_w, cudaStream_t stream) {
   const int warps = 8;
   return launch_pdl(router_select_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
-                    stream, logits, sel_bias, T, E, k, gate, renorm, topk_idx, topk_w);
+                    stream, logits, sel_bias, T, E, k, gate, renorm, ko.space, ko.noise, topk_idx,
+                    topk_w);
 }
 
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
-                               int32_t* topk_idx, float* topk_w, int32_t* refine_count,
-                               int32_t* refine_list, cudaStream_t stream) {
+                               const KeyOpts& ko, int32_t* topk_idx, float* topk_w,
+                               int32_t* refine_count, int32_t* refine_list, cudaStream_t stream) {
   const int warps = 8;
   return launch_pdl(router_select_fast_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
-                    stream, logits, logit_offset, sel_bias, T, E, k, gate, renorm, topk_idx,
-                    topk_w, refine_count, refine_list);
+                    stream, logits, logit_offset, sel_bias, T, E, k, gate, renorm, ko.space,
+                    ko.noise, topk_idx, topk_w, refine_count, refine_list);
 }
 
 cudaError_t router_refine(const void* x, const void* w_router, const float* logit_offset,
                           const float* sel_bias, int T, int d, int E, int k, int gate,
-                          int renorm, const int32_t* refine_count, const int32_t* refine_list,
-                          const int32_t* refine_cand, int32_t* topk_idx, float* topk_w, int sms,
-                          cudaStream_t stream) {
+                          int renorm, const KeyOpts& ko, const int32_t* refine_count,
+                          const int32_t* refine_list, const int32_t* refine_cand,
+                          int32_t* topk_idx, float* topk_w, int sms, cudaStream_t stream) {
   int grid = 2 * sms;
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
@@ -543,7 +625,8 @@ cudaError_t router_refine(const void* x, const void* w_router, const float* logi
   return launch_pdl(router_refine_kernel, dim3(grid), dim3(256), smem, stream,
                     static_cast<const __nv_bfloat16*>(x),
                     static_cast<const __nv_bfloat16*>(w_router), logit_offset, sel_bias, d, E, k,
-                    gate, renorm, refine_count, refine_list, refine_cand, topk_idx, topk_w);
+                    gate, renorm, ko.space, ko.noise, refine_count, refine_list, refine_cand,
+                    topk_idx, topk_w);
 }
 
 }  // namespace moe

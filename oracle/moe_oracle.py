@@ -88,13 +88,20 @@ def softmax_rows(z: np.ndarray) -> np.ndarray:
 
 
 def router(x, w_router, top_k: int, gate: int, norm_topk_prob: bool,
-           sel_bias=None, logit_offset=None) -> Routing:
+           sel_bias=None, logit_offset=None, bias_space: int = 0, sel_noise=None) -> Routing:
     """Router forward: logits, gate scores, biased selection, top-k, weights.
 
     Follows ``SigmoidRouter.forward`` ("moe-200m-qwen3-100b" README) for the
     sigmoid gate and the qwen3 preset (SpecForge PR #930, "What this adds") for
     the softmax gate.  ``logit_offset`` is a per-expert constant added to the
     logits before the gate (used only by the skewed-load workload).
+
+    Selection-key variants: ``bias_space=1`` adds the bias to the gate scores
+    instead of the logits (the score-space placement of the "noaux_tc" balance
+    bias the page-3 model card names without code); ``sel_noise`` [T, E] is
+    added to every key, the exploration noise of ``SigmoidRouter.forward``
+    (``sel_logits += randn * noise_std``) with the draws and the scale
+    supplied by the caller.  Both move the selection only.
     """
     x64, w64 = _as64(x), _as64(w_router)
     T, E = x64.shape[0], w64.shape[0]
@@ -111,8 +118,14 @@ def router(x, w_router, top_k: int, gate: int, norm_topk_prob: bool,
         scores = softmax_rows(logits)
     else:
         raise ValueError("unknown gate")
-    # 3. selection keys: the bias moves the selection only
-    keys = logits if sel_bias is None else logits + _as64(sel_bias)[None, :]
+    # 3. selection keys: the bias (and the noise) move the selection only
+    if bias_space not in (0, 1):
+        raise ValueError("bias_space must be 0 or 1")
+    keys = logits if bias_space == 0 else scores
+    if sel_bias is not None:
+        keys = keys + _as64(sel_bias)[None, :]
+    if sel_noise is not None:
+        keys = keys + _as64(sel_noise)
     # 4. top-k: stable ascending sort of -key = descending key, ties -> lower e
     order = np.argsort(-keys, axis=1, kind="stable")
     idx = order[:, :top_k]

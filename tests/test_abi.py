@@ -98,6 +98,16 @@ def test_null_and_misaligned_pointers_rejected(lib):
     st = B.moe_router_topk(cfg, ok, ok, None, None, ok, ok, _FakeTensor(1 << 20, 1024),
                            stream=0, check=False)
     assert st == B.MOE_ERR_WORKSPACE
+    # key-variant router: bias_space outside {0, 1}, misaligned noise
+    st = B.moe_router_topk_opts(cfg, ok, ok, None, None, ok, ok, ws, bias_space=2, stream=0,
+                                check=False)
+    assert st == B.MOE_ERR_INVALID
+    st = B.moe_router_topk_opts(cfg, ok, ok, None, None, ok, ok, ws, bias_space=1,
+                                sel_noise=_FakeTensor((1 << 20) + 2), stream=0, check=False)
+    assert st == B.MOE_ERR_INVALID
+    st = B.moe_router_topk_opts(cfg, None, ok, None, None, ok, ok, ws, bias_space=1, stream=0,
+                                check=False)
+    assert st == B.MOE_ERR_INVALID
     # shared expert weights missing for a layer with a shared expert
     w = {"w1": ok, "w3": ok, "w2": ok}
     st = B.moe_forward(cfg, ok, ok, None, None, w, ok, ok, ok, ok, ws, stream=0, check=False)

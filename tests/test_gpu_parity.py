@@ -255,6 +255,60 @@ def test_router_topk_call(name):
     P.check_routing(_np(idx), _np(w), P.oracle_routing(shape, host))
 
 
+@pytest.mark.parametrize("name", ["tiny", "page2_small", "qwen3_small", "skew_small"])
+@pytest.mark.parametrize("space,noisy", [(1, False), (0, True), (1, True)])
+def test_router_key_variants_call(name, space, noisy):
+    """moe_router_topk_opts: bias on the gate scores and/or a given
+    selection noise [T, E], against the oracle's router with the same
+    options; the weights stay the unbiased scores."""
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    if "sel_bias" not in host:
+        host["sel_bias"] = np.random.default_rng(31).uniform(
+            -0.05, 0.05, shape.n_experts).astype(np.float32)
+    cfg, ws = _buffers(shape)
+    dt = torch.bfloat16 if shape.dtype == I.DTYPE_BF16 else torch.float32
+    x = to_device(host["x"], dt, "cuda")
+    wr = to_device(host["w_router"], dt, "cuda")
+    bias = to_device(host["sel_bias"], torch.float32, "cuda")
+    off = (to_device(host["logit_offset"], torch.float32, "cuda")
+           if "logit_offset" in host else None)
+    noise = None
+    if noisy:
+        noise = (0.1 * np.random.default_rng(32).standard_normal(
+            (shape.T, shape.n_experts))).astype(np.float32)
+    idx = torch.empty((shape.T, shape.top_k), dtype=torch.int32, device="cuda")
+    w = torch.empty((shape.T, shape.top_k), dtype=torch.float32, device="cuda")
+    B.moe_router_topk_opts(cfg, x, wr, bias, off, idx, w, ws, bias_space=space,
+                           sel_noise=None if noise is None else to_device(noise, torch.float32,
+                                                                          "cuda"))
+    torch.cuda.synchronize()
+    r = O.router(host["x"], host["w_router"], shape.top_k, shape.gate,
+                 bool(shape.norm_topk_prob), host["sel_bias"], host.get("logit_offset"),
+                 bias_space=space, sel_noise=noise)
+    P.check_routing(_np(idx), _np(w), r)
+
+
+def test_router_opts_default_is_router_topk():
+    shape = SMALL["qwen3_small"]
+    host = I.make_inputs(shape)
+    cfg, ws = _buffers(shape)
+    x = to_device(host["x"], torch.bfloat16, "cuda")
+    wr = to_device(host["w_router"], torch.bfloat16, "cuda")
+    out = []
+    for opts in (False, True):
+        idx = torch.empty((shape.T, shape.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((shape.T, shape.top_k), dtype=torch.float32, device="cuda")
+        if opts:
+            B.moe_router_topk_opts(cfg, x, wr, None, None, idx, w, ws)
+        else:
+            B.moe_router_topk(cfg, x, wr, None, None, idx, w, ws)
+        torch.cuda.synchronize()
+        out.append((_np(idx), _np(w)))
+    np.testing.assert_array_equal(out[0][0], out[1][0])
+    np.testing.assert_array_equal(out[0][1], out[1][1])
+
+
 @pytest.mark.parametrize("name", FULL)
 def test_tensor_core_logit_error_is_far_below_the_refine_margin(name):
     """The router decides from tensor-core fp32 logits and re-decides on exact

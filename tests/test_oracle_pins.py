@@ -501,3 +501,57 @@ def test_stats_cv_uses_bessel_and_lse_matches_scipy():
     rr = O.router(inp["x"], inp["w_router"], 2, O.GATE_SIGMOID, True)
     lse = scipy.special.logsumexp(rr.logits, axis=1)
     assert abs(O.router_stats(rr)["z_loss"] - np.mean(lse ** 2)) < 1e-12
+
+
+# --------------------------------------------------------------------------- #
+# selection-key variants: score-space bias, selection noise                  #
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("name", ["score_space_bias_sigmoid", "score_space_bias_softmax"])
+def test_worked_score_space_bias(worked, name):
+    """Catches: bias_space ignored, bias added to the weights, or the score
+    transformation applied to the bias as well."""
+    c = worked[name]
+    x, w = _arr(c["x"]), _arr(c["w_router"])
+    b = np.array(c["sel_bias"])
+    for space, key in ((0, "logit_space"), (1, "score_space")):
+        r = O.router(x, w, c["top_k"], _gate(c["gate"]), c["norm_topk_prob"], sel_bias=b,
+                     bias_space=space)
+        assert r.topk_idx.tolist() == c[key]["expected_idx"], key
+        np.testing.assert_allclose(r.topk_w, _arr(c[key]["expected_w"]), rtol=0, atol=1e-15)
+
+
+def test_worked_selection_noise(worked):
+    """Catches: noise dropped, or noise leaking into the weights."""
+    c = worked["selection_noise_moves_selection_only"]
+    x, w = _arr(c["x"]), _arr(c["w_router"])
+    r = O.router(x, w, c["top_k"], _gate(c["gate"]), c["norm_topk_prob"],
+                 sel_noise=np.array(c["sel_noise"]))
+    assert r.topk_idx.tolist() == c["expected_idx"]
+    np.testing.assert_allclose(r.topk_w, _arr(c["expected_w"]), rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("gate", [O.GATE_SOFTMAX, O.GATE_SIGMOID])
+def test_score_space_without_bias_selects_like_logits(gate):
+    """Both gates are increasing in each token's logits, so with no bias the
+    score-space keys order the experts as the logits do.  Catches: a
+    decreasing or mixed-up score transform in the keys."""
+    rng = np.random.default_rng(7)
+    x, w = rng.standard_normal((64, 16)), rng.standard_normal((24, 16))
+    r0 = O.router(x, w, 5, gate, True)
+    r1 = O.router(x, w, 5, gate, True, bias_space=1)
+    np.testing.assert_array_equal(r0.topk_idx, r1.topk_idx)
+    np.testing.assert_array_equal(r0.topk_w, r1.topk_w)
+
+
+def test_token_constant_noise_equals_bias():
+    """Noise that is the same for every token is a selection bias.  Catches:
+    noise rows and columns transposed, or noise scaled twice."""
+    rng = np.random.default_rng(8)
+    x, w = rng.standard_normal((40, 12)), rng.standard_normal((10, 12))
+    b = rng.uniform(-0.5, 0.5, 10)
+    r_bias = O.router(x, w, 3, O.GATE_SIGMOID, True, sel_bias=b)
+    r_noise = O.router(x, w, 3, O.GATE_SIGMOID, True, sel_noise=np.tile(b, (40, 1)))
+    np.testing.assert_array_equal(r_bias.topk_idx, r_noise.topk_idx)
+    np.testing.assert_array_equal(r_bias.topk_w, r_noise.topk_w)
+    # and it moves nothing but the selection
+    np.testing.assert_array_equal(r_noise.scores, O.router(x, w, 3, O.GATE_SIGMOID, True).scores)
