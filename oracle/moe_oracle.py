@@ -339,3 +339,101 @@ def router_stats(routing: Routing) -> dict:
     unused = float(np.mean(counts == 0))
     return {"z_loss": z_loss, "aux_loss": aux_loss, "cv": cv, "entropy_bits": entropy_bits,
             "load_max_ratio": load_max_ratio, "unused_frac": unused, "counts": counts}
+
+
+def _swiglu_expert_backward(xr, w1, w3, w2, dy):
+    """Gradients of one SwiGLU expert y = w2 (silu(w1 x) * (w3 x)) on rows xr.
+
+    Chain rule through the three linears and silu, silu'(g) = s(g) (1 + g (1 - s(g)))
+    with s the logistic function.  Returns (dx [n, d], dw1 [F, d], dw3 [F, d],
+    dw2 [d, F]).
+    """
+    xr, dy = _as64(xr), _as64(dy)
+    w1, w3, w2 = _as64(w1), _as64(w3), _as64(w2)
+    g = xr @ w1.T
+    u = xr @ w3.T
+    sg = sigmoid(g)
+    h = g * sg * u                       # silu(g) * u
+    dh = dy @ w2                         # [n, F]
+    du = dh * (g * sg)                   # d/du of silu(g) u
+    dg = dh * u * (sg * (1.0 + g * (1.0 - sg)))
+    dx = dg @ w1 + du @ w3
+    return dx, dg.T @ xr, du.T @ xr, dy.T @ h
+
+
+def moe_backward(inp: dict, top_k: int, gate: int, norm_topk_prob: bool, dout,
+                 routing: Optional[Routing] = None) -> dict:
+    """Gradients of the layer output with respect to x and every weight.
+
+    The layer is the forward of ``moe_forward`` (the pages train it: the
+    "moe-200m-qwen3-100b" README trains the SigmoidRouter layer end to end,
+    SpecForge PR #930 trains the qwen3 drafter).  Given dout [T, d]:
+
+    * combine: dw[t, j] = <dout[t], y[t, j]>, the expert input gradient is
+      w[t, j] dout[t]; the shared expert gets dout[t] with weight 1;
+    * experts: the SwiGLU chain rule (``_swiglu_expert_backward``), weight
+      gradients summed over the expert's rows;
+    * router: the selection (top-k of logits + bias (+ noise)) is piecewise
+      constant, so bias and noise get no gradient; the weights are
+      w_j = s_j / (sum_i s_i + 1e-9) (or s_j without renormalisation) with
+      s = sigmoid(logits) or softmax(logits) over all E, so
+      ds_j = (dw_j - sum_i dw_i w_i) / (sum_i s_i + 1e-9) (ds_j = dw_j without
+      renormalisation), zero for experts not picked; dlogits =
+      ds * s (1 - s) for sigmoid and s * (ds - <ds, s>) for softmax;
+      logits = x w_router^T + offset gives dw_router = dlogits^T x and
+      dx += dlogits w_router.
+
+    Returns a dict of fp64 arrays: dx, dw_router, dw1, dw3, dw2, dws1, dws3,
+    dws2 (the last three only with a shared expert), dlogits, dtopk_w.
+    """
+    x = _as64(inp["x"])
+    dout = _as64(dout)
+    T, d = x.shape
+    if routing is None:
+        routing = router(x, inp["w_router"], top_k, gate, norm_topk_prob,
+                         inp.get("sel_bias"), inp.get("logit_offset"))
+    idx, w = routing.topk_idx, routing.topk_w
+    E = inp["w1"].shape[0]
+    dx = np.zeros((T, d))
+    dw1 = np.zeros(_as64(inp["w1"]).shape)
+    dw3 = np.zeros_like(dw1)
+    dw2 = np.zeros(_as64(inp["w2"]).shape)
+    dtopk_w = np.zeros((T, top_k))
+    for e in range(E):
+        rows, cols = np.nonzero(idx == e)
+        if rows.size == 0:
+            continue
+        xr = x[rows]
+        y = swiglu_expert(xr, inp["w1"][e], inp["w3"][e], inp["w2"][e])
+        dtopk_w[rows, cols] = np.sum(dout[rows] * y, axis=1)
+        dy = w[rows, cols][:, None] * dout[rows]
+        gx, g1, g3, g2 = _swiglu_expert_backward(xr, inp["w1"][e], inp["w3"][e],
+                                                 inp["w2"][e], dy)
+        np.add.at(dx, rows, gx)
+        dw1[e] += g1
+        dw3[e] += g3
+        dw2[e] += g2
+    out = {"dw1": dw1, "dw3": dw3, "dw2": dw2, "dtopk_w": dtopk_w}
+    if "ws1" in inp:
+        gx, g1, g3, g2 = _swiglu_expert_backward(x, inp["ws1"], inp["ws3"], inp["ws2"], dout)
+        dx += gx
+        out.update(dws1=g1, dws3=g3, dws2=g2)
+    # router
+    s = routing.scores
+    ds = np.zeros((T, E))
+    rr = np.arange(T)[:, None]
+    if norm_topk_prob:
+        ssel = np.take_along_axis(s, idx, axis=1)
+        denom = ssel.sum(axis=1, keepdims=True) + 1e-9
+        ds[rr, idx] = (dtopk_w - np.sum(dtopk_w * w, axis=1, keepdims=True)) / denom
+    else:
+        ds[rr, idx] = dtopk_w
+    if gate == GATE_SIGMOID:
+        dlogits = ds * s * (1.0 - s)
+    else:
+        dlogits = s * (ds - np.sum(ds * s, axis=1, keepdims=True))
+    out["dlogits"] = dlogits
+    out["dw_router"] = dlogits.T @ x
+    dx += dlogits @ _as64(inp["w_router"])
+    out["dx"] = dx
+    return out

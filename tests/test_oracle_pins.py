@@ -555,3 +555,73 @@ def test_token_constant_noise_equals_bias():
     np.testing.assert_array_equal(r_bias.topk_w, r_noise.topk_w)
     # and it moves nothing but the selection
     np.testing.assert_array_equal(r_noise.scores, O.router(x, w, 3, O.GATE_SIGMOID, True).scores)
+
+
+# --------------------------------------------------------------------------- #
+# layer backward                                                              #
+# --------------------------------------------------------------------------- #
+def _loss(inp, dout, top_k, gate, renorm, idx_fixed):
+    out, r = O.moe_forward(inp, top_k, gate, renorm)
+    assert np.array_equal(r.topk_idx, idx_fixed), "perturbation changed the selection"
+    return float(np.sum(dout * out))
+
+
+@pytest.mark.parametrize("gate,renorm,shared", [(O.GATE_SIGMOID, True, True),
+                                                (O.GATE_SOFTMAX, True, False),
+                                                (O.GATE_SOFTMAX, False, True),
+                                                (O.GATE_SIGMOID, False, False)])
+def test_backward_matches_central_differences(gate, renorm, shared):
+    """Every gradient the oracle returns equals the central difference of
+    <dout, out> computed from the forward alone.  Catches: a dropped term of
+    the SwiGLU chain rule, the renormalisation Jacobian, a transposed weight
+    gradient, or a missing router / shared-expert contribution to dx."""
+    rng = np.random.default_rng(11 + gate + 2 * renorm)
+    T, d, E, F, k = 6, 5, 4, 3, 2
+    inp = _random_layer(rng, T, d, E, F, k, shared=shared, bias=True, offset=True)
+    dout = rng.standard_normal((T, d))
+    r = O.router(inp["x"], inp["w_router"], k, gate, renorm, inp["sel_bias"],
+                 inp["logit_offset"])
+    assert np.all(r.edge_gap > 1e-3)     # no selection change under the perturbation
+    g = O.moe_backward(inp, k, gate, renorm, dout)
+    names = ["x", "w_router", "w1", "w3", "w2"] + (["ws1", "ws3", "ws2"] if shared else [])
+    grad_key = {"x": "dx", "w_router": "dw_router", "w1": "dw1", "w3": "dw3", "w2": "dw2",
+                "ws1": "dws1", "ws3": "dws3", "ws2": "dws2"}
+    h = 1e-6
+    for name in names:
+        base = inp[name]
+        num = np.zeros(base.shape)
+        for pos in np.ndindex(base.shape):
+            p = dict(inp)
+            a = base.copy(); a[pos] += h; p[name] = a
+            lp = _loss(p, dout, k, gate, renorm, r.topk_idx)
+            a = base.copy(); a[pos] -= h; p[name] = a
+            lm = _loss(p, dout, k, gate, renorm, r.topk_idx)
+            num[pos] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[grad_key[name]], num, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def test_backward_bias_and_offset_get_no_gradient_through_selection():
+    """The bias only moves the selection: with the selection unchanged, the
+    loss does not depend on it at all (zero central difference).  Catches: the
+    bias leaking into the weights and hence into the gradients."""
+    rng = np.random.default_rng(5)
+    inp = _random_layer(rng, 6, 5, 4, 3, 2, bias=True)
+    dout = rng.standard_normal((6, 5))
+    r = O.router(inp["x"], inp["w_router"], 2, O.GATE_SIGMOID, True, inp["sel_bias"])
+    assert np.all(r.edge_gap > 1e-3)
+    l0 = _loss(inp, dout, 2, O.GATE_SIGMOID, True, r.topk_idx)
+    for e in range(4):
+        p = dict(inp)
+        b = inp["sel_bias"].copy(); b[e] += 1e-7; p["sel_bias"] = b
+        assert _loss(p, dout, 2, O.GATE_SIGMOID, True, r.topk_idx) == l0
+
+
+def test_backward_top1_renormalised_has_no_router_gradient():
+    """With top-1 and renormalisation every weight is s / (s + 1e-9), almost
+    exactly 1, so the router gradient is (almost exactly) zero.  Catches a
+    renormalisation Jacobian with the wrong sign or a missing term."""
+    rng = np.random.default_rng(9)
+    inp = _random_layer(rng, 8, 6, 5, 4, 1)
+    dout = rng.standard_normal((8, 6))
+    g = O.moe_backward(inp, 1, O.GATE_SOFTMAX, True, dout)
+    assert np.max(np.abs(g["dw_router"])) < 1e-7
