@@ -94,6 +94,17 @@ typedef struct {
   const void* ws2;
 } moe_expert_weights;
 
+/* Gradients of the expert weights: the same shapes and dtype as the
+ * weights in moe_expert_weights; dws* are NULL when n_shared == 0. */
+typedef struct {
+  void* dw1;
+  void* dw3;
+  void* dw2;
+  void* dws1;
+  void* dws3;
+  void* dws2;
+} moe_expert_grads;
+
 /* Bytes of workspace every call below needs for this configuration
  * (0 on an invalid configuration). */
 size_t moe_workspace_size(const moe_config* cfg);
@@ -306,6 +317,36 @@ moe_status moe_selftest_bounded_wait(void* ws, size_t ws_bytes, double limit_sec
 
 /* Static description of a status code. */
 const char* moe_status_string(moe_status s);
+
+/* Backward of the layer (bf16 layers; fp32 layers return
+ * MOE_ERR_UNSUPPORTED).  The pages train the layer (the "moe-200m-qwen3-100b"
+ * README trains SigmoidRouter models end to end; SpecForge PR #930 trains the
+ * qwen3 drafter); this is the gradient of <dout, out> for the forward above:
+ *   combine   dw[t, j] = <dout[t], y[t, j]>, expert output gradient w[t, j] dout[t],
+ *             shared expert output gradient dout[t];
+ *   experts   SwiGLU chain rule, silu'(g) = s(g) (1 + g (1 - s(g)));
+ *   router    no gradient through the selection (bias, noise); through the
+ *             weights w = s_picked / (sum + 1e-9) (or s_picked) with s the
+ *             sigmoid or the softmax over all E: dlogits, then
+ *             dw_router = dlogits^T x and dx += dlogits w_router (fp32).
+ * Inputs: the forward's x, w_router, logit_offset, weights, topk_idx,
+ * topk_w (as moe_forward returned them) and dout [T, d] act.  fws is the
+ * workspace of that moe_forward call, unchanged since (the backward reads the
+ * routed rows, their order and the saved activations from it; the forward
+ * must have run with its default dispatch, which writes the permuted copy of
+ * x).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
+ * 256-byte aligned; its first word is a device status word read with
+ * moe_device_status(bws, ...).
+ * Outputs: dx [T, d] act; dw_router [E, d] fp32; g->dw1, dw3 [E, F, d],
+ * dw2 [E, d, F] act (and the shared expert's).  Activation gradients are
+ * bf16 between the steps, the contractions accumulate in fp32 (tensor cores;
+ * the router's on CUDA cores in fp32). */
+size_t moe_backward_workspace_size(const moe_config* cfg);
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router,
+                        const float* logit_offset, const moe_expert_weights* w,
+                        const int32_t* topk_idx, const float* topk_w, const void* dout, void* dx,
+                        float* dw_router, const moe_expert_grads* g, void* fws, size_t fws_bytes,
+                        void* bws, size_t bws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -48,6 +48,10 @@ class MoEExpertWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w1", "w3", "w2", "ws1", "ws3", "ws2")]
 
 
+class MoEExpertGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("dw1", "dw3", "dw2", "dws1", "dws3", "dws2")]
+
+
 class MoERouterOpts(ctypes.Structure):
     _fields_ = [("bias_space", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("sel_noise", ctypes.c_void_p)]
@@ -77,6 +81,9 @@ _SIGNATURES = {
     "moe_router_refined_tokens": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_int32)]),
     "moe_selftest_bounded_wait": (_I32, [_VP, _SZ, _F64, _VP]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
+    "moe_backward_workspace_size": (_SZ, [_CFG]),
+    "moe_backward": (_I32, [_CFG, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP,
+                            ctypes.POINTER(MoEExpertGrads), _VP, _SZ, _VP, _SZ, _VP]),
 }
 
 _lib = None
@@ -247,6 +254,24 @@ def moe_forward(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, to
                            _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),
                            _p(topk_w), _p(counts), _p(ws),
                            _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_backward_workspace_size(cfg: MoEConfig) -> int:
+    return int(lib().moe_backward_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_backward(cfg, x, w_router, logit_offset, weights: Dict, topk_idx, topk_w, dout, dx,
+                 dw_router, grads: Dict, fws, bws, stream=None, check=True) -> int:
+    """Backward of the layer after moe_forward ran with workspace ``fws``;
+    ``grads`` maps dw1, dw3, dw2 (and dws1, dws3, dws2) to output tensors."""
+    w = expert_weights(weights)
+    g = MoEExpertGrads(*[_p(grads.get(n)) for n in ("dw1", "dw3", "dw2", "dws1", "dws3",
+                                                      "dws2")])
+    st = lib().moe_backward(ctypes.byref(cfg), _p(x), _p(w_router), _p(logit_offset),
+                            ctypes.byref(w), _p(topk_idx), _p(topk_w), _p(dout), _p(dx),
+                            _p(dw_router), ctypes.byref(g), _p(fws), _nbytes(fws), _p(bws),
+                            _nbytes(bws), _s(stream))
     return _check(st, check)
 
 

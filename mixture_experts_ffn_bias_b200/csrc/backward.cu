@@ -1,0 +1,465 @@
+// Backward pass of the MoE layer: the memory-bound steps and the fp32 router
+// gradient.  The contractions of the experts run on the tensor cores (the
+// plain grouped GEMM of grouped_gemm_sm100.cu for dH and dX, the K-grouped
+// GEMM of grouped_gemm_wgrad_sm100.cu for the weight gradients); this file
+// holds what feeds and finishes them:
+//   bwd_dy_kernel       dw[t, j] = <dout[t], y_perm[slot]>, dY[slot] = w[t, j] dout[t]
+//   transpose_kernel    batched bf16 transpose (weights, once per backward)
+//   gtranspose_kernel   rows of each group -> padded columns (the K-grouped
+//                       operands), zeros in the padding
+//   pad_offsets_kernel  padded column offsets of the groups
+//   swiglu_bwd_kernel   dG = dH * U * silu'(G), dU = dH * silu(G)
+//   dx_gather_kernel    dx[t] = sum_j dX[slot(t, j)] + dx_router[t] (+ dx_shared[t])
+//   router_dlogits_kernel  dlogits from dw through the (renormalised) gate
+//   sgemm_kernel        fp32 CUDA-core GEMM for the router gradients (the
+//                       router runs in fp32: "moe-200m-qwen3-100b" README,
+//                       "Per-layer numerics")
+// The chain rule is that of the layer in the "moe-200m-qwen3-100b" README
+// ("Architecture diagram", SigmoidRouter forward): out = shared(x) +
+// sum_j w_j expert_j(x), w = gate scores of the picked experts, renormalised.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "launch.cuh"
+
+namespace moe {
+namespace {
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(h[i]);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint4 o;
+  uint32_t* p = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    p[i] = *reinterpret_cast<uint32_t*>(&v);
+  }
+  return o;
+}
+
+// One warp per token.  oct = d / 8 (uint4 of 8 bf16 per lane step).
+__global__ void __launch_bounds__(256)
+bwd_dy_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y_perm,
+              const int32_t* __restrict__ slot_pos, const float* __restrict__ topk_w,
+              uint4* __restrict__ dy, float* __restrict__ dw, int T, int oct, int k) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const uint4* drow = dout + static_cast<size_t>(t) * oct;
+  for (int j = 0; j < k; ++j) {
+    const size_t p = static_cast<size_t>(t) * k + j;
+    const int r = slot_pos[p];
+    if (r < 0) {
+      if (lane == 0) dw[p] = 0.f;
+      continue;
+    }
+    const float w = topk_w[p];
+    const uint4* yrow = y_perm + static_cast<size_t>(r) * oct;
+    uint4* dyrow = dy + static_cast<size_t>(r) * oct;
+    float dot = 0.f;
+    for (int c = lane; c < oct; c += 32) {
+      float a[8], b[8], o[8];
+      unpack8(drow[c], a);
+      unpack8(__ldcs(yrow + c), b);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        dot = fmaf(a[i], b[i], dot);
+        o[i] = w * a[i];
+      }
+      dyrow[c] = pack8(o);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lane == 0) dw[p] = dot;
+  }
+}
+
+// out[b][c][col_off + r] = in[b][r][c] for r < rows, c < cols; 32 x 32 tiles.
+__global__ void __launch_bounds__(256)
+transpose_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols, long long in_bstride,
+                 __nv_bfloat16* __restrict__ out, int ldo, int col_off, long long out_bstride) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __nv_bfloat16 tile[32][34];
+  const int b = blockIdx.z;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  const __nv_bfloat16* src = in + b * in_bstride;
+  __nv_bfloat16* dst = out + b * out_bstride;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int r = r0 + i, c = c0 + tx;
+    if (r < rows && c < cols) tile[i][tx] = src[static_cast<size_t>(r) * cols + c];
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i, r = r0 + tx;
+    if (r < rows && c < cols) dst[static_cast<size_t>(c) * ldo + col_off + r] = tile[tx][i];
+  }
+}
+
+// Padded column offsets: poff[g + 1] = poff[g] + roundup(rows_g, 64).
+// offsets null: one group of rows_single rows.
+__global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int G, int rows_single,
+                                   int32_t* __restrict__ poff) {
+  pdl_trigger();
+  pdl_wait();
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int run = 0;
+  poff[0] = 0;
+  for (int g = 0; g < G; ++g) {
+    const int rows = offsets ? offsets[g + 1] - offsets[g] : rows_single;
+    run += (rows + 63) / 64 * 64;
+    poff[g + 1] = run;
+  }
+}
+
+// out [cols, kp]: column p of out is row src(p) of in [rows, cols], where
+// p = poff[g] + i < poff[g] + rows_g maps to row offsets[g] + i (gathered
+// through `gather` when not null), and every other p is zero.  The grid
+// covers kp x cols in 32 x 32 tiles.
+__global__ void __launch_bounds__(256)
+gtranspose_kernel(const __nv_bfloat16* __restrict__ in, int cols,
+                  const int32_t* __restrict__ offsets, int G, int rows_single,
+                  const int32_t* __restrict__ poff, const int32_t* __restrict__ gather,
+                  __nv_bfloat16* __restrict__ out, int kp) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ __nv_bfloat16 tile[32][34];
+  __shared__ int s_src[32];
+  const int p0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  if (ty == 0) {
+    const int p = p0 + tx;
+    int src = -1;
+    if (p < poff[G]) {
+      int lo = 0, hi = G - 1;   // last g with poff[g] <= p
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (poff[mid] <= p) lo = mid; else hi = mid - 1;
+      }
+      const int base = offsets ? offsets[lo] : 0;
+      const int rows = offsets ? offsets[lo + 1] - offsets[lo] : rows_single;
+      const int i = p - poff[lo];
+      if (i < rows) src = gather ? gather[base + i] : base + i;
+    }
+    s_src[tx] = src;
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int src = s_src[i], c = c0 + tx;
+    __nv_bfloat16 v = __float2bfloat16(0.f);
+    if (src >= 0 && c < cols) v = in[static_cast<size_t>(src) * cols + c];
+    tile[i][tx] = v;
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int c = c0 + i, p = p0 + tx;
+    if (c < cols && p < kp) out[static_cast<size_t>(c) * kp + p] = tile[tx][i];
+  }
+}
+
+// dGU [n, 2F]: columns [0, F) = dG, [F, 2F) = dU; G, U, dH [n, F].  fq = F / 8.
+__global__ void __launch_bounds__(256)
+swiglu_bwd_kernel(const uint4* __restrict__ G, const uint4* __restrict__ U,
+                  const uint4* __restrict__ dH, uint4* __restrict__ dGU, long long n8, int fq) {
+  pdl_trigger();
+  pdl_wait();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / fq;
+    const int c = static_cast<int>(i - r * fq);
+    float g[8], u[8], dh[8], dg[8], du[8];
+    unpack8(G[i], g);
+    unpack8(U[i], u);
+    unpack8(dH[i], dh);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float s = 1.0f / (1.0f + expf(-g[q]));
+      du[q] = dh[q] * g[q] * s;
+      dg[q] = dh[q] * u[q] * (s * (1.0f + g[q] * (1.0f - s)));
+    }
+    dGU[r * 2 * fq + c] = pack8(dg);
+    dGU[r * 2 * fq + fq + c] = pack8(du);
+  }
+}
+
+// One warp per token: dx = sum_j dX[slot] + dxr (fp32) + dxs (bf16, may be null).
+__global__ void __launch_bounds__(256)
+dx_gather_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ slot_pos,
+                 const float4* __restrict__ dxr, const uint4* __restrict__ dxs,
+                 uint4* __restrict__ dx, int T, int oct, int k) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  for (int c = lane; c < oct; c += 32) {
+    float acc[8];
+    const float4 a = dxr[(static_cast<size_t>(t) * oct + c) * 2];
+    const float4 b = dxr[(static_cast<size_t>(t) * oct + c) * 2 + 1];
+    acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+    acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    if (dxs) {
+      float s[8];
+      unpack8(dxs[static_cast<size_t>(t) * oct + c], s);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += s[i];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int r = slot_pos[static_cast<size_t>(t) * k + j];
+      if (r < 0) continue;
+      float v[8];
+      unpack8(dxp[static_cast<size_t>(r) * oct + c], v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+    }
+    dx[static_cast<size_t>(t) * oct + c] = pack8(acc);
+  }
+}
+
+constexpr int kMaxLane = 8;   // E <= 256
+
+// One warp per token.  logits [T, E] fp32 (no offset), offset [E] or null.
+__global__ void __launch_bounds__(256)
+router_dlogits_kernel(const float* __restrict__ logits, const float* __restrict__ offset,
+                      const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_w,
+                      const float* __restrict__ dw, int T, int E, int k, int gate, int renorm,
+                      float* __restrict__ dlogits) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  float s[kMaxLane], ds[kMaxLane];
+  float lmax = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMaxLane; ++i) {
+    const int e = lane + 32 * i;
+    s[i] = e < E ? logits[static_cast<size_t>(t) * E + e] + (offset ? offset[e] : 0.f)
+                 : -INFINITY;
+    lmax = fmaxf(lmax, s[i]);
+    ds[i] = 0.f;
+  }
+  if (gate == 1) {
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i) s[i] = 1.0f / (1.0f + expf(-s[i]));   // 0 past E
+  } else {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i) {
+      s[i] = expf(s[i] - lmax);
+      sum += s[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i) s[i] /= sum;
+  }
+  // the picked experts' scores, their sum and sum_j dw_j w_j
+  float ssel = 0.f, dsum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    const size_t p = static_cast<size_t>(t) * k + j;
+    const int e = topk_idx[p];
+    float se = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i)
+      if (lane + 32 * i == e) se = s[i];
+    se = __shfl_sync(0xffffffffu, se, e & 31);
+    ssel += se;
+    dsum += dw[p] * topk_w[p];
+  }
+  for (int j = 0; j < k; ++j) {
+    const size_t p = static_cast<size_t>(t) * k + j;
+    const int e = topk_idx[p];
+    const float g = renorm ? (dw[p] - dsum) / (ssel + 1e-9f) : dw[p];
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i)
+      if (lane + 32 * i == e) ds[i] += g;
+  }
+  float dot = 0.f;
+  if (gate == 0) {
+#pragma unroll
+    for (int i = 0; i < kMaxLane; ++i) dot += ds[i] * s[i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+#pragma unroll
+  for (int i = 0; i < kMaxLane; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E)
+      dlogits[static_cast<size_t>(t) * E + e] =
+          gate == 1 ? ds[i] * s[i] * (1.0f - s[i]) : s[i] * (ds[i] - dot);
+  }
+}
+
+// fp32 CUDA-core GEMM, split over K: part[z][m][n] = sum_{k in slice z} A(m, k) B(k, n).
+// A(m, k) = a[m * lda + k] (A_T: a[k * lda + m]), fp32; B(k, n) = b[k * ldb + n], bf16.
+// 64 x 64 tile per block, 256 threads with 4 x 4 outputs each.
+template <bool A_T>
+__global__ void __launch_bounds__(256)
+sgemm_kernel(const float* __restrict__ a, int lda, const __nv_bfloat16* __restrict__ b, int ldb,
+             int M, int N, int K, int kslice, float* __restrict__ part) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ float As[16][64 + 4];
+  __shared__ float Bs[16][64 + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int kbeg = blockIdx.z * kslice, kend = min(K, kbeg + kslice);
+  float acc[4][4] = {};
+  for (int k0 = kbeg; k0 < kend; k0 += 16) {
+    for (int i = tid; i < 16 * 64; i += 256) {
+      const int kk = i / 64, mm = i % 64;
+      const int k = k0 + kk, m = m0 + mm;
+      float v = 0.f;
+      if (k < kend && m < M) v = A_T ? a[static_cast<size_t>(k) * lda + m]
+                                     : a[static_cast<size_t>(m) * lda + k];
+      As[kk][mm] = v;
+      const int n = n0 + mm;
+      Bs[kk][mm] = (k < kend && n < N) ? __bfloat162float(b[static_cast<size_t>(k) * ldb + n])
+                                       : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = As[kk][ty * 4 + i];
+        bv[i] = Bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  float* out = part + static_cast<size_t>(blockIdx.z) * M * N;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) out[static_cast<size_t>(m) * N + n] = acc[i][j];
+    }
+  }
+}
+
+// out[i] = sum_z part[z][i] (fixed order)
+__global__ void __launch_bounds__(256)
+sum_slices_kernel(const float* __restrict__ part, int slices, long long n,
+                  float* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int z = 0; z < slices; ++z) s += part[z * n + i];
+    out[i] = s;
+  }
+}
+
+int grid_1d(long long n) {
+  const long long b = (n + 255) / 256;
+  return static_cast<int>(b < 4096 ? (b > 0 ? b : 1) : 4096);
+}
+
+}  // namespace
+
+cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos,
+                   const float* topk_w, void* dy, float* dw, int T, int d, int k,
+                   cudaStream_t stream) {
+  const int warps = 8;
+  return launch_pdl(bwd_dy_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0, stream,
+                    static_cast<const uint4*>(dout), static_cast<const uint4*>(y_perm), slot_pos,
+                    topk_w, static_cast<uint4*>(dy), dw, T, d / 8, k);
+}
+
+cudaError_t transpose_bf16(const void* in, int batches, int rows, int cols, void* out, int ldo,
+                           int col_off, cudaStream_t stream) {
+  const dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches);
+  return launch_pdl(transpose_kernel, grid, dim3(256), 0, stream,
+                    static_cast<const __nv_bfloat16*>(in), rows, cols,
+                    static_cast<long long>(rows) * cols, static_cast<__nv_bfloat16*>(out), ldo,
+                    col_off, static_cast<long long>(cols) * ldo);
+}
+
+cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,
+                        cudaStream_t stream) {
+  return launch_pdl(pad_offsets_kernel, dim3(1), dim3(32), 0, stream, offsets, G, rows_single,
+                    poff);
+}
+
+cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,
+                            int rows_single, const int32_t* poff, const int32_t* gather,
+                            void* out, int kp, cudaStream_t stream) {
+  const dim3 grid((kp + 31) / 32, (cols + 31) / 32);
+  return launch_pdl(gtranspose_kernel, grid, dim3(256), 0, stream,
+                    static_cast<const __nv_bfloat16*>(in), cols, offsets, G, rows_single, poff,
+                    gather, static_cast<__nv_bfloat16*>(out), kp);
+}
+
+cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
+                       int F, cudaStream_t stream) {
+  const long long n8 = n * (F / 8);
+  return launch_pdl(swiglu_bwd_kernel, dim3(grid_1d(n8)), dim3(256), 0, stream,
+                    static_cast<const uint4*>(G), static_cast<const uint4*>(U),
+                    static_cast<const uint4*>(dH), static_cast<uint4*>(dGU), n8, F / 8);
+}
+
+cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr, const void* dxs,
+                      void* dx, int T, int d, int k, cudaStream_t stream) {
+  const int warps = 8;
+  return launch_pdl(dx_gather_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0, stream,
+                    static_cast<const uint4*>(dxp), slot_pos, reinterpret_cast<const float4*>(dxr),
+                    static_cast<const uint4*>(dxs), static_cast<uint4*>(dx), T, d / 8, k);
+}
+
+cudaError_t router_dlogits(const float* logits, const float* offset, const int32_t* topk_idx,
+                           const float* topk_w, const float* dw, int T, int E, int k, int gate,
+                           int renorm, float* dlogits, cudaStream_t stream) {
+  const int warps = 8;
+  return launch_pdl(router_dlogits_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
+                    stream, logits, offset, topk_idx, topk_w, dw, T, E, k, gate, renorm,
+                    dlogits);
+}
+
+int sgemm_slices(int K) {
+  int s = (K + 2047) / 2048;
+  return s < 1 ? 1 : (s > 16 ? 16 : s);
+}
+
+cudaError_t sgemm_f32(bool a_t, const float* a, int lda, const void* b, int ldb, int M, int N,
+                      int K, float* part, float* out, cudaStream_t stream) {
+  const int slices = sgemm_slices(K);
+  const int kslice = ((K + slices - 1) / slices + 15) / 16 * 16;
+  const dim3 grid((N + 63) / 64, (M + 63) / 64, slices);
+  if (slices == 1) part = out;   // one slice: the partial sum is the result
+  cudaError_t e =
+      a_t ? launch_pdl(sgemm_kernel<true>, grid, dim3(256), 0, stream, a, lda,
+                       static_cast<const __nv_bfloat16*>(b), ldb, M, N, K, kslice, part)
+          : launch_pdl(sgemm_kernel<false>, grid, dim3(256), 0, stream, a, lda,
+                       static_cast<const __nv_bfloat16*>(b), ldb, M, N, K, kslice, part);
+  if (e != cudaSuccess || slices == 1) return e;
+  const long long n = static_cast<long long>(M) * N;
+  return launch_pdl(sum_slices_kernel, dim3(grid_1d(n)), dim3(256), 0, stream, part, slices, n,
+                    out);
+}
+
+}  // namespace moe

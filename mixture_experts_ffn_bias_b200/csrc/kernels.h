@@ -106,6 +106,35 @@ cudaError_t grouped_down_f32(const float* A, int64_t a_rows, const int32_t* offs
                              int num_groups, int rows_single, const float* W2, int N, int K,
                              float* Y, cudaStream_t stream);
 
+// Backward -------------------------------------------------------------------
+// K-grouped weight gradient C_g [M, N] = A_g B_g^T over the padded column
+// ranges [poff[g], poff[g+1]) of A [M, kp] and B [N, kp]; C [G, M, N] bf16.
+cudaError_t grouped_wgrad_bf16(const void* A, const void* B, int64_t kp, const int32_t* poff,
+                               int G, int M, int N, void* C, uint32_t* status,
+                               cudaStream_t stream);
+cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos,
+                   const float* topk_w, void* dy, float* dw, int T, int d, int k,
+                   cudaStream_t stream);
+cudaError_t transpose_bf16(const void* in, int batches, int rows, int cols, void* out, int ldo,
+                           int col_off, cudaStream_t stream);
+cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,
+                        cudaStream_t stream);
+cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,
+                            int rows_single, const int32_t* poff, const int32_t* gather,
+                            void* out, int kp, cudaStream_t stream);
+cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
+                       int F, cudaStream_t stream);
+cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr, const void* dxs,
+                      void* dx, int T, int d, int k, cudaStream_t stream);
+cudaError_t router_dlogits(const float* logits, const float* offset, const int32_t* topk_idx,
+                           const float* topk_w, const float* dw, int T, int E, int k, int gate,
+                           int renorm, float* dlogits, cudaStream_t stream);
+int sgemm_slices(int K);
+// out [M, N] fp32 = A B with A(m, k) fp32 (a_t: stored [K, M]) and B [K, N] bf16;
+// part holds sgemm_slices(K) x M x N partial sums (unused when that is 1).
+cudaError_t sgemm_f32(bool a_t, const float* a, int lda, const void* b, int ldb, int M, int N,
+                      int K, float* part, float* out, cudaStream_t stream);
+
 // Combine / bias ---------------------------------------------------------------
 cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, const float* topk_w,
                     const void* y_shared, void* out, int T, int d, int k, cudaStream_t stream);

@@ -288,6 +288,165 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   return MOE_OK;
 }
 
+// Workspace of moe_backward (separate from the forward's, which it reads).
+struct BLayout {
+  size_t status, dw, logits, dlogits, part, dxr, poff, poff_sh, w2t, w13t, dy, dh, gb, ub, dgu,
+      dxp, dyT, hT, dguT, xT, ws2t, ws13t, dh_sh, g_sh, u_sh, dgu_sh, dxs, doutT, hshT, dgushT,
+      xTs, total;
+  int64_t kp, tp;
+};
+
+BLayout blayout(const moe_config& c) {
+  const size_t T = static_cast<size_t>(c.T), d = c.d_model, E = c.n_experts, F = c.d_ff,
+               k = c.top_k, R = T * k;
+  const size_t Fs = c.n_shared ? static_cast<size_t>(c.d_ff_shared) : 0;
+  BLayout B{};
+  // every group's column range is padded to a multiple of 64
+  B.kp = static_cast<int64_t>((R + 63 * E + 63) / 64 * 64);
+  B.tp = static_cast<int64_t>((T + 63) / 64 * 64);
+  const size_t kp = static_cast<size_t>(B.kp), tp = static_cast<size_t>(B.tp);
+  size_t o = 0;
+  B.status = o;  o += up(2 * sizeof(uint32_t));
+  B.dw = o;      o += up(R * 4);
+  B.logits = o;  o += up(T * E * 4);
+  B.dlogits = o; o += up(T * E * 4);
+  B.part = o;    o += up(static_cast<size_t>(moe::sgemm_slices(c.T)) * E * d * 4);
+  B.dxr = o;     o += up(T * d * 4);
+  B.poff = o;    o += up((E + 1) * 4);
+  B.poff_sh = o; o += up(2 * 4);
+  B.w2t = o;     o += up(E * F * d * 2);
+  B.w13t = o;    o += up(E * d * 2 * F * 2);
+  B.dy = o;      o += up(R * d * 2);
+  B.dh = o;      o += up(R * F * 2);
+  B.gb = o;      o += up(R * F * 2);
+  B.ub = o;      o += up(R * F * 2);
+  B.dgu = o;     o += up(R * 2 * F * 2);
+  B.dxp = o;     o += up(R * d * 2);
+  B.dyT = o;     o += up(d * kp * 2);
+  B.hT = o;      o += up(F * kp * 2);
+  B.dguT = o;    o += up(2 * F * kp * 2);
+  B.xT = o;      o += up(d * kp * 2);
+  B.ws2t = o;    o += up(Fs * d * 2);
+  B.ws13t = o;   o += up(d * 2 * Fs * 2);
+  B.dh_sh = o;   o += up(T * Fs * 2);
+  B.g_sh = o;    o += up(T * Fs * 2);
+  B.u_sh = o;    o += up(T * Fs * 2);
+  B.dgu_sh = o;  o += up(T * 2 * Fs * 2);
+  B.dxs = o;     o += up(Fs ? T * d * 2 : 0);
+  B.doutT = o;   o += up(Fs ? d * tp * 2 : 0);
+  B.hshT = o;    o += up(Fs * tp * 2);
+  B.dgushT = o;  o += up(2 * Fs * tp * 2);
+  B.xTs = o;     o += up(Fs ? d * tp * 2 : 0);
+  B.total = o;
+  return B;
+}
+
+// The layer's backward (bf16 layers).  fws holds the state of the forward:
+// offsets, slot_pos, perm_src, x_perm, h, y_perm (and h_sh).
+moe_status backward_impl(const moe_config* c, const void* x, const void* w_router,
+                         const float* logit_offset, const moe_expert_weights* w,
+                         const int32_t* topk_idx, const float* topk_w, const void* dout,
+                         void* dx, float* dw_router, const moe_expert_grads* g, void* fws,
+                         void* bws, cudaStream_t s) {
+  const Layout L = layout(*c);
+  const BLayout B = blayout(*c);
+  const int T = c->T, d = c->d_model, E = c->n_experts, F = c->d_ff, k = c->top_k;
+  const int64_t R = static_cast<int64_t>(T) * k;
+  uint32_t* status = at<uint32_t>(bws, B.status);
+  const int32_t* offsets = at<int32_t>(fws, L.offsets);
+  const int32_t* slot_pos = at<int32_t>(fws, L.slot_pos);
+  const int32_t* perm_src = at<int32_t>(fws, L.perm_src);
+  const void* x_perm = at<void>(fws, L.x_perm);
+  const void* h = at<void>(fws, L.h);
+  const void* y_perm = at<void>(fws, L.y_perm);
+  float* dw = at<float>(bws, B.dw);
+  int32_t* poff = at<int32_t>(bws, B.poff);
+  // combine: dw and the experts' output gradients
+  MOE_TRY(moe::bwd_dy(dout, y_perm, slot_pos, topk_w, at<void>(bws, B.dy), dw, T, d, k, s));
+  // transposed weights (W2^T [E, F, d]; [W1^T | W3^T] [E, d, 2F])
+  MOE_TRY(moe::transpose_bf16(w->w2, E, d, F, at<void>(bws, B.w2t), d, 0, s));
+  MOE_TRY(moe::transpose_bf16(w->w1, E, F, d, at<void>(bws, B.w13t), 2 * F, 0, s));
+  MOE_TRY(moe::transpose_bf16(w->w3, E, F, d, at<void>(bws, B.w13t), 2 * F, F, s));
+  // dH = dY W2 ; G, U recomputed ; dG, dU ; dX = [dG | dU] [W1 ; W3]
+  MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dy), R, offsets, E, 0, at<void>(bws, B.w2t), F,
+                                 d, at<void>(bws, B.dh), status, s));
+  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w1, F, d, at<void>(bws, B.gb),
+                                 status, s));
+  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w3, F, d, at<void>(bws, B.ub),
+                                 status, s));
+  MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.gb), at<void>(bws, B.ub), at<void>(bws, B.dh),
+                          at<void>(bws, B.dgu), R, F, s));
+  MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, at<void>(bws, B.w13t),
+                                 d, 2 * F, at<void>(bws, B.dxp), status, s));
+  // weight gradients over each expert's rows (transposed, padded operands)
+  MOE_TRY(moe::pad_offsets(offsets, E, 0, poff, s));
+  MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dy), d, offsets, E, 0, poff, nullptr,
+                               at<void>(bws, B.dyT), static_cast<int>(B.kp), s));
+  MOE_TRY(moe::gtranspose_bf16(h, F, offsets, E, 0, poff, nullptr, at<void>(bws, B.hT),
+                               static_cast<int>(B.kp), s));
+  MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dgu), 2 * F, offsets, E, 0, poff, nullptr,
+                               at<void>(bws, B.dguT), static_cast<int>(B.kp), s));
+  MOE_TRY(moe::gtranspose_bf16(x, d, offsets, E, 0, poff, perm_src, at<void>(bws, B.xT),
+                               static_cast<int>(B.kp), s));
+  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dyT), at<void>(bws, B.hT), B.kp, poff, E, d, F,
+                                  g->dw2, status, s));
+  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dguT), at<void>(bws, B.xT), B.kp, poff, E, F,
+                                  d, g->dw1, status, s));
+  MOE_TRY(moe::grouped_wgrad_bf16(at<uint8_t>(bws, B.dguT) + static_cast<size_t>(F) * B.kp * 2,
+                                  at<void>(bws, B.xT), B.kp, poff, E, F, d, g->dw3, status, s));
+  // shared expert (weight 1, all tokens)
+  const void* dxs = nullptr;
+  if (c->n_shared) {
+    const int Fs = c->d_ff_shared;
+    int32_t* poff_sh = at<int32_t>(bws, B.poff_sh);
+    MOE_TRY(moe::transpose_bf16(w->ws2, 1, d, Fs, at<void>(bws, B.ws2t), d, 0, s));
+    MOE_TRY(moe::transpose_bf16(w->ws1, 1, Fs, d, at<void>(bws, B.ws13t), 2 * Fs, 0, s));
+    MOE_TRY(moe::transpose_bf16(w->ws3, 1, Fs, d, at<void>(bws, B.ws13t), 2 * Fs, Fs, s));
+    MOE_TRY(moe::grouped_down_bf16(dout, T, nullptr, 1, T, at<void>(bws, B.ws2t), Fs, d,
+                                   at<void>(bws, B.dh_sh), status, s));
+    MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws1, Fs, d, at<void>(bws, B.g_sh),
+                                   status, s));
+    MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws3, Fs, d, at<void>(bws, B.u_sh),
+                                   status, s));
+    MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.g_sh), at<void>(bws, B.u_sh),
+                            at<void>(bws, B.dh_sh), at<void>(bws, B.dgu_sh), T, Fs, s));
+    MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dgu_sh), T, nullptr, 1, T,
+                                   at<void>(bws, B.ws13t), d, 2 * Fs, at<void>(bws, B.dxs),
+                                   status, s));
+    dxs = at<void>(bws, B.dxs);
+    MOE_TRY(moe::pad_offsets(nullptr, 1, T, poff_sh, s));
+    const int tp = static_cast<int>(B.tp);
+    MOE_TRY(moe::gtranspose_bf16(dout, d, nullptr, 1, T, poff_sh, nullptr,
+                                 at<void>(bws, B.doutT), tp, s));
+    MOE_TRY(moe::gtranspose_bf16(at<void>(fws, L.h_sh), Fs, nullptr, 1, T, poff_sh, nullptr,
+                                 at<void>(bws, B.hshT), tp, s));
+    MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dgu_sh), 2 * Fs, nullptr, 1, T, poff_sh,
+                                 nullptr, at<void>(bws, B.dgushT), tp, s));
+    MOE_TRY(moe::gtranspose_bf16(x, d, nullptr, 1, T, poff_sh, nullptr, at<void>(bws, B.xTs), tp,
+                                 s));
+    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.doutT), at<void>(bws, B.hshT), tp, poff_sh,
+                                    1, d, Fs, g->dws2, status, s));
+    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgushT), at<void>(bws, B.xTs), tp, poff_sh,
+                                    1, Fs, d, g->dws1, status, s));
+    MOE_TRY(moe::grouped_wgrad_bf16(at<uint8_t>(bws, B.dgushT) + static_cast<size_t>(Fs) * tp * 2,
+                                    at<void>(bws, B.xTs), tp, poff_sh, 1, Fs, d, g->dws3, status,
+                                    s));
+  }
+  // router (fp32): recomputed logits, dlogits, dW_router = dlogits^T x,
+  // dx_router = dlogits W_router
+  float* logits = at<float>(bws, B.logits);
+  float* dlogits = at<float>(bws, B.dlogits);
+  MOE_TRY(moe::router_logits_tc(x, T, w_router, E, d, logits, status, s));
+  MOE_TRY(moe::router_dlogits(logits, logit_offset, topk_idx, topk_w, dw, T, E, k, c->gate,
+                              c->norm_topk_prob, dlogits, s));
+  MOE_TRY(moe::sgemm_f32(true, dlogits, E, x, d, E, d, T, at<float>(bws, B.part), dw_router, s));
+  MOE_TRY(moe::sgemm_f32(false, dlogits, E, w_router, d, T, d, E, at<float>(bws, B.part),
+                         at<float>(bws, B.dxr), s));
+  MOE_TRY(moe::dx_gather(at<void>(bws, B.dxp), slot_pos, at<float>(bws, B.dxr), dxs, dx, T, d, k,
+                         s));
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -507,6 +666,38 @@ moe_status moe_router_refined_tokens(void* ws, size_t ws_bytes, void* stream, in
   MOE_TRY(cudaMemcpy(count, static_cast<int32_t*>(ws) + 1, sizeof(int32_t),
                      cudaMemcpyDeviceToHost));
   return MOE_OK;
+}
+
+size_t moe_backward_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;
+  return blayout(*cfg).total;
+}
+
+moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router,
+                        const float* logit_offset, const moe_expert_weights* w,
+                        const int32_t* topk_idx, const float* topk_w, const void* dout, void* dx,
+                        float* dw_router, const moe_expert_grads* g, void* fws, size_t fws_bytes,
+                        void* bws, size_t bws_bytes, void* stream) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  if (!x || !w_router || !topk_idx || !topk_w || !dout || !dx || !dw_router || !g || !g->dw1 ||
+      !g->dw3 || !g->dw2 || (cfg->n_shared && (!g->dws1 || !g->dws3 || !g->dws2)))
+    return MOE_ERR_INVALID;
+  if ((st = check_weights(cfg, w)) != MOE_OK) return st;
+  if (!aligned16(x) || !aligned16(w_router) || !aligned16(dout) || !aligned16(dx) ||
+      !aligned16(dw_router) || !aligned4(topk_idx) || !aligned4(topk_w) || !aligned16(g->dw1) ||
+      !aligned16(g->dw3) || !aligned16(g->dw2) || (logit_offset && !aligned4(logit_offset)) ||
+      (cfg->n_shared && (!aligned16(g->dws1) || !aligned16(g->dws3) || !aligned16(g->dws2))))
+    return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, fws, fws_bytes)) != MOE_OK) return st;
+  if (bws == nullptr || (reinterpret_cast<uintptr_t>(bws) & (kAlign - 1))) return MOE_ERR_INVALID;
+  if (bws_bytes < blayout(*cfg).total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = S(stream);
+  if ((st = clear_status(bws, s)) != MOE_OK) return st;
+  return backward_impl(cfg, x, w_router, logit_offset, w, topk_idx, topk_w, dout, dx, dw_router,
+                       g, fws, bws, s);
 }
 
 const char* moe_status_string(moe_status s) {

@@ -61,6 +61,24 @@ class MoELayer:
                       self.topk_idx, self.topk_w, self.counts, self.ws, stream)
         return self.out if out is None else out
 
+    def backward(self, dout: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
+        """Gradients of <dout, out> for the last forward (bf16 layers): dx,
+        dw_router (fp32) and dw1, dw3, dw2 (and the shared expert's)."""
+        if not hasattr(self, "bws"):
+            n = B.moe_backward_workspace_size(self.cfg)
+            if n == 0:
+                raise B.MoEError(B.MOE_ERR_UNSUPPORTED, "backward needs a bf16 layer")
+            self.bws = torch.empty((n,), dtype=torch.uint8, device=self.device)
+        g = {"dx": torch.empty_like(self.x),
+             "dw_router": torch.empty(self.w_router.shape, dtype=torch.float32,
+                                      device=self.device)}
+        for k, v in self.weights.items():
+            g["d" + k] = torch.empty_like(v)
+        B.moe_backward(self.cfg, self.x, self.w_router, self.logit_offset, self.weights,
+                       self.topk_idx, self.topk_w, dout, g["dx"], g["dw_router"], g, self.ws,
+                       self.bws, stream)
+        return g
+
     def bias_update(self, counts: Optional[torch.Tensor] = None, rate=1e-3, starved_frac=0.1,
                     starved_add=0.5, clamp=10.0, stream=None):
         if self.sel_bias is None:

@@ -124,3 +124,26 @@ def test_status_strings(lib):
     for s in range(7):
         assert B.status_string(s) and B.status_string(s) != "unknown status"
     assert B.status_string(99) == "unknown status"
+
+
+def test_backward_arguments_validated(lib):
+    shape = I.WORKLOADS["page2"]
+    cfg = B.config_from_shape(shape)
+    ok = _FakeTensor(1 << 20, 1 << 40)
+    w = {"w1": ok, "w3": ok, "w2": ok, "ws1": ok, "ws3": ok, "ws2": ok}
+    g = {"dw1": ok, "dw3": ok, "dw2": ok, "dws1": ok, "dws3": ok, "dws2": ok}
+    # shared-expert gradients missing for a layer with a shared expert
+    g2 = {"dw1": ok, "dw3": ok, "dw2": ok}
+    st = B.moe_backward(cfg, ok, ok, None, w, ok, ok, ok, ok, ok, g2, ok, ok, stream=0,
+                        check=False)
+    assert st == B.MOE_ERR_INVALID
+    # backward scratch too small
+    st = B.moe_backward(cfg, ok, ok, None, w, ok, ok, ok, ok, ok, g, ok, _FakeTensor(1 << 20, 256),
+                        stream=0, check=False)
+    assert st == B.MOE_ERR_WORKSPACE
+    # fp32 layers have no backward
+    cfg32 = B.config_from_shape(I.WORKLOADS["tiny"])
+    assert B.moe_backward_workspace_size(cfg32) == 0
+    st = B.moe_backward(cfg32, ok, ok, None, w, ok, ok, ok, ok, ok, g, ok, ok, stream=0,
+                        check=False)
+    assert st == B.MOE_ERR_UNSUPPORTED
