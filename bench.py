@@ -236,6 +236,54 @@ def run_reference(args, shape, rank: int, world: int):
 # --------------------------------------------------------------------------- #
 # GPU arm                                                                      #
 # --------------------------------------------------------------------------- #
+def run_backward(args, shape):
+    """--mode backward (one GPU): moe_backward after a forward, timed with
+    CUDA events over --steps calls after --warmup calls.  The expert GEMM
+    FLOPs of a backward are 16 R d F (+ 16 T d Fs for a shared expert):
+    dH, the recomputed G and U, dX (K = 2F) and the three weight gradients."""
+    import numpy as np
+    import torch
+    from mixture_experts_ffn_bias_b200 import binding as B
+    from mixture_experts_ffn_bias_b200.layer import MoELayer, to_device
+
+    dev = torch.device("cuda", 0)
+    host = I.make_inputs(shape)
+    layer = MoELayer(shape, host, dev)
+    if layer.sel_bias is None:
+        layer.sel_bias = torch.zeros(shape.n_experts, dtype=torch.float32, device=dev)
+    dout = to_device(I.round_to_bf16(np.random.default_rng(shape.seed + 77).standard_normal(
+        (shape.T, shape.d_model)).astype(np.float32)), torch.bfloat16, dev)
+    layer.forward()
+    for _ in range(args.warmup):
+        layer.backward(dout)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer.backward(dout)
+    e1.record()
+    torch.cuda.synchronize(dev)
+    st, flags = B.moe_device_status(layer.bws)
+    if st != B.MOE_OK:
+        raise SystemExit(f"device status after the backward: {B.status_string(st)} ({flags})")
+    ms = e0.elapsed_time(e1) / args.steps
+    R = shape.T * shape.top_k
+    fl = 16.0 * R * shape.d_model * shape.d_ff
+    if shape.n_shared:
+        fl += 16.0 * shape.T * shape.d_model * shape.d_ff_shared
+    peaks, kind = load_peaks()
+    sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    tf = fl / (ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "MoE-layer backward tokens/sec (moe_backward after moe_forward) on 1 B200",
+        "value": shape.T / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": describe(shape)},
+        "expert_gemm": {"tflops": tf, "frac_of_sustained": tf / sus,
+                        "peaks": kind, "flops_per_step": fl},
+        "workspace_gb": layer.bws.numel() / 1e9}), flush=True)
+
+
 def run_ours(args, shape, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -377,6 +425,8 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
+                    help="backward: time moe_backward instead (one GPU, its own JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -388,6 +438,10 @@ def main():
         shape = shape.replace(T=args.tokens)
     if args.impl == "reference":
         run_reference(args, shape, rank, world)
+        return
+    if args.mode == "backward":
+        if world == 1:
+            run_backward(args, shape)
         return
     if world > 1:
         import datetime

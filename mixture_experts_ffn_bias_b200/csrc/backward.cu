@@ -84,27 +84,55 @@ bwd_dy_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y_perm,
   }
 }
 
-// out[b][c][col_off + r] = in[b][r][c] for r < rows, c < cols; 32 x 32 tiles.
+// Transposes move 64 x 64 bf16 tiles through shared memory: 16-byte global
+// loads of the source rows (a warp reads four full 128-byte rows), and
+// 128-byte output rows written as bf16 pairs by a warp.  The tile's rows are
+// 66 elements apart (33 words), so the column reads hit at most two lanes
+// per bank.  All dimensions here are multiples of 64 (bf16 layers have d, F
+// multiples of 128; padded column counts are multiples of 64).
+constexpr int TT = 64;
+constexpr int TROW = TT + 2;
+
+// Loads source rows src_row(i), i < 64 (negative: zeros), columns [c0, c0+64).
+__device__ __forceinline__ void load_tile(uint16_t (*tile)[TROW], const __nv_bfloat16* in,
+                                          int cols, int c0, const int* src_row) {
+  for (int idx = threadIdx.x; idx < TT * 8; idx += blockDim.x) {
+    const int i = idx >> 3, v = idx & 7;
+    const int src = src_row[i];
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (src >= 0)
+      u = *reinterpret_cast<const uint4*>(in + static_cast<size_t>(src) * cols + c0 + v * 8);
+    uint32_t* t = reinterpret_cast<uint32_t*>(&tile[i][v * 8]);
+    t[0] = u.x; t[1] = u.y; t[2] = u.z; t[3] = u.w;
+  }
+}
+
+// Writes out[(c0 + c) * ldo + base + i] = tile[i][c] for c, i < 64.
+__device__ __forceinline__ void store_tile_t(const uint16_t (*tile)[TROW], __nv_bfloat16* out,
+                                             long long ldo, long long base, int c0) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c = warp; c < TT; c += nw) {
+    const uint32_t lo = tile[2 * lane][c], hi = tile[2 * lane + 1][c];
+    reinterpret_cast<uint32_t*>(out + (c0 + c) * ldo + base)[lane] = lo | (hi << 16);
+  }
+}
+
+// out[b][c][col_off + r] = in[b][r][c] for r < rows, c < cols.
 __global__ void __launch_bounds__(256)
 transpose_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols, long long in_bstride,
                  __nv_bfloat16* __restrict__ out, int ldo, int col_off, long long out_bstride) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __nv_bfloat16 tile[32][34];
+  __shared__ __align__(16) uint16_t tile[TT][TROW];
+  __shared__ int s_src[TT];
   const int b = blockIdx.z;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  const __nv_bfloat16* src = in + b * in_bstride;
-  __nv_bfloat16* dst = out + b * out_bstride;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + tx;
-    if (r < rows && c < cols) tile[i][tx] = src[static_cast<size_t>(r) * cols + c];
-  }
+  const int r0 = blockIdx.y * TT, c0 = blockIdx.x * TT;
+  if (threadIdx.x < TT) s_src[threadIdx.x] = r0 + static_cast<int>(threadIdx.x) < rows
+                                                  ? r0 + static_cast<int>(threadIdx.x) : -1;
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + tx;
-    if (r < rows && c < cols) dst[static_cast<size_t>(c) * ldo + col_off + r] = tile[tx][i];
-  }
+  load_tile(tile, in + b * in_bstride, cols, c0, s_src);
+  __syncthreads();
+  store_tile_t(tile, out + b * out_bstride, ldo, col_off + r0, c0);
 }
 
 // Padded column offsets: poff[g + 1] = poff[g] + roundup(rows_g, 64).
@@ -126,7 +154,8 @@ __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int G, i
 // out [cols, kp]: column p of out is row src(p) of in [rows, cols], where
 // p = poff[g] + i < poff[g] + rows_g maps to row offsets[g] + i (gathered
 // through `gather` when not null), and every other p is zero.  The grid
-// covers kp x cols in 32 x 32 tiles.
+// covers kp x cols in 64 x 64 tiles; the group offsets are staged in shared
+// memory for the per-position search.
 __global__ void __launch_bounds__(256)
 gtranspose_kernel(const __nv_bfloat16* __restrict__ in, int cols,
                   const int32_t* __restrict__ offsets, int G, int rows_single,
@@ -134,38 +163,34 @@ gtranspose_kernel(const __nv_bfloat16* __restrict__ in, int cols,
                   __nv_bfloat16* __restrict__ out, int kp) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __nv_bfloat16 tile[32][34];
-  __shared__ int s_src[32];
-  const int p0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  if (ty == 0) {
-    const int p = p0 + tx;
+  __shared__ __align__(16) uint16_t tile[TT][TROW];
+  __shared__ int s_poff[258];
+  __shared__ int s_off[258];
+  __shared__ int s_src[TT];
+  const int p0 = blockIdx.x * TT, c0 = blockIdx.y * TT;
+  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+    s_poff[g] = poff[g];
+    s_off[g] = offsets ? offsets[g] : (g == 0 ? 0 : rows_single);
+  }
+  __syncthreads();
+  if (threadIdx.x < TT) {
+    const int p = p0 + static_cast<int>(threadIdx.x);
     int src = -1;
-    if (p < poff[G]) {
+    if (p < s_poff[G]) {
       int lo = 0, hi = G - 1;   // last g with poff[g] <= p
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (poff[mid] <= p) lo = mid; else hi = mid - 1;
+        if (s_poff[mid] <= p) lo = mid; else hi = mid - 1;
       }
-      const int base = offsets ? offsets[lo] : 0;
-      const int rows = offsets ? offsets[lo + 1] - offsets[lo] : rows_single;
-      const int i = p - poff[lo];
-      if (i < rows) src = gather ? gather[base + i] : base + i;
+      const int i = p - s_poff[lo];
+      if (i < s_off[lo + 1] - s_off[lo]) src = gather ? gather[s_off[lo] + i] : s_off[lo] + i;
     }
-    s_src[tx] = src;
+    s_src[threadIdx.x] = src;
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int src = s_src[i], c = c0 + tx;
-    __nv_bfloat16 v = __float2bfloat16(0.f);
-    if (src >= 0 && c < cols) v = in[static_cast<size_t>(src) * cols + c];
-    tile[i][tx] = v;
-  }
+  load_tile(tile, in, cols, c0, s_src);
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int c = c0 + i, p = p0 + tx;
-    if (c < cols && p < kp) out[static_cast<size_t>(c) * kp + p] = tile[tx][i];
-  }
+  store_tile_t(tile, out, kp, p0, c0);
 }
 
 // dGU [n, 2F]: columns [0, F) = dG, [F, 2F) = dU; G, U, dH [n, F].  fq = F / 8.
@@ -393,7 +418,8 @@ cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos
 
 cudaError_t transpose_bf16(const void* in, int batches, int rows, int cols, void* out, int ldo,
                            int col_off, cudaStream_t stream) {
-  const dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches);
+  if (rows % TT || cols % TT || ldo % 2 || col_off % 2) return cudaErrorInvalidValue;
+  const dim3 grid(cols / TT, rows / TT, batches);
   return launch_pdl(transpose_kernel, grid, dim3(256), 0, stream,
                     static_cast<const __nv_bfloat16*>(in), rows, cols,
                     static_cast<long long>(rows) * cols, static_cast<__nv_bfloat16*>(out), ldo,
@@ -409,7 +435,8 @@ cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t*
 cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,
                             int rows_single, const int32_t* poff, const int32_t* gather,
                             void* out, int kp, cudaStream_t stream) {
-  const dim3 grid((kp + 31) / 32, (cols + 31) / 32);
+  if (kp % TT || cols % TT || G > 257) return cudaErrorInvalidValue;
+  const dim3 grid(kp / TT, cols / TT);
   return launch_pdl(gtranspose_kernel, grid, dim3(256), 0, stream,
                     static_cast<const __nv_bfloat16*>(in), cols, offsets, G, rows_single, poff,
                     gather, static_cast<__nv_bfloat16*>(out), kp);
