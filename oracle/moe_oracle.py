@@ -1,4 +1,5 @@
-"""CPU oracle for the MoE FFN layer forward and the selection-bias update.
+"""CPU oracle for the MoE FFN layer: forward, backward, router statistics and
+the selection-bias updates.
 
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or run
 this module: only the tests, the smoke check and the benchmark's CPU-baseline
