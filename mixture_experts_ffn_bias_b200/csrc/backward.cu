@@ -331,58 +331,107 @@ router_dlogits_kernel(const float* __restrict__ logits, const float* __restrict_
 
 // fp32 CUDA-core GEMM, split over K: part[z][m][n] = sum_{k in slice z} A(m, k) B(k, n).
 // A(m, k) = a[m * lda + k] (A_T: a[k * lda + m]), fp32; B(k, n) = b[k * ldb + n], bf16.
-// 64 x 64 tile per block, 256 threads with 4 x 4 outputs each.
+// 128 x 128 tile per block, K in steps of 8 through shared memory, 256
+// threads with an 8 x 8 register tile each (rows ty + 16 i, columns
+// 4 tx + 64 j + q, so the shared-memory reads are float4 and conflict free).
+// N a multiple of 128, any M and K (rows past M and k past the slice read
+// as zero); kslice a multiple of 8.
+constexpr int SG_T = 128, SG_K = 8;
+
 template <bool A_T>
 __global__ void __launch_bounds__(256)
 sgemm_kernel(const float* __restrict__ a, int lda, const __nv_bfloat16* __restrict__ b, int ldb,
              int M, int N, int K, int kslice, float* __restrict__ part) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
+  __shared__ __align__(16) float As[SG_K][SG_T];
+  __shared__ __align__(16) float Bs[SG_K][SG_T];
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int m0 = blockIdx.y * SG_T, n0 = blockIdx.x * SG_T;
   const int kbeg = blockIdx.z * kslice, kend = min(K, kbeg + kslice);
-  float acc[4][4] = {};
-  for (int k0 = kbeg; k0 < kend; k0 += 16) {
-    for (int i = tid; i < 16 * 64; i += 256) {
-      const int kk = i / 64, mm = i % 64;
+  const bool vec = (lda & 3) == 0;   // 16-byte aligned rows of A
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int k0 = kbeg; k0 < kend; k0 += SG_K) {
+    // A tile: 8 x 128 floats = 256 float4
+    if (A_T) {
+      const int kk = tid >> 5, mm = (tid & 31) * 4;   // row kk, columns mm..mm+3
       const int k = k0 + kk, m = m0 + mm;
-      float v = 0.f;
-      if (k < kend && m < M) v = A_T ? a[static_cast<size_t>(k) * lda + m]
-                                     : a[static_cast<size_t>(m) * lda + k];
-      As[kk][mm] = v;
-      const int n = n0 + mm;
-      Bs[kk][mm] = (k < kend && n < N) ? __bfloat162float(b[static_cast<size_t>(k) * ldb + n])
-                                       : 0.f;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k < kend) {
+        const float* src = a + static_cast<size_t>(k) * lda + m;
+        if (vec && m + 3 < M) {
+          v = *reinterpret_cast<const float4*>(src);
+        } else {
+          v.x = m < M ? src[0] : 0.f;
+          v.y = m + 1 < M ? src[1] : 0.f;
+          v.z = m + 2 < M ? src[2] : 0.f;
+          v.w = m + 3 < M ? src[3] : 0.f;
+        }
+      }
+      *reinterpret_cast<float4*>(&As[kk][mm]) = v;
+    } else {
+      const int mm = tid >> 1, kk = (tid & 1) * 4;     // row mm, k columns kk..kk+3
+      const int m = m0 + mm, k = k0 + kk;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m < M) {
+        const float* src = a + static_cast<size_t>(m) * lda + k;
+        if (vec && k + 3 < kend) {
+          v = *reinterpret_cast<const float4*>(src);
+        } else {
+          v.x = k < kend ? src[0] : 0.f;
+          v.y = k + 1 < kend ? src[1] : 0.f;
+          v.z = k + 2 < kend ? src[2] : 0.f;
+          v.w = k + 3 < kend ? src[3] : 0.f;
+        }
+      }
+      As[kk][mm] = v.x;
+      As[kk + 1][mm] = v.y;
+      As[kk + 2][mm] = v.z;
+      As[kk + 3][mm] = v.w;
+    }
+    // B tile: 8 x 128 bf16 = 128 x 16 bytes
+    if (tid < 128) {
+      const int kk = tid >> 4, nn = (tid & 15) * 8;
+      const int k = k0 + kk, n = n0 + nn;
+      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (k < kend && n + 7 < N) {
+        const uint4 u = *reinterpret_cast<const uint4*>(b + static_cast<size_t>(k) * ldb + n);
+        unpack8(u, f);
+      }
+      *reinterpret_cast<float4*>(&Bs[kk][nn]) = make_float4(f[0], f[1], f[2], f[3]);
+      *reinterpret_cast<float4*>(&Bs[kk][nn + 4]) = make_float4(f[4], f[5], f[6], f[7]);
     }
     __syncthreads();
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float av[4], bv[4];
+    for (int kk = 0; kk < SG_K; ++kk) {
+      float av[8], bv[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        av[i] = As[kk][ty * 4 + i];
-        bv[i] = Bs[kk][tx * 4 + i];
-      }
+      for (int i = 0; i < 8; ++i) av[i] = As[kk][ty + 16 * i];
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx + 64]);
+      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
+      bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
     __syncthreads();
   }
   float* out = part + static_cast<size_t>(blockIdx.z) * M * N;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int m = m0 + ty + 16 * i;
     if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < N) out[static_cast<size_t>(m) * N + n] = acc[i][j];
-    }
+    float* row = out + static_cast<size_t>(m) * N + n0 + 4 * tx;
+    *reinterpret_cast<float4*>(row) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    *reinterpret_cast<float4*>(row + 64) =
+        make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
   }
 }
 
@@ -468,15 +517,16 @@ cudaError_t router_dlogits(const float* logits, const float* offset, const int32
 }
 
 int sgemm_slices(int K) {
-  int s = (K + 2047) / 2048;
+  int s = (K + 1023) / 1024;
   return s < 1 ? 1 : (s > 16 ? 16 : s);
 }
 
 cudaError_t sgemm_f32(bool a_t, const float* a, int lda, const void* b, int ldb, int M, int N,
                       int K, float* part, float* out, cudaStream_t stream) {
+  if (N % SG_T || ldb % 8) return cudaErrorInvalidValue;
   const int slices = sgemm_slices(K);
-  const int kslice = ((K + slices - 1) / slices + 15) / 16 * 16;
-  const dim3 grid((N + 63) / 64, (M + 63) / 64, slices);
+  const int kslice = ((K + slices - 1) / slices + SG_K - 1) / SG_K * SG_K;
+  const dim3 grid(N / SG_T, (M + SG_T - 1) / SG_T, slices);
   if (slices == 1) part = out;   // one slice: the partial sum is the result
   cudaError_t e =
       a_t ? launch_pdl(sgemm_kernel<true>, grid, dim3(256), 0, stream, a, lda,
