@@ -84,3 +84,49 @@ def test_without_allreduce_replicas_drift():
 def test_single_process_is_a_noop():
     c = torch.arange(5, dtype=torch.int32)
     assert allreduce_counts(c).tolist() == [0, 1, 2, 3, 4]
+
+
+def _grad_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from mixture_experts_ffn_bias_b200.dp import allreduce_grads
+        host = I.make_inputs(GSHAPE)
+        dout = np.random.default_rng(3).standard_normal((GSHAPE.T, GSHAPE.d_model))
+        lo, hi = rank * GSHAPE.T // world, (rank + 1) * GSHAPE.T // world
+        shard = dict(host)
+        shard["x"] = host["x"][lo:hi]
+        g = O.moe_backward(shard, GSHAPE.top_k, GSHAPE.gate, True, dout[lo:hi])
+        grads = {k: torch.from_numpy(g[k]) for k in ("dw_router", "dw1", "dw3", "dw2", "dws1",
+                                                     "dws3", "dws2")}
+        allreduce_grads(grads)
+        q.put((rank, {k: v.numpy() for k, v in grads.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+GSHAPE = I.WORKLOADS["skew"].replace(T=96, d_model=16, n_experts=8, d_ff=8, d_ff_shared=8,
+                                     top_k=2)
+
+
+def test_weight_gradients_summed_over_shards_equal_full_batch():
+    """Data-parallel backward: each rank differentiates its own token shard
+    (the oracle stands in for moe_backward, which needs a GPU); the
+    all-reduced weight gradients equal the gradients of the whole batch,
+    since every weight gradient is a sum over tokens."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_grad_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    host = I.make_inputs(GSHAPE)
+    dout = np.random.default_rng(3).standard_normal((GSHAPE.T, GSHAPE.d_model))
+    full = O.moe_backward(host, GSHAPE.top_k, GSHAPE.gate, True, dout)
+    for r in (0, 1):
+        for k, v in res[r].items():
+            np.testing.assert_allclose(v, full[k], rtol=1e-9, atol=1e-12, err_msg=k)
