@@ -7,16 +7,20 @@
 // (softmax over all experts, top-k weights renormalised).
 //
 // bf16 layers (the production path):
-//   1. logits = x . Wr^T on the tensor cores (router_logits_tc in
-//      grouped_gemm_sm100.cu): exact bf16 x bf16 products, fp32 accumulation.
-//   2. router_select_fast_kernel: one warp per token, fp32 keys and gate;
-//      a token whose k-th / (k+1)-th keys, or two adjacent keys inside its
-//      top-k, are closer than kRefineMargin is not decided here but appended
-//      to a refine list.
+//   1. logits = x . Wr^T on the tensor cores (router_sm100.cu): exact bf16 x
+//      bf16 products, fp32 accumulation in 128-wide K chunks.  With E <= 128
+//      and k <= 8 the same kernel also selects (fused select) and lists the
+//      near-tie tokens with their candidate experts; otherwise it writes the
+//      logits and
+//   2. router_select_fast_kernel decides: one warp per token, fp32 keys and
+//      gate; a token whose k-th / (k+1)-th keys, or two adjacent keys inside
+//      its top-k, are closer than kRefineMargin is not decided here but
+//      appended to a refine list.
 //   3. router_refine_kernel: for each listed token, exact logits (fp64 sums of
-//      exact products) and the selection and weights in fp64.
-//   The fp32 accumulation error of a logit is orders of magnitude below the
-//   margin, so every token's decision equals the one taken on exact logits.
+//      exact products) over its candidates (or all experts) and the
+//      selection in fp64.
+//   The fp32 accumulation error of a logit (< 5e-6) is far below the margin,
+//   so every token's decision equals the one taken on exact logits.
 // fp32 layers: logits on CUDA cores (fp32 products summed in fp32 over
 // 32-wide K chunks, chunk sums added in fp64), selection in fp64.
 //
