@@ -162,7 +162,7 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = c0 + 32 * u;
-      if (c < vecs) v[u] = __ldg(src + c);
+      if (c < vecs) v[u] = __ldcs(src + c);   // last use of x: evict first
     }
     for (int j = 0; j < k; ++j) {
       const int s = __shfl_sync(0xffffffffu, my_slot, j);

@@ -67,6 +67,25 @@ struct RCfg {
 
 constexpr int KMAX_FUSED = 8;
 
+// TMA tile load with an L2 eviction-priority policy (the router's x tiles
+// are marked evict-last, so the dispatch scatter that re-reads x right after
+// the router finds most of it in L2).
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map,
+                                                 uint64_t* bar, int32_t x, int32_t y,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+        "r"(x), "r"(y), "l"(policy)
+      : "memory");
+}
+
 struct RouterOut {
   float* logits;                 // unfused: [T, E] fp32
   const float* offset;           // fused: per-expert logit offset or null
@@ -310,11 +329,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       int stage = 0;
       uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
       bool ok = true;
+      const uint64_t keep_x = l2_evict_last_policy();
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
-          tma_load_2d(sA + stage * R_A_BYTES, &tmX, &full_bar[stage], kb * RBK, tile * RBM);
+          tma_load_2d_hint(sA + stage * R_A_BYTES, &tmX, &full_bar[stage], kb * RBK, tile * RBM,
+                           keep_x);
           tma_load_2d(sB + stage * C::B_BYTES, &tmW, &full_bar[stage], kb * RBK, 0);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
