@@ -17,8 +17,8 @@
 //   warp 1      TMEM allocation; one lane issues tcgen05.mma (M = 128,
 //               N = BN, K = 16 per instruction) into a double-buffered
 //               accumulator
-//   warps 2..5  epilogue: TMEM -> registers -> bf16 -> global, one row per
-//               thread
+//   warps 2..5  epilogue: TMEM -> registers -> bf16, staged 32 rows x 64
+//               columns per warp in shared memory, TMA tensor stores
 // Every wait is bounded; a wait that gives up aborts the CTA and sets the
 // timeout bit of the status word.
 #include <cuda.h>
@@ -46,7 +46,9 @@ struct WCfg {
   static constexpr int STAGE_BYTES = W_A_BYTES + B_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 1024;
+  // epilogue staging: per epilogue warp 32 rows x 64 bf16 (128-byte swizzle)
+  static constexpr int EPI_BYTES = 4 * 32 * 128;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
 };
 
 struct WgradArgs {
@@ -64,7 +66,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 template <int BN>
 __global__ void __launch_bounds__(W_THREADS, 1)
 wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-             const WgradArgs args) {
+             const __grid_constant__ CUtensorMap tmC, const WgradArgs args) {
   using Cfg = WCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr uint32_t IDESC = idesc_bf16_f32(WBM, BN);
@@ -73,7 +75,8 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * W_A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * Cfg::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + Cfg::EPI_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -103,6 +106,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(&s_tmem, Cfg::TMEM_COLS);
@@ -206,24 +210,43 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       if (!ok) break;
       tc_fence_after();
       const uint32_t taddr = tmem + acc * BN + (static_cast<uint32_t>(q * 32) << 16);
+      // Each warp stages its 32 rows x 64 columns in shared memory with the
+      // 128-byte swizzle and writes them with one TMA tensor store.
+      uint8_t* stage_buf = sEpi + (warp - 2) * (32 * 128);
+      const int crow0 = g * args.M + m * WBM + q * 32;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-        tmem_ld16(taddr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-        tmem_ld_wait();
-        uint32_t p[16];
+      for (int cb = 0; cb < BN / 64; ++cb) {
+        uint32_t p[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          p[i] = pack2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
+          tmem_ld16(taddr + cb * 64 + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          tmem_ld16(taddr + cb * 64 + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
+          tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          dst[c0 / 8 + c] = make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+          for (int i = 0; i < 16; ++i)
+            p[half * 16 + i] = pack2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        if (lane == 0) bulk_wait_read_all();     // the previous store has left the buffer
+        __syncwarp();
+        // row `lane`, 16-byte chunk c lands at chunk c ^ (lane % 8)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(stage_buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+              make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+        fence_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmC, stage_buf, n * BN + cb * 64, crow0);
+          bulk_commit();
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
     }
+    if (lane == 0) bulk_wait_all();            // this warp's TMA stores are complete
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -268,8 +291,8 @@ bool map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
 }
 
 template <int BN>
-cudaError_t launch_wgrad(const CUtensorMap& ta, const CUtensorMap& tb, const WgradArgs& a,
-                         cudaStream_t stream) {
+cudaError_t launch_wgrad(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                         const WgradArgs& a, cudaStream_t stream) {
   using Cfg = WCfg<BN>;
   auto kern = wgrad_kernel<BN>;
   static unsigned long long attr_done = 0;
@@ -288,7 +311,7 @@ cudaError_t launch_wgrad(const CUtensorMap& ta, const CUtensorMap& tb, const Wgr
   const long long tiles = static_cast<long long>(a.G) * (a.M / WBM) * (a.N / BN);
   if (tiles <= 0) return cudaSuccess;
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  return launch_pdl(kern, dim3(grid), dim3(W_THREADS), Cfg::SMEM_BYTES, stream, ta, tb, a);
+  return launch_pdl(kern, dim3(grid), dim3(W_THREADS), Cfg::SMEM_BYTES, stream, ta, tb, tc, a);
 }
 
 }  // namespace
@@ -298,11 +321,13 @@ cudaError_t grouped_wgrad_bf16(const void* A, const void* B, int64_t kp, const i
                                cudaStream_t stream) {
   if (M % WBM || N % 128 || G > W_MAX_GROUPS - 1 || kp % WBK) return cudaErrorInvalidValue;
   const int bn = (N % 256 == 0) ? 256 : 128;
-  CUtensorMap ta, tb;
-  if (!map_rows(&ta, A, M, kp, WBM) || !map_rows(&tb, B, N, kp, bn)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb, tc;
+  if (!map_rows(&ta, A, M, kp, WBM) || !map_rows(&tb, B, N, kp, bn) ||
+      !map_rows(&tc, C, static_cast<int64_t>(G) * M, N, 32))
+    return cudaErrorInvalidValue;
   WgradArgs a{poff, G, M, N, static_cast<__nv_bfloat16*>(C), status};
-  if (bn == 256) return launch_wgrad<256>(ta, tb, a, stream);
-  return launch_wgrad<128>(ta, tb, a, stream);
+  if (bn == 256) return launch_wgrad<256>(ta, tb, tc, a, stream);
+  return launch_wgrad<128>(ta, tb, tc, a, stream);
 }
 
 }  // namespace moe
