@@ -27,6 +27,10 @@ def test_header_symbols_exported(lib):
 def test_struct_layout():
     assert ctypes.sizeof(B.MoEConfig) == 40
     assert ctypes.sizeof(B.MoEExpertWeights) == 6 * ctypes.sizeof(ctypes.c_void_p)
+    assert ctypes.sizeof(B.MoEExpertGrads) == 6 * ctypes.sizeof(ctypes.c_void_p)
+    # moe_router_opts: int32 bias_space, int32 reserved, const float* sel_noise
+    assert ctypes.sizeof(B.MoERouterOpts) == 8 + ctypes.sizeof(ctypes.c_void_p)
+    assert B.MoERouterOpts.sel_noise.offset == 8
 
 
 @pytest.mark.parametrize("name", I.WORKLOAD_ORDER)
