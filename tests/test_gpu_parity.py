@@ -504,3 +504,23 @@ def test_bounded_wait_gives_up_and_reports_timeout():
     shape = SMALL["qwen3_small"].replace(T=64)
     host = I.make_inputs(shape)
     _check_layer(shape, host, _run(shape, host))
+
+
+@pytest.mark.parametrize("name", ["qwen3_small", "skew_small"])
+def test_token_sharded_routing_equals_whole_batch(name):
+    """Data-parallel replicas route their own token shards: every token's
+    experts and weights must equal those of the single-GPU run bit for bit
+    (the page-2 DDP-vs-single-GPU parity check).  Shards are cut at a
+    position that is not a multiple of the 128-token router tile."""
+    shape = SMALL[name]
+    host = I.make_inputs(shape)
+    full = _run(shape, host)
+    cut = shape.T // 3 + 5
+    parts = []
+    for lo, hi in ((0, cut), (cut, shape.T)):
+        h = dict(host)
+        h["x"] = host["x"][lo:hi]
+        sub = _run(shape.replace(T=hi - lo), h)
+        parts.append((_np(sub.topk_idx), _np(sub.topk_w)))
+    np.testing.assert_array_equal(np.concatenate([p[0] for p in parts]), _np(full.topk_idx))
+    np.testing.assert_array_equal(np.concatenate([p[1] for p in parts]), _np(full.topk_w))
