@@ -120,10 +120,16 @@ moe_status moe_check_config(const moe_config* cfg);
  *   per-expert constant added to the logits before the gate and the
  *   selection).
  *   out: topk_idx [T, k] int32, descending selection key, equal keys -> lower
- *   expert id; topk_w [T, k] fp32.  Logits: products of the inputs in fp32
- *   (exact for bf16 inputs), summed in fp32 over 32-wide K chunks, chunk sums
- *   added in fp64; selection keys, gate scores and the renormalisation in
- *   fp64; weights stored as fp32. */
+ *   expert id; topk_w [T, k] fp32.
+ *   bf16 layers: logits from exact bf16 products on the tensor cores, summed
+ *   in fp32 per 128-wide K chunk with the chunk sums added in fp32 (within
+ *   5e-6 of the exact logits); keys, gate and weights in fp32; every token
+ *   with two of its top-(k+1) keys closer than 1e-4 is re-decided on exact
+ *   logits (fp64 sums) over its candidate experts, so the selection equals
+ *   the one taken on exact logits.
+ *   fp32 layers: products in fp32 summed in fp32 over 32-wide K chunks, chunk
+ *   sums added in fp64; keys, gate and renormalisation in fp64.  Weights are
+ *   stored as fp32 in both cases. */
 moe_status moe_router_topk(const moe_config* cfg, const void* x, const void* w_router,
                            const float* sel_bias, const float* logit_offset,
                            int32_t* topk_idx, float* topk_w,
