@@ -11,15 +11,16 @@ second, timed on the device (CUDA events, max over ranks).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
-Prints one JSON line on rank 0.
+With --gpus N > 1 and no torchrun environment, the script re-launches itself
+under torch.distributed.run with N ranks (one per GPU, NCCL).  Prints one
+JSON line on rank 0.
 """
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
 import os
-import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -35,6 +36,8 @@ from mixture_experts_ffn_bias_b200 import inputs as I  # noqa: E402
 METRIC = "MoE-layer fwd tokens/sec and grouped-GEMM TFLOP/s (% bf16 peak) on 1 B200"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0      # B200 dense bf16, NVIDIA's nominal figure
+L2_BYTES = 126 * 1024 * 1024
 
 
 # --------------------------------------------------------------------------- #
@@ -66,26 +69,29 @@ def load_peaks() -> tuple:
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def gemm_source_hash() -> str:
-    h = hashlib.sha256()
-    for name in ("grouped_gemm_sm100.cu", "sm100.cuh"):
-        with open(os.path.join(ROOT, "mixture_experts_ffn_bias_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
+def step_bytes(s: I.MoEShape) -> int:
+    """Bytes one forward step touches at least once: weights, x, the
+    permuted rows, h, the expert outputs and out."""
+    b = 2 if s.dtype == I.DTYPE_BF16 else 4
+    R = s.T * s.top_k
+    w = (3 * s.n_experts * s.d_ff * s.d_model + s.n_experts * s.d_model
+         + 3 * s.n_shared * s.d_ff_shared * s.d_model) * b
+    act = (2 * s.T * s.d_model + 2 * R * s.d_model + R * s.d_ff
+           + s.n_shared * s.T * (s.d_ff_shared + s.d_model)) * b
+    return w + act
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the gate/up GEMM from the committed ncu summary,
-    or None when the summary is missing or was taken on other kernel source."""
-    p = os.path.join(ROOT, "profiles", f"grouped_gemm_gateup_{workload}.md")
-    if not os.path.exists(p):
-        return None
-    text = open(p).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
-    if not m or not h or h.group(1) != gemm_source_hash():
-        return None
-    return float(m.group(1))
+def host_cpu() -> dict:
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": len(os.sched_getaffinity(0)), "cpu_model": model}
 
 
 # --------------------------------------------------------------------------- #
@@ -201,7 +207,7 @@ def cpu_baseline(shape, host, seconds=15.0) -> dict:
     return {"value": tot_m / tot_t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{tot_m} of the workload's tokens in windows of {n}: router, dispatch, "
                       f"{shape.n_experts} experts{' + shared' if shape.n_shared else ''}, "
-                      f"combine, fp64 numpy ({tot_t:.1f} s)"}
+                      f"combine, fp64 numpy ({tot_t:.1f} s)", **host_cpu()}
 
 
 def run_reference(args, shape, rank: int, world: int):
@@ -227,7 +233,8 @@ def run_reference(args, shape, rank: int, world: int):
         "config": {"workload": describe(shape), "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
                          "kind": "oracle",
-                         "sample": f"{n} tokens per step (of {shape.T}), full layer in fp64"},
+                         "sample": f"{n} tokens per step (of {shape.T}), full layer in fp64",
+                         **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -284,6 +291,22 @@ def run_backward(args, shape):
         "workspace_gb": layer.bws.numel() / 1e9}), flush=True)
 
 
+def path_bytes(s: I.MoEShape) -> dict:
+    """Algorithmic bytes of the HBM-bound steps: the router reads x and the
+    router weight and writes the routing; dispatch reads x once and writes
+    the permuted rows; the combine reads the expert rows (and the shared
+    expert's output) and writes out.  Each tensor counted once per step that
+    reads or writes it."""
+    b = 2 if s.dtype == I.DTYPE_BF16 else 4
+    R = s.T * s.top_k
+    return {
+        "router": s.T * s.d_model * b + s.n_experts * s.d_model * b + s.T * s.top_k * 8,
+        "dispatch": s.T * s.d_model * b + R * s.d_model * b + R * 8,
+        "combine": R * s.d_model * b + R * 8 + s.n_shared * s.T * s.d_model * b
+        + s.T * s.d_model * b,
+    }
+
+
 def run_ours(args, shape, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -301,10 +324,14 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         layer.sel_bias = torch.zeros(shape.n_experts, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     nph = B.FORWARD_PHASES
+    # A step whose data fits a few times in L2 would be timed warm: write a
+    # buffer larger than L2 before every timed step instead.
+    flush = args.l2_flush == "on" or (args.l2_flush == "auto" and step_bytes(shape) < 4 * L2_BYTES)
+    flush_buf = torch.empty(4 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
 
-    def step(evs=None, x=None):
+    def step(evs=None, x=None, out=None):
         if evs is None:
-            layer.forward(x=x)
+            layer.forward(x=x, out=out)
         else:
             B.moe_forward_profiled(layer.cfg, layer.x if x is None else x, layer.w_router,
                                    layer.sel_bias, layer.logit_offset, layer.weights, layer.out,
@@ -317,6 +344,8 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
             dist.barrier()
 
     for _ in range(args.warmup):
+        if flush:
+            flush_buf.fill_(1)
         step()
     st, flags = layer.device_status()
     if st != B.MOE_OK:
@@ -324,6 +353,8 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nph + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    per = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)] if flush else []
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local_rank))
     barrier()
@@ -331,16 +362,23 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
     sampler.start()
     start.record(stream)
     for i in range(args.steps):
+        if flush:
+            flush_buf.fill_(i & 0xff)
+            per[i][0].record(stream)
         step()
+        if flush:
+            per[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     barrier()
-    t_ms = start.elapsed_time(end)
+    t_ms = (sum(a.elapsed_time(b) for a, b in per) if flush else start.elapsed_time(end))
     # Per-phase times come from separate steps with events between the
     # phases: an event breaks the early launch of the kernel after it, so
     # the timed steps above run without them.
     for i in range(args.steps):
+        if flush:
+            flush_buf.fill_(i & 0xff)
         step(evs[i])
     torch.cuda.synchronize(dev)
     barrier()
@@ -351,19 +389,46 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         raise SystemExit(f"device status after timing: {B.status_string(st)} ({flags})")
     refined = B.moe_router_refined_tokens(layer.ws)
 
-    # end-to-end: pinned host x in, result back, through the public layer call
+    # End to end through the public layer call: every step copies its x in
+    # from pinned host memory and its output back.  Two buffers each way and
+    # one copy stream per direction, so step i's copies overlap the compute
+    # of its neighbours (both directions of the link at once).
     e2e_steps = max(3, min(args.steps, 50))
     x_host = layer.x.to("cpu").pin_memory()
-    out_host = torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory()
-    x_dev = torch.empty_like(layer.x)
+    out_host = [torch.empty(layer.out.shape, dtype=layer.out.dtype).pin_memory() for _ in range(2)]
+    x_dev = [torch.empty_like(layer.x) for _ in range(2)]
+    out_dev = [torch.empty_like(layer.out) for _ in range(2)]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        x_dev.copy_(x_host, non_blocking=True)
-        step(x=x_dev)
-        out_host.copy_(layer.out, non_blocking=True)
+    h2d.wait_event(e0)
+    d2h.wait_event(e0)
+    with torch.cuda.stream(h2d):
+        x_dev[0].copy_(x_host, non_blocking=True)
+        h2d_done[0].record(h2d)
+    for i in range(e2e_steps):
+        b = i & 1
+        stream.wait_event(h2d_done[b])
+        if i >= 2:
+            stream.wait_event(d2h_done[b])          # out_dev[b] read out by then
+        step(x=x_dev[b], out=out_dev[b])
+        comp_done[b].record(stream)
+        if i + 1 < e2e_steps:
+            with torch.cuda.stream(h2d):
+                if i >= 1:
+                    h2d.wait_event(comp_done[1 - b])  # step i-1 done with x_dev[1-b]
+                x_dev[1 - b].copy_(x_host, non_blocking=True)
+                h2d_done[1 - b].record(h2d)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(comp_done[b])
+            out_host[b].copy_(out_dev[b], non_blocking=True)
+            d2h_done[b].record(d2h)
+    for b in range(min(2, e2e_steps)):
+        stream.wait_event(d2h_done[b])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -380,12 +445,20 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         peaks, peak_kind = load_peaks()
         sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
         burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         t_gateup = phases[2] * 1e-3
         t_gemm = (phases[2] + phases[3] + phases[4]) * 1e-3
         achieved = fl["gate_up"] / t_gateup / 1e12
         gemm_tflops = (fl["gate_up"] + fl["down"] + fl["shared"]) / t_gemm / 1e12
+        pb = path_bytes(shape)
+        t_path = (phases[0] + phases[1] + phases[5]) * 1e-3
+        path_gbs = sum(pb.values()) / t_path / 1e9
         router_launches = 2   # bf16: fused TC router + refine; fp32: logits + select
         per_step_launches = router_launches + 3 + 2 + 2 * shape.n_shared + 1 + 1
+        l2 = ("flushed: a 504 MB buffer is written before every timed step (the step's data "
+              "would fit in L2)" if flush else
+              f"not flushed: each step streams {step_bytes(shape) / 1e9:.2f} GB (weights + "
+              "activations) through the 126 MB L2")
         line = {
             "metric": METRIC, "value": shape.T * world / (ms * 1e-3), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -393,19 +466,30 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
             if shape.dtype == I.DTYPE_BF16 else "f32", "data": "synthetic",
             "config": {"workload": describe(shape), "tokens_per_gpu": shape.T,
                        "parallelism": f"dp{world} (replicated layer, counts all-reduce)",
-                       "l2": "not flushed: each step streams > 2 GB (weights + activations) "
-                             "through the 126 MB L2"},
-            "grouped_gemm": {"tflops": gemm_tflops, "frac_of_sustained": gemm_tflops / sus,
-                             "frac_of_burst": gemm_tflops / burst, "peaks": peak_kind},
+                       "l2": l2},
+            "grouped_gemm": {"tflops": gemm_tflops, "frac_of_burst": gemm_tflops / burst,
+                             "frac_of_sustained": gemm_tflops / sus,
+                             "frac_of_nominal": gemm_tflops / NOMINAL_BF16_TFLOPS,
+                             "peaks": peak_kind},
+            "routing_permute_combine": {"bytes": sum(pb.values()), "ms": t_path * 1e3,
+                                        "gbs": path_gbs, "frac_of_hbm": path_gbs / hbm,
+                                        "peaks": peak_kind},
             "phases_ms": dict(zip(["router", "dispatch", "gate_up", "down", "shared", "combine"],
                                   phases)),
             "roofline": {"kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)", "bound": "tensor",
-                         "achieved": achieved, "peak": sus, "unit": "TFLOP/s",
-                         "frac": achieved / sus, "peak_kind": f"bf16_tflops_sustained ({peak_kind})",
-                         "traffic": profiled_traffic(shape.name)},
+                         "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
+                         "frac": achieved / burst,
+                         "peak_kind": f"bf16_tflops, burst ({peak_kind})",
+                         "frac_of_sustained": achieved / sus,
+                         "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
+                         "traffic": None,
+                         "traffic_note": "not measured in this run; per-launch DRAM bytes of "
+                                         "an ncu capture are in profiles/"},
             "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": layer.x.numel() * layer.x.element_size(),
-                    "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size()},
+                    "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size(),
+                    "copies": "pinned host, one cudaMemcpyAsync per tensor per step, "
+                              "double-buffered on two copy streams"},
             "router_refined_tokens_last_step": refined,
             "gpu_launches": per_step_launches * args.steps,
             "clocks": clocks,
@@ -413,6 +497,53 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(shape, host)
         print(json.dumps(line), flush=True)
+
+
+def check_ranks(args, rank: int, world: int, local_rank: int):
+    """--check-ranks: the multi-rank plumbing alone.  Every rank sums a
+    per-expert count vector with the others (NCCL on GPUs, gloo without
+    one); rank 0 prints the world size and whether the sum came out right."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    from mixture_experts_ffn_bias_b200.dp import allreduce_counts
+
+    cuda = torch.cuda.is_available()
+    if world > 1:
+        kw = {}
+        if cuda:
+            torch.cuda.set_device(local_rank)
+            kw["device_id"] = torch.device("cuda", local_rank)
+        dist.init_process_group("nccl" if cuda else "gloo",
+                                timeout=datetime.timedelta(seconds=60), **kw)
+    dev = torch.device("cuda", local_rank) if cuda else torch.device("cpu")
+    try:
+        counts = torch.full((8,), rank + 1, dtype=torch.int32, device=dev)
+        allreduce_counts(counts)
+        ok = bool((counts == world * (world + 1) // 2).all())
+        if rank == 0:
+            print(json.dumps({"check": "ranks", "n_gpus": args.gpus, "world_size": world,
+                              "backend": dist.get_backend() if world > 1 else None,
+                              "counts_allreduce_ok": ok}), flush=True)
+        if not ok:
+            raise SystemExit("counts all-reduce gave a wrong sum")
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+def free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_command(argv, n: int, port: int) -> list:
+    """torch.distributed.run command that starts this script on n ranks."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__)] + list(argv)
 
 
 def main():
@@ -425,14 +556,30 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases for profiling; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--l2-flush", choices=["auto", "on", "off"], default="auto",
+                    help="write a buffer larger than L2 before every timed step (auto: when "
+                         "the step's data is under 4x the L2 size)")
     ap.add_argument("--mode", choices=["forward", "backward"], default="forward",
                     help="backward: time moe_backward instead (one GPU, its own JSON line)")
+    ap.add_argument("--check-ranks", action="store_true",
+                    help="start the ranks and all-reduce a count vector, time nothing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start this script again under torchrun
+        cmd = relaunch_command(sys.argv[1:], args.gpus, free_port())
+        raise SystemExit(subprocess.run(cmd).returncode)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
+    if args.check_ranks:
+        check_ranks(args, rank, world, local_rank)
+        return
     shape = I.WORKLOADS[args.workload]
     if args.tokens is not None:
         shape = shape.replace(T=args.tokens)
@@ -440,8 +587,9 @@ def main():
         run_reference(args, shape, rank, world)
         return
     if args.mode == "backward":
-        if world == 1:
-            run_backward(args, shape)
+        if world > 1:
+            raise SystemExit("--mode backward runs on one GPU")
+        run_backward(args, shape)
         return
     if world > 1:
         import datetime

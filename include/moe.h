@@ -22,9 +22,11 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library
  *     never allocates or frees device memory.  Scratch comes from the caller's
  *     workspace `ws` of `ws_bytes` bytes (>= moe_workspace_size(cfg)), 256-byte
- *     aligned.  Tensors are dense row-major.  "act" below means the activation /
- *     weight dtype cfg->dtype (fp32 or bf16); router logits, scores, weights and
- *     the selection bias are fp32 whatever the act dtype.
+ *     aligned -- except for moe_permute_noalloc, whose scratch is a fixed
+ *     array in the library's own device memory (see there).  Tensors are
+ *     dense row-major.  "act" below means the activation / weight dtype
+ *     cfg->dtype (fp32 or bf16); router logits, scores, weights and the
+ *     selection bias are fp32 whatever the act dtype.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
  *     asynchronous on it and performs no host synchronisation, except
  *     moe_device_status().
@@ -35,8 +37,9 @@
  *     never fault: the kernel records them in a status word inside `ws` and
  *     skips the offending work.  Each call clears the word when it starts;
  *     read it with moe_device_status().
- *   - No global state, no exceptions.  Calls on different streams with
- *     different workspaces may run concurrently.
+ *   - No global state (except moe_permute_noalloc's fixed scratch array and
+ *     its per-device address cache), no exceptions.  Calls on different
+ *     streams with different workspaces may run concurrently.
  *   - Limits: 1 <= top_k <= min(E, 32), E <= 256.  bf16: d_model, d_ff and
  *     d_ff_shared multiples of 128; fp32: d_model multiple of 4.  Pointers
  *     16-byte aligned.
@@ -224,7 +227,9 @@ moe_status moe_grouped_swiglu(const moe_config* cfg, const void* x_perm, const i
 /* Combine: out[t] = y_shared[t] + sum_{j<k, j ascending} topk_w[t, j] *
  * y_perm[slot_pos[t, j]], accumulated in fp32, stored once in act dtype.
  * ("moe-200m-qwen3-100b" README, "Architecture diagram": weighted sum.)
- *   y_shared may be NULL (no shared expert); slot_pos entries < 0 are skipped. */
+ *   y_shared may be NULL (no shared expert).  A slot_pos entry outside
+ *   [0, T*k) is skipped (contributes nothing); this call has no workspace, so
+ *   such entries are not reported. */
 moe_status moe_combine(const moe_config* cfg, const void* y_perm, const int32_t* slot_pos,
                        const float* topk_w, const void* y_shared, void* out, void* stream);
 
@@ -258,6 +263,42 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
                        const moe_expert_weights* w, void* out,
                        int32_t* topk_idx, float* topk_w, int32_t* counts,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* Alternatives of moe_forward's expert path, chosen per call.
+ *   gather_rows 0 (default): dispatch writes the permuted copy x_perm and the
+ *     gate/up grouped GEMM reads it with TMA tiles.
+ *   gather_rows 1 (bf16 layers only): dispatch writes no x_perm; the gate/up
+ *     GEMM gathers each tile's rows from x through the permutation (16-byte
+ *     asynchronous copies, single-CTA kernel).  Same results; measured slower
+ *     on B200, because every n-tile of a row block gathers the same rows
+ *     again.  moe_backward cannot follow a forward run this way (it reads
+ *     x_perm).
+ *   reserved: must be 0. */
+typedef struct {
+  int32_t gather_rows;
+  int32_t reserved[3];
+} moe_forward_opts;
+
+/* moe_forward with the options above (opts must not be NULL; a field
+ * outside its values is MOE_ERR_INVALID; gather_rows on an fp32 layer is
+ * MOE_ERR_UNSUPPORTED). */
+moe_status moe_forward_ex(const moe_config* cfg, const void* x, const void* w_router,
+                          const float* sel_bias, const float* logit_offset,
+                          const moe_expert_weights* w, void* out,
+                          int32_t* topk_idx, float* topk_w, int32_t* counts,
+                          const moe_forward_opts* opts, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Where moe_forward keeps the routed order inside its workspace (host
+ * arithmetic only, nothing is launched or read): offsets [E+1], slot_pos
+ * [T, k] and perm_src [T*k] int32, as moe_permute defines them, valid after a
+ * moe_forward / moe_forward_ex call on `ws` has completed on its stream and
+ * until the next call that uses `ws`.  The pointers point into ws; the
+ * caller reads them (e.g. to check the permutation, or for its own backward)
+ * and must not write them while moe_backward may still read them. */
+moe_status moe_forward_dispatch_view(const moe_config* cfg, const void* ws, size_t ws_bytes,
+                                     const int32_t** offsets, const int32_t** slot_pos,
+                                     const int32_t** perm_src);
 
 /* moe_forward with CUDA events (cudaEvent_t, created by the caller) recorded
  * on `stream` at the phase boundaries, for per-phase device timing:
@@ -339,8 +380,8 @@ const char* moe_status_string(moe_status s);
  * topk_w (as moe_forward returned them) and dout [T, d] act.  fws is the
  * workspace of that moe_forward call, unchanged since (the backward reads the
  * routed rows, their order and the saved activations from it; the forward
- * must have run with its default dispatch, which writes the permuted copy of
- * x).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
+ * must have run with its default dispatch, gather_rows 0, which writes the
+ * permuted copy of x).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
  * 256-byte aligned; its first word is a device status word read with
  * moe_device_status(bws, ...).
  * Outputs: dx [T, d] act; dw_router [E, d] fp32; g->dw1, dw3 [E, F, d],

@@ -52,6 +52,10 @@ class MoEExpertGrads(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("dw1", "dw3", "dw2", "dws1", "dws3", "dws2")]
 
 
+class MoEForwardOpts(ctypes.Structure):
+    _fields_ = [("gather_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
 class MoERouterOpts(ctypes.Structure):
     _fields_ = [("bias_space", ctypes.c_int32), ("reserved", ctypes.c_int32),
                 ("sel_noise", ctypes.c_void_p)]
@@ -76,6 +80,10 @@ _SIGNATURES = {
     "moe_forward": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_forward_profiled": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP, _VP, _SZ,
                                      _VP, ctypes.POINTER(ctypes.c_void_p)]),
+    "moe_forward_ex": (_I32, [_CFG, _VP, _VP, _VP, _VP, _WTS, _VP, _VP, _VP, _VP,
+                               ctypes.POINTER(MoEForwardOpts), _VP, _SZ, _VP]),
+    "moe_forward_dispatch_view": (_I32, [_CFG, _VP, _SZ, ctypes.POINTER(_VP),
+                                          ctypes.POINTER(_VP), ctypes.POINTER(_VP)]),
     "moe_permute_noalloc": (_I32, [_CFG, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_device_status": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_router_refined_tokens": (_I32, [_VP, _SZ, _VP, ctypes.POINTER(ctypes.c_int32)]),
@@ -255,6 +263,34 @@ def moe_forward(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, to
                            _p(topk_w), _p(counts), _p(ws),
                            _nbytes(ws) if ws is not None else 0, _s(stream))
     return _check(st, check)
+
+
+def moe_forward_ex(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, topk_idx,
+                   topk_w, counts, ws, gather_rows=0, stream=None, check=True) -> int:
+    """moe_forward with the expert-path options (gather_rows=1: the gate/up
+    GEMM gathers its rows from x instead of reading a permuted copy)."""
+    w = expert_weights(weights)
+    opts = MoEForwardOpts(int(gather_rows))
+    st = lib().moe_forward_ex(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
+                              _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),
+                              _p(topk_w), _p(counts), ctypes.byref(opts), _p(ws),
+                              _nbytes(ws) if ws is not None else 0, _s(stream))
+    return _check(st, check)
+
+
+def moe_forward_dispatch_view(cfg, ws):
+    """(offsets, slot_pos, perm_src) int32 views into the forward's workspace
+    ``ws`` (a torch uint8 tensor): the routed order the last forward wrote."""
+    import torch
+    ptrs = [ctypes.c_void_p(0) for _ in range(3)]
+    _check(lib().moe_forward_dispatch_view(ctypes.byref(cfg), _p(ws), _nbytes(ws),
+                                           *[ctypes.byref(p) for p in ptrs]), True)
+    E, T, k = cfg.n_experts, cfg.T, cfg.top_k
+    out = []
+    for p, n in zip(ptrs, (E + 1, T * k, T * k)):
+        off = int(p.value) - ws.data_ptr()
+        out.append(ws[off:off + 4 * n].view(torch.int32))
+    return out[0], out[1].view(T, k), out[2]
 
 
 def moe_backward_workspace_size(cfg: MoEConfig) -> int:

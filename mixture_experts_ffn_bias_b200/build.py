@@ -6,6 +6,7 @@ tree; nothing is installed elsewhere.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -49,11 +50,16 @@ def build(verbose: bool = False, force: bool = False) -> str:
              "-I", os.path.join(os.path.dirname(HERE), "include")]
     if verbose:
         flags += ["-Xptxas", "-v"]
-    objs = []
-    for src in sources():
+    def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, "-c", src, "-o", obj] + flags
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        r = subprocess.run([nvcc, "-c", src, "-o", obj] + flags, capture_output=True, text=True)
+        return src, obj, r
+
+    objs = []
+    workers = max(1, min(len(sources()), os.cpu_count() or 1))
+    with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+        results = list(pool.map(compile_one, sources()))
+    for src, obj, r in results:
         if verbose or r.returncode != 0:
             sys.stderr.write(r.stdout + r.stderr)
         if r.returncode != 0:

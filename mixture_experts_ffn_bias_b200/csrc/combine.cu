@@ -57,7 +57,9 @@ struct Vec<false> {
 };
 
 // KT > 0: k == KT known at compile time, so each lane issues the loads of all
-// k rows (and the shared row) before it accumulates; KT == 0: any k.
+// k rows (and the shared row) before it accumulates; KT == 0: any k.  A slot
+// outside [0, T*k) (a skipped pair, or a caller's bad slot) contributes
+// nothing.
 template <bool BF16, int KT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slot_pos,
@@ -75,6 +77,7 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slo
   if (lane < k) {
     my_slot = slot_pos[static_cast<size_t>(t) * k + lane];
     my_w = topk_w[static_cast<size_t>(t) * k + lane];
+    if (static_cast<long long>(my_slot) >= static_cast<long long>(T) * k) my_slot = -1;
   }
   if (KT > 0) {
     int sl[KT > 0 ? KT : 1];

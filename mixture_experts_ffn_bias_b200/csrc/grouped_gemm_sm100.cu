@@ -9,9 +9,14 @@
 // PR #930, "Why FSDP is enough here": compute scales with routed tokens, not
 // with the number of experts; weights stacked [E, out, in]).
 //
-// Kernel design (one CTA per SM, persistent, static round-robin over tiles):
+// Two kernels share one design (persistent, static round-robin over tiles):
+// the CTA-pair kernel below (cta_group::2, M = 256), which every grouped GEMM
+// of the layer uses, and the single-CTA kernel here, which is kept only for
+// the gate/up pass that gathers its A rows from x (no permuted copy).  Roles
+// of the single-CTA kernel:
 //   warp 0      TMA producer: A tile 128 x 64 and B tile(s) N x 64 per stage,
-//               128-byte swizzle, STAGES-deep ring of shared-memory buffers.
+//               128-byte swizzle, STAGES-deep ring of shared-memory buffers
+//               (gathered rows: 16-byte cp.async by the whole warp).
 //   warp 1      allocates TMEM (2 accumulators), one lane issues
 //               tcgen05.mma (M=128, N=BN_ACC, K=16, bf16 x bf16 -> fp32) and
 //               tcgen05.commit to release smem stages / publish accumulators.
@@ -28,7 +33,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <cstdlib>
 
 #include "kernels.h"
 #include "launch.cuh"
@@ -810,13 +814,6 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
                     c, a2);
 }
 
-// The CTA-pair kernel is the default; MOE_B200_GEMM_1SM=1 selects the
-// single-CTA kernel.
-bool use_pair() {
-  const char* v = std::getenv("MOE_B200_GEMM_1SM");
-  return !(v != nullptr && v[0] == '1');
-}
-
 }  // namespace
 
 // h[r] = silu(A[r] W1[g]^T) * (A[r] W3[g]^T), bf16 out.
@@ -832,9 +829,7 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  if (use_pair())
-    return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
-  return launch<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
+  return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
 }
 
 // Gate/up pass whose A rows are gathered from X [x_rows, K]: output row r
@@ -862,20 +857,15 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
   const int64_t c_rows = offsets ? a_rows : rows_single;
   const int bn = (N % 256 == 0) ? 256 : 128;
-  const bool pair = use_pair();
-  // the pair kernel's CTAs each load half of the B tile
-  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, pair ? bn / 2 : bn) ||
+  // each CTA of the pair loads half of the B tile
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  if (pair) {
-    if (bn == 256)
-      return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
-    return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
-  }
-  if (bn == 256) return launch<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
-  return launch<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+  if (bn == 256)
+    return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+  return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
 }
 
 

@@ -4,7 +4,6 @@
 
 #include <cstddef>
 #include <cstdint>
-#include <cstdlib>
 
 #include "../../include/moe.h"
 #include "kernels.h"
@@ -235,9 +234,15 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
                         const float* sel_bias, const float* logit_offset,
                         const moe_expert_weights* w, void* out, int32_t* topk_idx,
                         float* topk_w, int32_t* counts, void* ws, size_t ws_bytes, void* stream,
-                        void* const* events) {
+                        void* const* events, const moe_forward_opts* opts = nullptr) {
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
+  if (opts != nullptr &&
+      ((opts->gather_rows != 0 && opts->gather_rows != 1) || opts->reserved[0] != 0 ||
+       opts->reserved[1] != 0 || opts->reserved[2] != 0))
+    return MOE_ERR_INVALID;
+  const bool gather = opts != nullptr && opts->gather_rows == 1;
+  if (gather && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!counts) return MOE_ERR_INVALID;
   if (cfg->T == 0) {
     MOE_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, S(stream)));
@@ -268,12 +273,10 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   void* y_perm = at<void>(ws, L.y_perm);
   void* y_sh = cfg->n_shared ? at<void>(ws, L.y_sh) : nullptr;
   // Default: dispatch writes the permuted copy x_perm and the gate/up GEMM
-  // reads it with TMA tiles.  MOE_B200_GATHER_A=1 (bf16 only) skips the copy
+  // reads it with TMA tiles.  opts->gather_rows (bf16 only) skips the copy
   // and lets the gate/up GEMM gather its rows from x by perm_src; it moves
   // less memory but measured slower on B200 (each of an m-tile's n-tile CTAs
   // gathers the same rows again).
-  const char* ga = std::getenv("MOE_B200_GATHER_A");
-  const bool gather = cfg->dtype == MOE_BF16 && ga != nullptr && ga[0] == '1';
   int32_t* perm_src = at<int32_t>(ws, L.perm_src);
   if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
                         gather ? nullptr : x_perm, ws, s)) != MOE_OK)
@@ -646,6 +649,31 @@ moe_status moe_forward_profiled(const moe_config* cfg, const void* x, const void
   if (events == nullptr) return MOE_ERR_INVALID;
   return forward_impl(cfg, x, w_router, sel_bias, logit_offset, w, out, topk_idx, topk_w, counts,
                       ws, ws_bytes, stream, events);
+}
+
+moe_status moe_forward_ex(const moe_config* cfg, const void* x, const void* w_router,
+                          const float* sel_bias, const float* logit_offset,
+                          const moe_expert_weights* w, void* out, int32_t* topk_idx,
+                          float* topk_w, int32_t* counts, const moe_forward_opts* opts, void* ws,
+                          size_t ws_bytes, void* stream) {
+  if (opts == nullptr) return MOE_ERR_INVALID;
+  return forward_impl(cfg, x, w_router, sel_bias, logit_offset, w, out, topk_idx, topk_w, counts,
+                      ws, ws_bytes, stream, nullptr, opts);
+}
+
+moe_status moe_forward_dispatch_view(const moe_config* cfg, const void* ws, size_t ws_bytes,
+                                     const int32_t** offsets, const int32_t** slot_pos,
+                                     const int32_t** perm_src) {
+  moe_status st = check_cfg(cfg);
+  if (st != MOE_OK) return st;
+  if (!offsets || !slot_pos || !perm_src) return MOE_ERR_INVALID;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+  const Layout L = layout(*cfg);
+  void* base = const_cast<void*>(ws);
+  *offsets = at<int32_t>(base, L.offsets);
+  *slot_pos = at<int32_t>(base, L.slot_pos);
+  *perm_src = at<int32_t>(base, L.perm_src);
+  return MOE_OK;
 }
 
 moe_status moe_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags) {

@@ -55,11 +55,21 @@ class MoELayer:
 
     # ----------------------------------------------------------------- calls
     def forward(self, x: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                stream=None) -> torch.Tensor:
-        B.moe_forward(self.cfg, self.x if x is None else x, self.w_router, self.sel_bias,
-                      self.logit_offset, self.weights, self.out if out is None else out,
-                      self.topk_idx, self.topk_w, self.counts, self.ws, stream)
+                stream=None, gather_rows: bool = False) -> torch.Tensor:
+        """The layer forward (moe_forward; moe_forward_ex with gather_rows)."""
+        args = (self.cfg, self.x if x is None else x, self.w_router, self.sel_bias,
+                self.logit_offset, self.weights, self.out if out is None else out,
+                self.topk_idx, self.topk_w, self.counts, self.ws)
+        if gather_rows:
+            B.moe_forward_ex(*args, gather_rows=1, stream=stream)
+        else:
+            B.moe_forward(*args, stream=stream)
         return self.out if out is None else out
+
+    def dispatch_view(self):
+        """(offsets, slot_pos, perm_src) of the last forward, read from the
+        workspace (int32 device views; valid until the next call on it)."""
+        return B.moe_forward_dispatch_view(self.cfg, self.ws)
 
     def backward(self, dout: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
         """Gradients of <dout, out> for the last forward (bf16 layers): dx,

@@ -84,13 +84,27 @@ def check_dispatch(gpu_idx, counts, offsets, slot_pos, perm_src, r: O.Routing, E
 
 
 def check_counts_vs_oracle(counts, r: O.Routing, gpu_idx, E, excluded):
-    """Per-expert counts bit-exact after removing the excluded tokens' pairs."""
+    """The GPU's own per-expert counts, bit-exact with the oracle's after
+    removing the excluded tokens' pairs from both sides (the GPU's pairs of
+    an excluded token are its own picks, subtracted from its counts)."""
     keep = ~excluded
-    c_gpu = np.bincount(gpu_idx[keep].reshape(-1), minlength=E)
     c_ref = np.bincount(r.topk_idx[keep].reshape(-1), minlength=E)
-    np.testing.assert_array_equal(c_gpu, c_ref)
-    if not excluded.any():
-        np.testing.assert_array_equal(counts, c_ref)
+    c_gpu_excl = np.bincount(gpu_idx[excluded].reshape(-1), minlength=E)
+    np.testing.assert_array_equal(np.asarray(counts, np.int64) - c_gpu_excl, c_ref)
+    assert int(np.sum(counts)) == gpu_idx.size
+
+
+# near-tie exclusions seen by the parity tests, reported at the end of the run
+EXCLUSIONS = {}
+
+
+def record_exclusions(shape, excluded: np.ndarray, ordered: int) -> None:
+    key = f"{shape.name} T={shape.T} d={shape.d_model} E={shape.n_experts} k={shape.top_k}"
+    EXCLUSIONS[key] = (shape.T, int(excluded.sum()), int(ordered))
+
+
+def abs_err(gpu_out: np.ndarray, ref_out: np.ndarray) -> float:
+    return float(np.max(np.abs(gpu_out.astype(np.float64) - ref_out))) if ref_out.size else 0.0
 
 
 def rel_err(gpu_out: np.ndarray, ref_out: np.ndarray) -> float:

@@ -151,3 +151,41 @@ def test_backward_arguments_validated(lib):
     st = B.moe_backward(cfg32, ok, ok, None, w, ok, ok, ok, ok, ok, g, ok, ok, stream=0,
                         check=False)
     assert st == B.MOE_ERR_UNSUPPORTED
+
+
+def test_forward_options_layout_and_validation(lib):
+    assert ctypes.sizeof(B.MoEForwardOpts) == 16
+    cfg = B.config_from_shape(I.WORKLOADS["page2"])
+    ok = _FakeTensor(1 << 20)
+    ws = _FakeTensor(1 << 20, B.moe_workspace_size(cfg))
+    w = {k: ok for k in ("w1", "w3", "w2", "ws1", "ws3", "ws2")}
+    st = B.moe_forward_ex(cfg, ok, ok, None, None, w, ok, ok, ok, ok, ws, gather_rows=2,
+                          stream=0, check=False)
+    assert st == B.MOE_ERR_INVALID
+    tiny = B.config_from_shape(I.WORKLOADS["tiny"])
+    ws32 = _FakeTensor(1 << 20, B.moe_workspace_size(tiny))
+    st = B.moe_forward_ex(tiny, ok, ok, None, None, w, ok, ok, ok, ok, ws32, gather_rows=1,
+                          stream=0, check=False)
+    assert st == B.MOE_ERR_UNSUPPORTED
+
+
+def test_forward_dispatch_view_points_into_the_workspace(lib):
+    """Host arithmetic only: the three regions lie inside ws, in order, are
+    256-byte aligned and large enough for offsets [E+1], slot_pos [T, k] and
+    perm_src [T*k]."""
+    shape = I.WORKLOADS["qwen3_30b"]
+    cfg = B.config_from_shape(shape)
+    n = B.moe_workspace_size(cfg)
+    base = 1 << 30
+    ptrs = [ctypes.c_void_p(0) for _ in range(3)]
+    st = lib.moe_forward_dispatch_view(ctypes.byref(cfg), base, n, *[ctypes.byref(p) for p in ptrs])
+    assert st == B.MOE_OK
+    offs, slot, src = (p.value - base for p in ptrs)
+    E, R = shape.n_experts, shape.T * shape.top_k
+    assert 0 < offs and offs + 4 * (E + 1) <= slot and slot + 4 * R <= src
+    assert src + 4 * R <= n
+    assert offs % 256 == slot % 256 == src % 256 == 0
+    assert lib.moe_forward_dispatch_view(ctypes.byref(cfg), base, n - 1,
+                                         *[ctypes.byref(p) for p in ptrs]) == B.MOE_ERR_WORKSPACE
+    assert lib.moe_forward_dispatch_view(ctypes.byref(cfg), base + 8, n,
+                                         *[ctypes.byref(p) for p in ptrs]) == B.MOE_ERR_INVALID

@@ -130,3 +130,31 @@ def test_weight_gradients_summed_over_shards_equal_full_batch():
     for r in (0, 1):
         for k, v in res[r].items():
             np.testing.assert_allclose(v, full[k], rtol=1e-9, atol=1e-12, err_msg=k)
+
+
+def test_bench_launches_one_rank_per_gpu():
+    """bench.py --gpus 2 without a torchrun environment starts itself again on
+    two ranks; --check-ranks makes them all-reduce a count vector (gloo here)
+    and rank 0 reports the world size it saw."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--check-ranks"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(s) for s in r.stdout.splitlines() if s.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["world_size"] == 2 and lines[0]["counts_allreduce_ok"]
+
+
+def test_bench_refuses_a_world_size_that_differs_from_gpus():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--check-ranks"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode != 0 and "launcher started 1 ranks" in r.stderr

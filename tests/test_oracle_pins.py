@@ -625,3 +625,22 @@ def test_backward_top1_renormalised_has_no_router_gradient():
     dout = rng.standard_normal((8, 6))
     g = O.moe_backward(inp, 1, O.GATE_SOFTMAX, True, dout)
     assert np.max(np.abs(g["dw_router"])) < 1e-7
+
+
+def test_near_tie_table_is_the_oracles():
+    """tests/golden/near_ties.json (written by make_near_ties.py from the
+    oracle alone): its rule, its workloads, and the tiny workload's entry
+    recomputed here (the full-size entries are recomputed by the GPU parity
+    tests, which route those workloads with the oracle anyway)."""
+    import json
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "near_ties.json")
+    with open(path) as f:
+        table = json.load(f)
+    assert "1e-6" in table["rule"]
+    assert set(table["workloads"]) == set(I.WORKLOAD_ORDER)
+    for name, e in table["workloads"].items():
+        assert e["T"] == I.WORKLOADS[name].T and e["excluded"] == len(e["tokens"])
+    shape = I.WORKLOADS["tiny"]
+    host = I.make_inputs(shape)
+    r = O.router(host["x"], host["w_router"], shape.top_k, shape.gate, True)
+    assert (r.edge_gap < 1e-6).nonzero()[0].tolist() == table["workloads"]["tiny"]["tokens"]
