@@ -15,6 +15,9 @@
 //            exclusive scan over experts (offsets).
 //   scatter  one warp per token: final row = base + rank, x row read once
 //            and written to its k rows with 16-byte vector accesses.
+// The forward's fused router (router_topk_pair) produces the ranks and block
+// counts itself, over blocks of its own size, and usually the scan as well;
+// the scatter then takes that block size.
 // Pairs with an expert id outside [0, E), or repeating an expert the token
 // already chose, are skipped (row -1) and flagged in the status word.
 #include <cuda_runtime.h>
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ topk_idx,
                         const int32_t* __restrict__ bases, int32_t* __restrict__ slot_pos,
                         int32_t* __restrict__ perm_src, uint4* __restrict__ x_perm, int T,
-                        int vecs, int k, int E) {
+                        int vecs, int k, int E, int blk_tokens) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -151,7 +154,7 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
     const int r = slot_pos[p];
     if (r >= 0) {
       const int e = topk_idx[p];
-      my_slot = bases[static_cast<size_t>(t / kRankBlock) * E + e] + r;
+      my_slot = bases[static_cast<size_t>(t / blk_tokens) * E + e] + r;
       perm_src[my_slot] = t;
     }
     slot_pos[p] = my_slot;
@@ -181,12 +184,12 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
 __global__ void __launch_bounds__(256)
 dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ bases,
                           int32_t* __restrict__ slot_pos, int32_t* __restrict__ perm_src, int T,
-                          int k, int E) {
+                          int k, int E, int blk_tokens) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
-  const int32_t* b = bases + static_cast<size_t>(t / kRankBlock) * E;
+  const int32_t* b = bases + static_cast<size_t>(t / blk_tokens) * E;
   for (int j = 0; j < k; ++j) {
     const size_t p = static_cast<size_t>(t) * k + j;
     const int r = slot_pos[p];
@@ -203,9 +206,9 @@ dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* _
 
 cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
                                int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
-                               cudaStream_t stream) {
+                               int blk_tokens, cudaStream_t stream) {
   return launch_pdl(dispatch_positions_kernel, dim3((T + 255) / 256), dim3(256), 0, stream,
-                    topk_idx, blk_bases, slot_pos, perm_src, T, k, E);
+                    topk_idx, blk_bases, slot_pos, perm_src, T, k, E, blk_tokens);
 }
 
 cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,
@@ -222,12 +225,13 @@ cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
 
 cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              const int32_t* blk_bases, int32_t* slot_pos, int32_t* perm_src,
-                             void* x_perm, int T, int d, int k, int E, cudaStream_t stream) {
+                             void* x_perm, int T, int d, int k, int E, int blk_tokens,
+                             cudaStream_t stream) {
   const int vecs = d * (bf16 ? 2 : 4) / 16;
   const int warps = 8;
   return launch_pdl(dispatch_scatter_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
                     stream, static_cast<const uint4*>(x), topk_idx, blk_bases, slot_pos, perm_src,
-                    static_cast<uint4*>(x_perm), T, vecs, k, E);
+                    static_cast<uint4*>(x_perm), T, vecs, k, E, blk_tokens);
 }
 
 }  // namespace moe

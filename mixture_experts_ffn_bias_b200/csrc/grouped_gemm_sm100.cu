@@ -458,14 +458,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 // barrier.  No load uses cluster multicast.
 constexpr int BM2 = 256;
 
+// BN_ACC accumulator columns per tile (gate and up columns together for
+// SwiGLU).  Up to 256 the TMEM accumulator is double buffered, so the
+// epilogue of a tile overlaps the MMAs of the next.  BN_ACC = 512 fills TMEM
+// with one accumulator of two N = 256 halves (two MMAs per K step): each
+// staged byte of A then feeds twice the MMA work, which matters because the
+// tiles are streamed from L2; the producer keeps prefetching the next
+// tile's stages while the epilogue drains the accumulator.
 template <int BN_ACC>
 struct PairCfg {
+  static constexpr int NSUB = BN_ACC > 256 ? BN_ACC / 256 : 1;   // MMAs per K step
+  static constexpr int N_MMA = BN_ACC / NSUB;                     // N of one MMA
+  static constexpr int NACC = BN_ACC > 256 ? 1 : 2;               // TMEM buffers
   static constexpr int B_HALF_BYTES = (BN_ACC / 2) * BK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_HALF_BYTES;
   static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
-  static constexpr int TMEM_COLS = 2 * BN_ACC;
+  static constexpr int TMEM_COLS = NACC * BN_ACC;
   static constexpr int EPI_BYTES = 4 * 32 * 128;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024 + 1024;
+  static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
 };
 
 template <int BN_ACC, int MODE>
@@ -478,7 +489,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr int STAGES = Cfg::STAGES;
   constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
   constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM2, BN_ACC);
+  constexpr int NSUB = Cfg::NSUB;
+  constexpr int NACC = Cfg::NACC;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM2, Cfg::N_MMA);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -584,8 +597,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t phase = 0;
       bool ok = true, issued_any = false;
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = it % NACC;
+        const uint32_t acc_phase = (it / NACC) & 1;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN_ACC;
@@ -596,8 +609,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t b_addr = smem_u32(smemB + stage * Cfg::B_HALF_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc_mma_f16_pair(d_tmem, smem_desc_sw128(a_addr + kk * 32),
-                            smem_desc_sw128(b_addr + kk * 32), IDESC, (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int sub = 0; sub < NSUB; ++sub)   // sub-tile: B rows [128 sub, 128 sub + 128)
+              tc_mma_f16_pair(d_tmem + sub * Cfg::N_MMA, smem_desc_sw128(a_addr + kk * 32),
+                              smem_desc_sw128(b_addr + sub * (Cfg::N_MMA / 2) * 128 + kk * 32),
+                              IDESC, (kb | kk) != 0 ? 1u : 0u);
           issued_any = true;
           tc_commit_pair(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -618,8 +634,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     const int row = q * 32 + lane;
     int it = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = it % NACC;
+      const uint32_t acc_phase = (it / NACC) & 1;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -632,22 +648,38 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool warp_full = (r0 + q * 32 + 32) <= rows_g;
       const int warp_row0 = s_off[g] + r0 + q * 32;
       uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
-      const size_t crow_off = static_cast<size_t>(s_off[g] + r0 + row) * args.ldc +
-                              static_cast<size_t>(n) * BN_OUT;
+      const size_t crow_off = static_cast<size_t>(s_off[g] + r0 + row) * args.ldc;
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int cb = 0; cb < BN_OUT / 64; ++cb) {
+        // accumulator column of this 64-column chunk and its output column:
+        // sub-tile `sub` holds N_MMA columns, its first half from rank 0's B
+        // rows and its second half from rank 1's (SwiGLU: gate, then up)
+        int acol, ocol;
+        if (SWIGLU) {
+          const int sub = (cb * 64) / (Cfg::N_MMA / 2);
+          const int c = (cb * 64) % (Cfg::N_MMA / 2);
+          acol = sub * Cfg::N_MMA + c;
+          ocol = n * BN_OUT + cb * 64;
+        } else {
+          const int sub = (cb * 64) / Cfg::N_MMA;
+          const int jj = (cb * 64) % Cfg::N_MMA;
+          acol = cb * 64;
+          ocol = n * BN_ACC + (jj / (Cfg::N_MMA / 2)) * (BN_ACC / 2) + sub * (Cfg::N_MMA / 2) +
+                 jj % (Cfg::N_MMA / 2);
+        }
         uint32_t packed[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const int c0 = cb * 64 + half * 32;
+          const int c0 = acol + half * 32;
           uint32_t v[32];
           if (SWIGLU) {
             uint32_t u[32];
+            constexpr int UP = Cfg::N_MMA / 2;   // up columns follow the gate columns
             tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
             tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-            tmem_ld16(t_addr + BN_OUT + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
-            tmem_ld16(t_addr + BN_OUT + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
+            tmem_ld16(t_addr + UP + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
+            tmem_ld16(t_addr + UP + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -677,12 +709,12 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmC, stage_buf, n * BN_OUT + cb * 64, warp_row0);
+            tma_store_2d(&tmC, stage_buf, ocol, warp_row0);
             bulk_commit();
           }
         } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
-                                                cb * 64);
+                                                ocol);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
@@ -824,11 +856,15 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
   CUtensorMap ta, tb0, tb1, tc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
   const int64_t c_rows = offsets ? a_rows : rows_single;
-  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
-      !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, c_rows, F, 32))
+  // 256 output columns per tile (512 accumulator columns) when F allows
+  const bool wide = F % 256 == 0;
+  const int bh = wide ? 256 : 128;   // B rows each CTA of the pair loads
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, bh) ||
+      !make_map(&tb1, W3, b_rows, K, bh) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (wide) return launch_pair<512, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
   return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
 }
 
@@ -856,13 +892,15 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   CUtensorMap ta, tb, tc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
   const int64_t c_rows = offsets ? a_rows : rows_single;
-  const int bn = (N % 256 == 0) ? 256 : 128;
+  const int bn = (N % 512 == 0) ? 512 : (N % 256 == 0) ? 256 : 128;
   // each CTA of the pair loads half of the B tile
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (bn == 512)
+    return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
   if (bn == 256)
     return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
   return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);

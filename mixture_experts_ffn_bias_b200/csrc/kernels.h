@@ -48,6 +48,21 @@ cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, in
                            cudaStream_t stream);
 cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
                              float* logits, uint32_t* status, cudaStream_t stream);
+// Fused router on CTA pairs (E <= 128, k <= 8): logits, selection, exact
+// re-decision of near ties inside the kernel, and the dispatch's per-block
+// ranks (rank_out [T, k]) and counts (blk [router_pair_blocks(T), E], blocks
+// of router_pair_block_tokens(T) tokens).  When *scan_fused comes back true
+// the last CTA has also turned blk into block bases and written counts and
+// offsets; otherwise dispatch_scan must follow.  done: a zeroed counter.
+constexpr int kRouterPairs = 74;   // CTA pairs the token tiles are sized for
+int router_pair_block_tokens(int T);
+int router_pair_blocks(int T);
+cudaError_t router_topk_pair(const void* x, int T, const void* w_router, int E, int K,
+                             const float* logit_offset, const float* sel_bias, int k, int gate,
+                             int renorm, int32_t* topk_idx, float* topk_w, int32_t* rank_out,
+                             int32_t* blk, int32_t* counts, int32_t* offsets,
+                             int32_t* refine_count, uint32_t* status, uint32_t* done,
+                             bool* scan_fused, cudaStream_t stream);
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
                                const KeyOpts& ko, int32_t* topk_idx, float* topk_w,
@@ -78,13 +93,15 @@ cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t*
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream);
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream);
-// slot_pos (in: rank, out: row) and perm_src only, no row copy.
+// slot_pos (in: rank inside its block of blk_tokens tokens, out: row) and
+// perm_src only, no row copy.
 cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
                                int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
-                               cudaStream_t stream);
+                               int blk_tokens, cudaStream_t stream);
 cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              const int32_t* blk_bases, int32_t* slot_pos, int32_t* perm_src,
-                             void* x_perm, int T, int d, int k, int E, cudaStream_t stream);
+                             void* x_perm, int T, int d, int k, int E, int blk_tokens,
+                             cudaStream_t stream);
 
 // Experts --------------------------------------------------------------------
 cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,

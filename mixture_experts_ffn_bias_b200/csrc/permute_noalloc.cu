@@ -86,7 +86,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                          s) != cudaSuccess ||
       moe::dispatch_scan(blk, nblk, cfg->n_experts, counts, offsets, s) != cudaSuccess ||
       moe::dispatch_scatter(cfg->dtype == MOE_BF16, x, topk_idx, blk, slot_pos, perm_src, x_perm,
-                            cfg->T, cfg->d_model, cfg->top_k, cfg->n_experts, s) != cudaSuccess)
+                            cfg->T, cfg->d_model, cfg->top_k, cfg->n_experts, moe::kRankBlock,
+                            s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }
