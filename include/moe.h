@@ -268,11 +268,8 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  *   gather_rows 0 (default): dispatch writes the permuted copy x_perm and the
  *     gate/up grouped GEMM reads it with TMA tiles.
  *   gather_rows 1 (bf16 layers only): dispatch writes no x_perm; the gate/up
- *     GEMM gathers each tile's rows from x through the permutation (16-byte
- *     asynchronous copies, single-CTA kernel).  Same results; measured slower
- *     on B200, because every n-tile of a row block gathers the same rows
- *     again.  moe_backward cannot follow a forward run this way (it reads
- *     x_perm).
+ *     GEMM gathers each tile's rows from x through the permutation (TMA
+ *     tile::gather4 loads, four rows per load).  Same results.
  *   reserved: must be 0. */
 typedef struct {
   int32_t gather_rows;
@@ -303,9 +300,10 @@ moe_status moe_forward_dispatch_view(const moe_config* cfg, const void* ws, size
 /* moe_forward with CUDA events (cudaEvent_t, created by the caller) recorded
  * on `stream` at the phase boundaries, for per-phase device timing:
  *   events[0] start            events[1] after the router
- *   events[2] after dispatch   events[3] after the routed gate/up GEMM
- *   events[4] after the routed down GEMM
- *   events[5] after the shared expert (== events[4] time when none)
+ *   events[2] after dispatch   events[3] after the gate/up GEMM
+ *   events[4] after the down GEMM
+ *   events[5] right after events[4] (the shared expert runs as one more
+ *             group inside the two GEMM launches of bf16 layers)
  *   events[6] after the combine (end)
  * Same launches and results as moe_forward. */
 #define MOE_FORWARD_PHASES 6
@@ -378,10 +376,9 @@ const char* moe_status_string(moe_status s);
  *             dw_router = dlogits^T x and dx += dlogits w_router (fp32).
  * Inputs: the forward's x, w_router, logit_offset, weights, topk_idx,
  * topk_w (as moe_forward returned them) and dout [T, d] act.  fws is the
- * workspace of that moe_forward call, unchanged since (the backward reads the
- * routed rows, their order and the saved activations from it; the forward
- * must have run with its default dispatch, gather_rows 0, which writes the
- * permuted copy of x).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
+ * workspace of that moe_forward (or moe_forward_ex) call, unchanged since
+ * (the backward reads the routed order and the saved activations h and y
+ * from it; x's rows are gathered again by the permutation).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
  * 256-byte aligned; its first word is a device status word read with
  * moe_device_status(bws, ...).
  * Outputs: dx [T, d] act; dw_router [E, d] fp32; g->dw1, dw3 [E, F, d],

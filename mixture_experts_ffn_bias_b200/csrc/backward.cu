@@ -4,7 +4,6 @@
 // GEMM of grouped_gemm_wgrad_sm100.cu for the weight gradients); this file
 // holds what feeds and finishes them:
 //   bwd_dy_kernel       dw[t, j] = <dout[t], y_perm[slot]>, dY[slot] = w[t, j] dout[t]
-//   transpose_kernel    batched bf16 transpose (weights, once per backward)
 //   gtranspose_kernel   rows of each group -> padded columns (the K-grouped
 //                       operands), zeros in the padding
 //   pad_offsets_kernel  padded column offsets of the groups
@@ -118,23 +117,6 @@ __device__ __forceinline__ void store_tile_t(const uint16_t (*tile)[TROW], __nv_
 }
 
 // out[b][c][col_off + r] = in[b][r][c] for r < rows, c < cols.
-__global__ void __launch_bounds__(256)
-transpose_kernel(const __nv_bfloat16* __restrict__ in, int rows, int cols, long long in_bstride,
-                 __nv_bfloat16* __restrict__ out, int ldo, int col_off, long long out_bstride) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ __align__(16) uint16_t tile[TT][TROW];
-  __shared__ int s_src[TT];
-  const int b = blockIdx.z;
-  const int r0 = blockIdx.y * TT, c0 = blockIdx.x * TT;
-  if (threadIdx.x < TT) s_src[threadIdx.x] = r0 + static_cast<int>(threadIdx.x) < rows
-                                                  ? r0 + static_cast<int>(threadIdx.x) : -1;
-  __syncthreads();
-  load_tile(tile, in + b * in_bstride, cols, c0, s_src);
-  __syncthreads();
-  store_tile_t(tile, out + b * out_bstride, ldo, col_off + r0, c0);
-}
-
 // Padded column offsets: poff[g + 1] = poff[g] + roundup(rows_g, 64).
 // offsets null: one group of rows_single rows.
 __global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int G, int rows_single,
@@ -463,16 +445,6 @@ cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos
   return launch_pdl(bwd_dy_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0, stream,
                     static_cast<const uint4*>(dout), static_cast<const uint4*>(y_perm), slot_pos,
                     topk_w, static_cast<uint4*>(dy), dw, T, d / 8, k);
-}
-
-cudaError_t transpose_bf16(const void* in, int batches, int rows, int cols, void* out, int ldo,
-                           int col_off, cudaStream_t stream) {
-  if (rows % TT || cols % TT || ldo % 2 || col_off % 2) return cudaErrorInvalidValue;
-  const dim3 grid(cols / TT, rows / TT, batches);
-  return launch_pdl(transpose_kernel, grid, dim3(256), 0, stream,
-                    static_cast<const __nv_bfloat16*>(in), rows, cols,
-                    static_cast<long long>(rows) * cols, static_cast<__nv_bfloat16*>(out), ldo,
-                    col_off, static_cast<long long>(cols) * ldo);
 }
 
 cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,

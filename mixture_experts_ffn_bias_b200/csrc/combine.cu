@@ -79,7 +79,7 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slo
     my_w = topk_w[static_cast<size_t>(t) * k + lane];
     if (static_cast<long long>(my_slot) >= static_cast<long long>(T) * k) my_slot = -1;
   }
-  if (KT > 0) {
+  if constexpr (KT > 0) {
     int sl[KT > 0 ? KT : 1];
     float wj[KT > 0 ? KT : 1];
 #pragma unroll
@@ -111,26 +111,26 @@ combine_kernel(const uint4* __restrict__ y_perm, const int32_t* __restrict__ slo
       }
       out[static_cast<size_t>(t) * vecs + c] = V::store(acc);
     }
-    return;
-  }
-  for (int c = lane; c < vecs; c += 32) {
-    float acc[V::N];
-    if (y_shared) {
-      V::load(__ldg(y_shared + static_cast<size_t>(t) * vecs + c), acc);
-    } else {
+  } else {
+    for (int c = lane; c < vecs; c += 32) {
+      float acc[V::N];
+      if (y_shared) {
+        V::load(__ldg(y_shared + static_cast<size_t>(t) * vecs + c), acc);
+      } else {
 #pragma unroll
-      for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
-    }
-    for (int j = 0; j < k; ++j) {
-      const int s = __shfl_sync(0xffffffffu, my_slot, j);
-      const float w = __shfl_sync(0xffffffffu, my_w, j);
-      if (s < 0) continue;
-      float f[V::N];
-      V::load(__ldg(y_perm + static_cast<size_t>(s) * vecs + c), f);
+        for (int i = 0; i < V::N; ++i) acc[i] = 0.f;
+      }
+      for (int j = 0; j < k; ++j) {
+        const int s = __shfl_sync(0xffffffffu, my_slot, j);
+        const float w = __shfl_sync(0xffffffffu, my_w, j);
+        if (s < 0) continue;
+        float f[V::N];
+        V::load(__ldg(y_perm + static_cast<size_t>(s) * vecs + c), f);
 #pragma unroll
-      for (int i = 0; i < V::N; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+        for (int i = 0; i < V::N; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      }
+      out[static_cast<size_t>(t) * vecs + c] = V::store(acc);
     }
-    out[static_cast<size_t>(t) * vecs + c] = V::store(acc);
   }
 }
 

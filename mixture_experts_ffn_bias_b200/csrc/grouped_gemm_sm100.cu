@@ -9,25 +9,24 @@
 // PR #930, "Why FSDP is enough here": compute scales with routed tokens, not
 // with the number of experts; weights stacked [E, out, in]).
 //
-// Two kernels share one design (persistent, static round-robin over tiles):
-// the CTA-pair kernel below (cta_group::2, M = 256), which every grouped GEMM
-// of the layer uses, and the single-CTA kernel here, which is kept only for
-// the gate/up pass that gathers its A rows from x (no permuted copy).  Roles
-// of the single-CTA kernel:
-//   warp 0      TMA producer: A tile 128 x 64 and B tile(s) N x 64 per stage,
-//               128-byte swizzle, STAGES-deep ring of shared-memory buffers
-//               (gathered rows: 16-byte cp.async by the whole warp).
-//   warp 1      allocates TMEM (2 accumulators), one lane issues
-//               tcgen05.mma (M=128, N=BN_ACC, K=16, bf16 x bf16 -> fp32) and
-//               tcgen05.commit to release smem stages / publish accumulators.
-//   warps 2-5   epilogue: tcgen05.ld the accumulator (thread = row), apply
-//               SwiGLU (gate and up columns of the same output column sit in
-//               the same accumulator: B rows 0-127 come from W1, 128-255 from
-//               W3), round to bf16 and store the row segment.
-// The TMEM accumulator is double buffered so the epilogue of tile i overlaps
-// the MMAs of tile i+1.  Tile order is (group, m-tile, n-tile) with n fastest,
-// so CTAs running at the same time share the A tile and one expert's weights
-// in L2.
+// One persistent kernel on CTA pairs (cluster of two, tcgen05.mma.cta_group::2,
+// M = 256 rows per tile, static round-robin over tiles):
+//   warp 0      TMA producer: per stage this CTA's 128 A rows x 64 K and its
+//               half of the B tile, 128-byte swizzle, a ring of stages; A rows
+//               may instead be gathered from x by the permutation
+//               (tile::gather4, four rows per lane)
+//   warp 1      allocates TMEM; on rank 0 one lane issues the MMAs for the
+//               pair (bf16 x bf16 -> fp32) and commits stages / accumulators
+//               to both CTAs
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (thread = row), SwiGLU
+//               in fp32 (gate and up columns of an output column sit in the
+//               same accumulator row: rank 0 holds the W1 rows of the B tile,
+//               rank 1 the W3 rows), bf16 rounding, TMA tensor stores
+// The TMEM accumulator is double buffered (up to 256 columns) so the
+// epilogue of tile i overlaps the MMAs of tile i+1.  Tile order is (group,
+// m-tile, n-tile) with n fastest, so CTAs running at the same time share the A
+// tile and one expert's weights in L2.  The shared expert can run as one more
+// group after the routed ones, with tensors of its own.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,21 +46,14 @@ constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;          // 6 warps
 constexpr int MAX_GROUPS = 257;
 
-template <int BN_ACC>
-struct GemmCfg {
-  static constexpr int B_STAGE_BYTES = BN_ACC * BK * 2;
-  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-  static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
-  static constexpr int TMEM_COLS = 2 * BN_ACC;      // double-buffered accumulator
-  // epilogue staging: per epilogue warp 32 rows x 64 bf16 (128-byte swizzle)
-  static constexpr int EPI_BYTES = 4 * 32 * 128;
-  static constexpr int SMEM_BYTES =
-      STAGES * STAGE_BYTES + EPI_BYTES + 1024 /*align*/ + 1024 /*bars*/;
-};
 
-// Epilogue modes.
+// Epilogue / operand modes.
 constexpr int MODE_PLAIN_BF16 = 0;    // C = A B^T, rounded to bf16
 constexpr int MODE_SWIGLU_BF16 = 1;   // C = silu(A B0^T) * (A B1^T), rounded to bf16
+// C = A B with B stored [K, N] per group (MN-major, N contiguous), rounded to
+// bf16; the K rows of a group come from B0 (the first kb_split k-blocks) and
+// then from B1, so [W1; W3] needs no concatenated copy.
+constexpr int MODE_PLAIN_BMN = 2;
 
 struct GemmArgs {
   const int32_t* offsets;  // [G+1] device, or nullptr: one group [0, rows_single)
@@ -75,6 +67,28 @@ struct GemmArgs {
   const int32_t* gather_rows;  // GATHER: A row of output row r is gather_src[gather_rows[r]]
   const void* gather_src;      // GATHER: [rows, K] bf16
   int m_fastest;               // tile order inside a group: 1 = m-tiles fastest
+  int kb_split;                // PLAIN_BMN: k-blocks read from B0, the rest from B1
+  int b0_rows;                 // PLAIN_BMN: K rows of a group in B0
+  int b1_rows;                 // PLAIN_BMN: K rows of a group in B1
+  // CTA-pair kernel: one extra group after the routed ones, with tensors of
+  // its own (the shared expert over all tokens), or x_rows = 0
+  int x_rows;                  // its rows (A rows from 0)
+  int x_n;                     // its output columns (B rows per half as above)
+  int x_K;                     // its K
+  void* x_C;                   // its output
+  int x_ldc;
+  int gather_limit;            // GATHER: entries of gather_rows
+  int gather_src_rows;         // GATHER: rows of gather_src
+};
+
+// Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
+// one of the extra group's (tiles after all routed ones, n fastest).
+struct PairTile {
+  bool x;        // the extra group
+  int g, m, n;
+  int row0;      // first row of the group in its A and C tensors
+  int rows;      // rows of the group
+  int kblocks;
 };
 
 __device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
@@ -153,299 +167,6 @@ __device__ __forceinline__ int find_group(const int* s_prefix, int G, int tile) 
   return lo;
 }
 
-template <int BN_ACC, int MODE, bool GATHER>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                    const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1,
-                    const __grid_constant__ CUtensorMap tmC,
-                    const GemmArgs args) {
-  using Cfg = GemmCfg<BN_ACC>;
-  constexpr int STAGES = Cfg::STAGES;
-  constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
-  constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN_ACC);
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* smemA = smem;
-  uint8_t* smemB = smem + STAGES * A_STAGE_BYTES;
-  uint8_t* smemEpi = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smemEpi + Cfg::EPI_BYTES);
-  uint64_t* full_bar = bars;
-  uint64_t* empty_bar = bars + STAGES;
-  uint64_t* tfull_bar = bars + 2 * STAGES;
-  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
-  uint64_t* drain_bar = bars + 2 * STAGES + 4;
-
-  __shared__ int s_off[MAX_GROUPS + 1];
-  __shared__ int s_prefix[MAX_GROUPS + 1];
-  __shared__ uint32_t s_tmem_base;
-  __shared__ int s_abort;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int n_tiles = args.n_per_group / BN_OUT;
-  const int G = args.offsets == nullptr ? 1 : args.num_groups;
-
-  if (threadIdx.x == 0) {
-    s_abort = 0;
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 4);
-    }
-    mbar_init(drain_bar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    if (!GATHER) tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB0);
-    if (SWIGLU) tma_prefetch_desc(&tmB1);
-    tma_prefetch_desc(&tmC);
-  }
-  if (warp == 1) {
-    tmem_alloc(&s_tmem_base, Cfg::TMEM_COLS);
-    tmem_relinquish();
-  }
-  pdl_wait();   // everything above touches no global memory
-  if (warp == 2) build_tile_prefix(args, n_tiles, s_off, s_prefix);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
-  const uint32_t tmem_base = s_tmem_base;
-  const int total_tiles = s_prefix[G];
-  volatile int* abort_flag = &s_abort;
-  const int kblocks = args.K / BK;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Lane 0 drives the ring.  With GATHER the whole warp fills the A tile
-    // with 16-byte cp.async: warp instruction i copies rows 4i..4i+3 (lane
-    // / 8 picks the row, lane % 8 the 16-byte chunk), written at the
-    // 128-byte-swizzled position the MMA descriptor expects; each lane's
-    // copies are tracked on the stage barrier by cp.async.mbarrier.arrive.
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t issued_mask = 0;     // stages with a load in flight at exit
-    uint32_t issued_phase = 0;    // parity of that load's phase
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-      const int g = find_group(s_prefix, G, tile);
-      int m, n;
-      tile_mn(tile - s_prefix[g], s_off[g + 1] - s_off[g], n_tiles, args.m_fastest, m, n);
-      const int arow = s_off[g] + m * BM;
-      const int brow = g * args.n_per_group + n * BN_OUT;
-      int tok[GATHER ? 32 : 1];
-      if (GATHER) {
-        // rows past the group's end read a valid row (the first of the
-        // tile); the epilogue never stores them
-        const int rows_g = s_off[g + 1] - s_off[g];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = 4 * i + (lane >> 3);
-          tok[i] = args.gather_rows[m * BM + r < rows_g ? arow + r : arow];
-        }
-      }
-      for (int kb = 0; kb < kblocks; ++kb) {
-        bool w_ok = true;
-        if (lane == 0) w_ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
-        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-        if (!w_ok) { ok = false; break; }
-        if (GATHER) {
-          const int c = lane & 7;
-          uint8_t* a_tile = smemA + stage * A_STAGE_BYTES;
-          const __nv_bfloat16* xa = static_cast<const __nv_bfloat16*>(args.gather_src) +
-                                    kb * BK + c * 8;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int r = 4 * i + (lane >> 3);
-            cp_async_16(a_tile + r * 128 + ((c ^ (r & 7)) << 4),
-                        xa + static_cast<size_t>(tok[i]) * args.K);
-          }
-          cp_async_arrive(&full_bar[stage]);
-          __syncwarp();
-        }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full_bar[stage],
-                                GATHER ? Cfg::B_STAGE_BYTES : Cfg::STAGE_BYTES);
-          if (!GATHER)
-            tma_load_2d(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
-          uint8_t* b = smemB + stage * Cfg::B_STAGE_BYTES;
-          if (SWIGLU) {
-            tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
-            tma_load_2d(b + (BN_ACC / 2) * BK * 2, &tmB1, &full_bar[stage], kb * BK, brow);
-          } else {
-            tma_load_2d(b, &tmB0, &full_bar[stage], kb * BK, brow);
-          }
-        }
-        issued_mask |= 1u << stage;
-        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-      }
-    }
-    if (lane == 0) pdl_trigger();   // all loads issued: the next kernel may launch
-    if (!ok && lane == 0) {
-      // Let every TMA copy this CTA started land before the CTA exits.
-      for (int s = 0; s < STAGES; ++s) {
-        if (!(issued_mask & (1u << s))) continue;
-        const uint32_t par = (issued_phase >> s) & 1u;
-        const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(&full_bar[s], par)) {
-          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      bool ok = true;
-      bool issued_any = false;
-      for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN_ACC;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
-          // cp.async wrote the A tile through the generic proxy; make it
-          // visible to the tensor core's async-proxy reads
-          if (GATHER) fence_async_shared();
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smemA + stage * A_STAGE_BYTES);
-          const uint32_t b_addr = smem_u32(smemB + stage * Cfg::B_STAGE_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a_addr + kk * 32);
-            const uint64_t bd = smem_desc_sw128(b_addr + kk * 32);
-            tc_mma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
-          }
-          issued_any = true;
-          tc_commit(&empty_bar[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-        tc_commit(&tfull_bar[acc]);
-      }
-      if (!ok && issued_any) {
-        // Wait (bounded) for the MMAs already issued before TMEM is freed.
-        tc_commit(drain_bar);
-        const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0)) {
-          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;                   // TMEM lane quadrant of this warp
-    const int row = q * 32 + lane;            // accumulator row owned by this thread
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
-      // every lane waits (memory ordering); the decision is made warp-uniform
-      // so the .sync.aligned TMEM loads below never run with a lane missing
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      const int g = find_group(s_prefix, G, tile);
-      const int rows_g = s_off[g + 1] - s_off[g];
-      int m, n;
-      tile_mn(tile - s_prefix[g], rows_g, n_tiles, args.m_fastest, m, n);
-      const bool valid = (m * BM + row) < rows_g;
-      // a warp whose 32 rows all belong to this group stages its rows in
-      // shared memory and writes them with one TMA store per 64 columns;
-      // a warp that straddles the end of the group stores its valid rows
-      // directly, so the next group's rows are never touched
-      const bool warp_full = (m * BM + q * 32 + 32) <= rows_g;
-      const int warp_row0 = s_off[g] + m * BM + q * 32;
-      uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
-      const size_t crow_off = static_cast<size_t>(s_off[g] + m * BM + row) * args.ldc +
-                              static_cast<size_t>(n) * BN_OUT;
-      const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-      for (int cb = 0; cb < BN_OUT / 64; ++cb) {
-        uint32_t packed[32];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int c0 = cb * 64 + half * 32;      // first output column of this half
-          uint32_t v[32];
-          if (SWIGLU) {
-            uint32_t u[32];
-            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-            tmem_ld16(t_addr + BN_OUT + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
-            tmem_ld16(t_addr + BN_OUT + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
-              const float h1 =
-                  silu_f32(__uint_as_float(v[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-              packed[half * 16 + i] = pack_bf16x2(h0, h1);
-            }
-          } else {
-            tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
-            tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[half * 16 + i] =
-                  pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-          }
-        }
-        if (warp_full) {
-          if (lane == 0) bulk_wait_read_all();     // previous store has left the buffer
-          __syncwarp();
-          // row `lane`, 16-byte chunk c lands at chunk c ^ (lane % 8) (128-byte swizzle)
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(stage_buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
-                           packed[4 * c + 3]);
-          fence_async_shared();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmC, stage_buf, n * BN_OUT + cb * 64, warp_row0);
-            bulk_commit();
-          }
-        } else if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
-                                                cb * 64);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
-                                packed[4 * c + 3]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-    }
-    if (lane == 0) bulk_wait_all();            // this warp's TMA stores are complete
-    __syncwarp();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0 && s_abort) atomicOr(args.status, kDevTimeout);
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
-  }
-}
-
 // --------------------------------------------------- CTA-pair (2-SM) kernel
 // The same grouped GEMM with a cluster of two CTAs per 256 x BN_ACC tile:
 // rank r holds rows [128 r, 128 r + 128) of the A tile and half of the B tile
@@ -479,19 +200,50 @@ struct PairCfg {
   static_assert(TMEM_COLS <= 512, "TMEM holds 512 columns");
 };
 
-template <int BN_ACC, int MODE>
+template <int BN_OUT>
+__device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_off,
+                                              const int* s_prefix, int G, int n_tiles, int tile) {
+  PairTile t;
+  if (tile >= s_prefix[G]) {
+    const int local = tile - s_prefix[G];
+    const int xn = a.x_n / BN_OUT;
+    t.x = true;
+    t.g = 0;
+    t.m = local / xn;
+    t.n = local - t.m * xn;
+    t.row0 = 0;
+    t.rows = a.x_rows;
+    t.kblocks = a.x_K / BK;
+  } else {
+    t.x = false;
+    t.g = find_group(s_prefix, G, tile);
+    t.row0 = s_off[t.g];
+    t.rows = s_off[t.g + 1] - s_off[t.g];
+    tile_mn<BM2>(tile - s_prefix[t.g], t.rows, n_tiles, a.m_fastest, t.m, t.n);
+    t.kblocks = a.K / BK;
+  }
+  return t;
+}
+
+template <int BN_ACC, int MODE, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1,
-                         const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+                         const __grid_constant__ CUtensorMap tmC,
+                         const __grid_constant__ CUtensorMap tmA2,
+                         const __grid_constant__ CUtensorMap tmB0_2,
+                         const __grid_constant__ CUtensorMap tmB1_2,
+                         const __grid_constant__ CUtensorMap tmC2, const GemmArgs args) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
+  constexpr bool BMN = MODE == MODE_PLAIN_BMN;
   constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
   constexpr int NSUB = Cfg::NSUB;
   constexpr int NACC = Cfg::NACC;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM2, Cfg::N_MMA);
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM2, Cfg::N_MMA, BMN);
+  constexpr int BOX_MN = 64 * 128;   // PLAIN_BMN: one 64-column box of 64 k-rows
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -535,8 +287,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    if (SWIGLU) tma_prefetch_desc(&tmB1);
+    if (SWIGLU || BMN) tma_prefetch_desc(&tmB1);
     tma_prefetch_desc(&tmC);
+    if (args.x_rows > 0) {
+      tma_prefetch_desc(&tmA2);
+      tma_prefetch_desc(&tmB0_2);
+      if (SWIGLU) tma_prefetch_desc(&tmB1_2);
+      tma_prefetch_desc(&tmC2);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(&s_tmem_base, Cfg::TMEM_COLS);
@@ -550,34 +308,77 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int total_tiles = s_prefix[G];
+  const int x_tiles = args.x_rows > 0 ? (args.x_rows + BM2 - 1) / BM2 * (args.x_n / BN_OUT) : 0;
+  const int total_tiles = s_prefix[G] + x_tiles;
   volatile int* abort_flag = &s_abort;
-  const int kblocks = args.K / BK;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
-      bool ok = true;
-      for (int tile = pair; tile < total_tiles && ok; tile += npairs) {
-        const int g = find_group(s_prefix, G, tile);
-        int m, n;
-        tile_mn<BM2>(tile - s_prefix[g], s_off[g + 1] - s_off[g], n_tiles, args.m_fastest, m, n);
-        const int arow = s_off[g] + m * BM2 + static_cast<int>(rank) * BM;
-        const int brow = SWIGLU ? g * args.n_per_group + n * BN_OUT
-                                : g * args.n_per_group + n * BN_OUT + static_cast<int>(rank) * (BN_ACC / 2);
-        const CUtensorMap* mb = (SWIGLU && rank == 1) ? &tmB1 : &tmB0;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
-          tma_load_2d_pair(smemA + stage * A_STAGE_BYTES, &tmA, &full_bar[stage], kb * BK, arow);
-          tma_load_2d_pair(smemB + stage * Cfg::B_HALF_BYTES, mb, &full_bar[stage], kb * BK, brow);
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    // Lane 0 waits for free stages, arms the barrier and loads B (and A
+    // tiles).  GATHER: the A rows of a routed tile are gathered from x by
+    // the permutation instead, every lane fetching four rows per stage with
+    // one tile::gather4 load (row r of the tile, r = 4 lane + q, is token
+    // gather_rows[first row + r], clamped into range; rows past the group
+    // load a valid row whose result is never stored).
+    int stage = 0;
+    uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
+    bool ok = true;
+    // without gathers lane 0 alone drives the ring
+    for (int tile = pair; tile < total_tiles && ok && (GATHER || lane == 0); tile += npairs) {
+      const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
+      const int g = pt.g, n = pt.n, kblocks = pt.kblocks;
+      const int arow = pt.row0 + pt.m * BM2 + static_cast<int>(rank) * BM;
+      const int gbase = pt.x ? 0 : g * args.n_per_group;
+      const int brow = SWIGLU ? gbase + n * BN_OUT
+                              : gbase + n * BN_OUT + static_cast<int>(rank) * (BN_ACC / 2);
+      const CUtensorMap* ma = pt.x ? &tmA2 : &tmA;
+      const CUtensorMap* mb = (SWIGLU && rank == 1) ? (pt.x ? &tmB1_2 : &tmB1)
+                                                    : (pt.x ? &tmB0_2 : &tmB0);
+      const bool gathered = GATHER && !pt.x;
+      int tok[4] = {0, 0, 0, 0};
+      if (gathered) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          int r = arow + 4 * lane + q;
+          r = r < args.gather_limit ? r : args.gather_limit - 1;
+          const int t = __ldg(args.gather_rows + r);
+          tok[q] = t < 0 ? 0 : (t >= args.gather_src_rows ? args.gather_src_rows - 1 : t);
         }
       }
+      for (int kb = 0; kb < kblocks; ++kb) {
+        bool w_ok = true;
+        if (lane == 0) w_ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
+        if (GATHER) w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
+        if (!w_ok) { ok = false; break; }
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
+          if (!gathered)
+            tma_load_2d_pair(smemA + stage * A_STAGE_BYTES, ma, &full_bar[stage], kb * BK, arow);
+          if (BMN) {
+            // this CTA's BN_ACC/2 columns of B, 64 columns (one box) at a time
+            const bool first = kb < args.kb_split;
+            const CUtensorMap* mbk = first ? &tmB0 : &tmB1;
+            const int krow = first ? g * args.b0_rows + kb * BK
+                                   : g * args.b1_rows + (kb - args.kb_split) * BK;
+            const int col0 = n * BN_ACC + static_cast<int>(rank) * (BN_ACC / 2);
+#pragma unroll
+            for (int j = 0; j < BN_ACC / 128; ++j)
+              tma_load_2d_pair(smemB + stage * Cfg::B_HALF_BYTES + j * BOX_MN, mbk,
+                               &full_bar[stage], col0 + j * 64, krow);
+          } else {
+            tma_load_2d_pair(smemB + stage * Cfg::B_HALF_BYTES, mb, &full_bar[stage], kb * BK,
+                             brow);
+          }
+        }
+        if (gathered)
+          tma_gather4_pair(smemA + stage * A_STAGE_BYTES + lane * 512, ma, &full_bar[stage],
+                           kb * BK, tok[0], tok[1], tok[2], tok[3]);
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (lane == 0) {
       pdl_trigger();   // all loads issued: the next kernel may launch
       if (!ok && rank == 0) {
         // rank 0's stage barriers count both CTAs' copies: let them all land
@@ -599,6 +400,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++it) {
         const int acc = it % NACC;
         const uint32_t acc_phase = (it / NACC) & 1;
+        const int kblocks = tile >= s_prefix[G] ? args.x_K / BK : args.K / BK;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN_ACC;
@@ -610,10 +412,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
 #pragma unroll
-            for (int sub = 0; sub < NSUB; ++sub)   // sub-tile: B rows [128 sub, 128 sub + 128)
-              tc_mma_f16_pair(d_tmem + sub * Cfg::N_MMA, smem_desc_sw128(a_addr + kk * 32),
-                              smem_desc_sw128(b_addr + sub * (Cfg::N_MMA / 2) * 128 + kk * 32),
+            for (int sub = 0; sub < NSUB; ++sub) {  // sub-tile: B rows [128 sub, 128 sub + 128)
+              const uint32_t bsub = b_addr + sub * (Cfg::N_MMA / 2) * 128;
+              const uint64_t bd = BMN ? smem_desc_sw128_mn(bsub + kk * 16 * 128, BOX_MN)
+                                      : smem_desc_sw128(bsub + kk * 32);
+              tc_mma_f16_pair(d_tmem + sub * Cfg::N_MMA, smem_desc_sw128(a_addr + kk * 32), bd,
                               IDESC, (kb | kk) != 0 ? 1u : 0u);
+            }
           issued_any = true;
           tc_commit_pair(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -639,16 +444,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const int g = find_group(s_prefix, G, tile);
-      const int rows_g = s_off[g + 1] - s_off[g];
-      int m, n;
-      tile_mn<BM2>(tile - s_prefix[g], rows_g, n_tiles, args.m_fastest, m, n);
-      const int r0 = m * BM2 + static_cast<int>(rank) * BM;   // first row (in group) of this CTA
+      const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
+      const int rows_g = pt.rows, n = pt.n;
+      const int r0 = pt.m * BM2 + static_cast<int>(rank) * BM;   // first row (in group) of this CTA
       const bool valid = (r0 + row) < rows_g;
       const bool warp_full = (r0 + q * 32 + 32) <= rows_g;
-      const int warp_row0 = s_off[g] + r0 + q * 32;
+      const int warp_row0 = pt.row0 + r0 + q * 32;
       uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
-      const size_t crow_off = static_cast<size_t>(s_off[g] + r0 + row) * args.ldc;
+      const CUtensorMap* mc = pt.x ? &tmC2 : &tmC;
+      __nv_bfloat16* cbase = static_cast<__nv_bfloat16*>(pt.x ? args.x_C : args.C);
+      const size_t crow_off = static_cast<size_t>(pt.row0 + r0 + row) * (pt.x ? args.x_ldc : args.ldc);
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
       for (int cb = 0; cb < BN_OUT / 64; ++cb) {
@@ -709,12 +514,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmC, stage_buf, ocol, warp_row0);
+            tma_store_2d(mc, stage_buf, ocol, warp_row0);
             bulk_commit();
           }
         } else if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.C) + crow_off +
-                                                ocol);
+          uint4* dst = reinterpret_cast<uint4*>(cbase + crow_off + ocol);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2],
@@ -782,45 +586,13 @@ int num_sms() {
 }
 
 template <int BN_ACC, int MODE, bool GATHER = false>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                   const CUtensorMap& c, const GemmArgs& args, int rows_upper,
-                   cudaStream_t stream) {
-  using Cfg = GemmCfg<BN_ACC>;
-  constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
-  auto kern = grouped_gemm_kernel<BN_ACC, MODE, GATHER>;
-  static unsigned long long attr_done = 0;   // one bit per device (attribute is per device)
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_done & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done |= bit;
-  }
-  const int G = args.offsets == nullptr ? 1 : args.num_groups;
-  // m-fastest order once one group's weights (B rows x K, both halves for
-  // SwiGLU) exceed 32 MB, a quarter of the L2
-  GemmArgs a2 = args;
-  const double b_bytes = static_cast<double>(BN_OUT == BN_ACC ? args.n_per_group
-                                                              : 2 * args.n_per_group) *
-                         args.K * 2.0;
-  a2.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
-  const long long m_tiles_upper = (rows_upper + BM - 1) / BM + (G > 1 ? G : 0);
-  const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
-  if (tiles_upper <= 0) return cudaSuccess;
-  const int grid = static_cast<int>(tiles_upper < num_sms() ? tiles_upper : num_sms());
-  return launch_pdl(kern, dim3(grid), dim3(NUM_THREADS), Cfg::SMEM_BYTES, stream, a, b0, b1, c,
-                    a2);
-}
-
-template <int BN_ACC, int MODE>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const CUtensorMap& c, const GemmArgs& args, int rows_upper,
-                        cudaStream_t stream) {
+                        const CUtensorMap& c, const CUtensorMap& a2, const CUtensorMap& b0_2,
+                        const CUtensorMap& b1_2, const CUtensorMap& c2, const GemmArgs& args,
+                        int rows_upper, cudaStream_t stream) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
-  auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE>;
+  auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE, GATHER>;
   static unsigned long long attr_done = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -832,79 +604,188 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     attr_done |= bit;
   }
   const int G = args.offsets == nullptr ? 1 : args.num_groups;
-  GemmArgs a2 = args;
+  GemmArgs a2r = args;
   const double b_bytes = static_cast<double>(BN_OUT == BN_ACC ? args.n_per_group
                                                               : 2 * args.n_per_group) *
                          args.K * 2.0;
-  a2.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
+  a2r.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
   const long long m_tiles_upper = (rows_upper + BM2 - 1) / BM2 + (G > 1 ? G : 0);
-  const long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
+  long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
+  if (args.x_rows > 0)
+    tiles_upper += static_cast<long long>((args.x_rows + BM2 - 1) / BM2) * (args.x_n / BN_OUT);
   if (tiles_upper <= 0) return cudaSuccess;
   const int max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles_upper < max_pairs ? tiles_upper : max_pairs);
   return launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), Cfg::SMEM_BYTES, stream, a, b0, b1,
-                    c, a2);
+                    c, a2, b0_2, b1_2, c2, a2r);
 }
 
 }  // namespace
 
-// h[r] = silu(A[r] W1[g]^T) * (A[r] W3[g]^T), bf16 out.
+// h[r] = silu(A[r] W1[g]^T) * (A[r] W3[g]^T), bf16 out.  extra: one more
+// group with tensors of its own (the shared expert), in the same launch.
 cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
-                                       cudaStream_t stream) {
-  CUtensorMap ta, tb0, tb1, tc;
+                                       cudaStream_t stream, const GemmExtraGroup* extra) {
+  CUtensorMap ta, tb0, tb1, tc, xa, xb0, xb1, xc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
   const int64_t c_rows = offsets ? a_rows : rows_single;
-  // 256 output columns per tile (512 accumulator columns) when F allows
-  const bool wide = F % 256 == 0;
-  const int bh = wide ? 256 : 128;   // B rows each CTA of the pair loads
+  // 128 output columns (gate + up = 256 accumulator columns, double
+  // buffered) per tile.  Measured on B200: 256 output columns per tile with
+  // one 512-column accumulator was slower on every workload (qwen3_30b
+  // gate/up 0.92 vs 0.66-0.70 ms): the epilogue is no longer hidden.
+  const int bh = 128;   // B rows each CTA of the pair loads
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, bh) ||
       !make_map(&tb1, W3, b_rows, K, bh) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0};
+  GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0, 0, 0, 0,
+                0, 0, 0, nullptr, 0, 0, 0};
+  if (extra != nullptr && extra->rows > 0) {
+    if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
+        !make_map(&xb0, extra->B0, extra->n, extra->K, bh) ||
+        !make_map(&xb1, extra->B1, extra->n, extra->K, bh) ||
+        !make_map(&xc, extra->C, extra->rows, extra->n, 32))
+      return cudaErrorInvalidValue;
+    args.x_rows = extra->rows;
+    args.x_n = extra->n;
+    args.x_K = extra->K;
+    args.x_C = extra->C;
+    args.x_ldc = extra->n;
+  } else {
+    xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
+  }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  if (wide) return launch_pair<512, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
-  return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, args, rows_upper, stream);
+  return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args, rows_upper,
+                                            stream);
 }
 
 // Gate/up pass whose A rows are gathered from X [x_rows, K]: output row r
-// (expert-contiguous order, r < R) reads X[rows[r]].  H is [R, F].
+// (expert-contiguous order, r < R) reads X[rows[r]] (tile::gather4 loads in
+// the CTA-pair kernel).  H is [R, F].  extra as for the plain gate/up pass
+// (its A rows are read directly).
 cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows,
                                               int64_t R, const int32_t* offsets, int num_groups,
                                               const void* W1, const void* W3, int F, int K,
-                                              void* H, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap tb0, tb1, tc;
+                                              void* H, uint32_t* status, cudaStream_t stream,
+                                              const GemmExtraGroup* extra) {
+  CUtensorMap ta, tb0, tb1, tc, xa, xb0, xb1, xc;
   const int64_t b_rows = static_cast<int64_t>(num_groups) * F;
-  (void)x_rows;
-  if (!make_map(&tb0, W1, b_rows, K, 128) || !make_map(&tb1, W3, b_rows, K, 128) ||
-      !make_map(&tc, H, R, F, 32))
+  if (!make_map(&ta, X, x_rows, K, 1) || !make_map(&tb0, W1, b_rows, K, 128) ||
+      !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, R, F, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0};
-  // tmA is unused in gather mode (A comes through cp.async)
-  return launch<256, MODE_SWIGLU_BF16, true>(tb0, tb0, tb1, tc, args, static_cast<int>(R), stream);
+  GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0, 0, 0, 0,
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
+  if (extra != nullptr && extra->rows > 0) {
+    if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
+        !make_map(&xb0, extra->B0, extra->n, extra->K, 128) ||
+        !make_map(&xb1, extra->B1, extra->n, extra->K, 128) ||
+        !make_map(&xc, extra->C, extra->rows, extra->n, 32))
+      return cudaErrorInvalidValue;
+    args.x_rows = extra->rows;
+    args.x_n = extra->n;
+    args.x_K = extra->K;
+    args.x_C = extra->C;
+    args.x_ldc = extra->n;
+  } else {
+    xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
+  }
+  return launch_pair<256, MODE_SWIGLU_BF16, true>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
+                                                  static_cast<int>(R), stream);
 }
 
-// Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.
+// Y[r] = X[rows[r]] W[g]^T for the expert-contiguous rows r < R (A rows
+// gathered from X [x_rows, K] as above); Y is [R, N].
+cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
+                                     const int32_t* offsets, int num_groups, const void* W, int N,
+                                     int K, void* Y, uint32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb, tc;
+  const int64_t b_rows = static_cast<int64_t>(num_groups) * N;
+  const int bn = (N % 256 == 0) ? 256 : 128;
+  if (!make_map(&ta, X, x_rows, K, 1) || !make_map(&tb, W, b_rows, K, bn / 2) ||
+      !make_map(&tc, Y, R, N, 32))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, 0, N, K, Y, N, status, rows, X, 0, 0, 0, 0,
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
+  if (bn == 256)
+    return launch_pair<256, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, ta, tb, tb, tc, args,
+                                                   static_cast<int>(R), stream);
+  return launch_pair<128, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, ta, tb, tb, tc, args,
+                                                 static_cast<int>(R), stream);
+}
+
+// Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.  extra: one
+// more group (the shared expert's down projection, same N), same launch.
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
-                              void* Y, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap ta, tb, tc;
+                              void* Y, uint32_t* status, cudaStream_t stream,
+                              const GemmExtraGroup* extra) {
+  CUtensorMap ta, tb, tc, xa, xb, xc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
   const int64_t c_rows = offsets ? a_rows : rows_single;
-  const int bn = (N % 512 == 0) ? 512 : (N % 256 == 0) ? 256 : 128;
+  // 512 accumulator columns (one TMEM buffer) only for long K, where the
+  // exposed epilogue is a small part of a tile: measured on B200, wide's
+  // down GEMM (K = 4352) 0.616 -> 0.551 ms, but qwen3_30b's (K = 768) 0.33 ->
+  // 0.38 ms
+  const int bn = (N % 512 == 0 && K >= 4096) ? 512 : (N % 256 == 0) ? 256 : 128;
   // each CTA of the pair loads half of the B tile
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
-  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0};
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0, 0, 0, 0,
+                0, 0, 0, nullptr, 0, 0, 0};
+  if (extra != nullptr && extra->rows > 0) {
+    if (extra->n != N || !make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
+        !make_map(&xb, extra->B0, N, extra->K, bn / 2) ||
+        !make_map(&xc, extra->C, extra->rows, N, 32))
+      return cudaErrorInvalidValue;
+    args.x_rows = extra->rows;
+    args.x_n = N;
+    args.x_K = extra->K;
+    args.x_C = extra->C;
+    args.x_ldc = N;
+  } else {
+    xa = ta; xb = tb; xc = tc;
+  }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (bn == 512)
-    return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+    return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
+                                             stream);
   if (bn == 256)
-    return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
-  return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, args, rows_upper, stream);
+    return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
+                                             stream);
+  return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
+                                           stream);
 }
 
+// Y[r] = A[r] B_g with B_g stored [K, N] (MN-major): its first b0_rows rows
+// from B0 [G * b0_rows, N], the remaining K - b0_rows from B1 [G * (K -
+// b0_rows), N] (B1 may be null when b0_rows == K).  b0_rows a multiple of 64.
+cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                  int num_groups, int rows_single, const void* B0,
+                                  const void* B1, int b0_rows, int N, int K, void* Y,
+                                  uint32_t* status, cudaStream_t stream) {
+  if (b0_rows % BK || b0_rows > K || (b0_rows < K && B1 == nullptr) || N % 128)
+    return cudaErrorInvalidValue;
+  CUtensorMap ta, tb0, tb1, tc;
+  const int64_t G = offsets ? num_groups : 1;
+  const int64_t c_rows = offsets ? a_rows : rows_single;
+  const int b1_rows = K - b0_rows;
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, B0, G * b0_rows, N, BK) ||
+      !make_map(&tb1, b1_rows ? B1 : B0, G * (b1_rows ? b1_rows : b0_rows), N, BK) ||
+      !make_map(&tc, Y, c_rows, N, 32))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
+                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0};
+  const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (N % 512 == 0 && K >= 4096)
+    return launch_pair<512, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
+                                            stream);
+  if (N % 256 == 0)
+    return launch_pair<256, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
+                                            stream);
+  return launch_pair<128, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
+                                          stream);
+}
 
 }  // namespace moe

@@ -104,17 +104,43 @@ cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              cudaStream_t stream);
 
 // Experts --------------------------------------------------------------------
+// One more group with tensors of its own, run in the same launch after the
+// routed groups: the shared expert over all T tokens (A = x or h_sh, B = its
+// weights, C = its output).  B1 is the up projection (gate/up pass only).
+struct GemmExtraGroup {
+  const void* A;
+  int rows;
+  const void* B0;
+  const void* B1;
+  int n;     // output columns
+  int K;
+  void* C;
+};
 cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
-                                       cudaStream_t stream);
+                                       cudaStream_t stream,
+                                       const GemmExtraGroup* extra = nullptr);
 cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows,
                                               int64_t R, const int32_t* offsets, int num_groups,
                                               const void* W1, const void* W3, int F, int K,
-                                              void* H, uint32_t* status, cudaStream_t stream);
+                                              void* H, uint32_t* status, cudaStream_t stream,
+                                              const GemmExtraGroup* extra = nullptr);
+// Y[r] = X[rows[r]] W[g]^T over the expert-contiguous rows r < R (A rows
+// gathered from X by the permutation; no permuted copy).
+cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
+                                     const int32_t* offsets, int num_groups, const void* W, int N,
+                                     int K, void* Y, uint32_t* status, cudaStream_t stream);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
-                              void* Y, uint32_t* status, cudaStream_t stream);
+                              void* Y, uint32_t* status, cudaStream_t stream,
+                              const GemmExtraGroup* extra = nullptr);
+// Y[r] = A[r] B_g, B_g [K, N] read MN-major (no transposed copy): its first
+// b0_rows rows from B0 [G * b0_rows, N], the others from B1.
+cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                  int num_groups, int rows_single, const void* B0,
+                                  const void* B1, int b0_rows, int N, int K, void* Y,
+                                  uint32_t* status, cudaStream_t stream);
 cudaError_t grouped_swiglu_gateup_f32(const float* A, int64_t a_rows, const int32_t* offsets,
                                       int num_groups, int rows_single, const float* W1,
                                       const float* W3, int F, int K, float* H,
@@ -132,8 +158,6 @@ cudaError_t grouped_wgrad_bf16(const void* A, const void* B, int64_t kp, const i
 cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos,
                    const float* topk_w, void* dy, float* dw, int T, int d, int k,
                    cudaStream_t stream);
-cudaError_t transpose_bf16(const void* in, int batches, int rows, int cols, void* out, int ldo,
-                           int col_off, cudaStream_t stream);
 cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,
                         cudaStream_t stream);
 cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,

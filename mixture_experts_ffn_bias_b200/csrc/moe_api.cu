@@ -213,23 +213,23 @@ moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* o
   const int E = c->n_experts, F = c->d_ff, d = c->d_model;
   void* h = at<void>(ws, L.h);
   if (c->dtype == MOE_BF16) {
-    if (x_perm == nullptr)
+    // the shared expert runs as one more group of the routed launches
+    void* hs = at<void>(ws, L.h_sh);
+    const int Fs = c->d_ff_shared;
+    const moe::GemmExtraGroup sh_up{x, c->T, w->ws1, w->ws3, Fs, d, hs};
+    const moe::GemmExtraGroup sh_down{hs, c->T, w->ws2, nullptr, d, Fs, y_shared};
+    if (x_perm == nullptr) {
       MOE_TRY(moe::grouped_swiglu_gateup_gather_bf16(x, c->T, gather_rows, R, offsets, E, w->w1,
-                                                     w->w3, F, d, h, status, s));
-    else
+                                                     w->w3, F, d, h, status, s,
+                                                     c->n_shared ? &sh_up : nullptr));
+    } else {
       MOE_TRY(moe::grouped_swiglu_gateup_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d, h,
-                                              status, s));
-    if (!mk.rec(3)) return MOE_ERR_CUDA;
-    MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s));
-    if (!mk.rec(4)) return MOE_ERR_CUDA;
-    if (c->n_shared) {
-      void* hs = at<void>(ws, L.h_sh);
-      const int Fs = c->d_ff_shared;
-      MOE_TRY(moe::grouped_swiglu_gateup_bf16(x, c->T, nullptr, 1, c->T, w->ws1, w->ws3, Fs, d,
-                                              hs, status, s));
-      MOE_TRY(moe::grouped_down_bf16(hs, c->T, nullptr, 1, c->T, w->ws2, d, Fs, y_shared,
-                                     status, s));
+                                              status, s, c->n_shared ? &sh_up : nullptr));
     }
+    if (!mk.rec(3)) return MOE_ERR_CUDA;
+    MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s,
+                                   c->n_shared ? &sh_down : nullptr));
+    if (!mk.rec(4)) return MOE_ERR_CUDA;
   } else {
     float* hf = static_cast<float*>(h);
     MOE_TRY(moe::grouped_swiglu_gateup_f32(static_cast<const float*>(x_perm), R, offsets, E, 0,
@@ -342,9 +342,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
 
 // Workspace of moe_backward (separate from the forward's, which it reads).
 struct BLayout {
-  size_t status, dw, logits, dlogits, part, dxr, poff, poff_sh, w2t, w13t, dy, dh, gb, ub, dgu,
-      dxp, dyT, hT, dguT, xT, ws2t, ws13t, dh_sh, g_sh, u_sh, dgu_sh, dxs, doutT, hshT, dgushT,
-      xTs, total;
+  size_t status, dw, logits, dlogits, part, dxr, poff, poff_sh, dy, dh, gb, ub, dgu, dxp, dyT,
+      hT, dguT, xT, dh_sh, g_sh, u_sh, dgu_sh, dxs, doutT, hshT, dgushT, xTs, total;
   int64_t kp, tp;
 };
 
@@ -366,8 +365,6 @@ BLayout blayout(const moe_config& c) {
   B.dxr = o;     o += up(T * d * 4);
   B.poff = o;    o += up((E + 1) * 4);
   B.poff_sh = o; o += up(2 * 4);
-  B.w2t = o;     o += up(E * F * d * 2);
-  B.w13t = o;    o += up(E * d * 2 * F * 2);
   B.dy = o;      o += up(R * d * 2);
   B.dh = o;      o += up(R * F * 2);
   B.gb = o;      o += up(R * F * 2);
@@ -378,8 +375,6 @@ BLayout blayout(const moe_config& c) {
   B.hT = o;      o += up(F * kp * 2);
   B.dguT = o;    o += up(2 * F * kp * 2);
   B.xT = o;      o += up(d * kp * 2);
-  B.ws2t = o;    o += up(Fs * d * 2);
-  B.ws13t = o;   o += up(d * 2 * Fs * 2);
   B.dh_sh = o;   o += up(T * Fs * 2);
   B.g_sh = o;    o += up(T * Fs * 2);
   B.u_sh = o;    o += up(T * Fs * 2);
@@ -394,7 +389,7 @@ BLayout blayout(const moe_config& c) {
 }
 
 // The layer's backward (bf16 layers).  fws holds the state of the forward:
-// offsets, slot_pos, perm_src, x_perm, h, y_perm (and h_sh).
+// offsets, slot_pos, perm_src, h, y_perm (and h_sh).
 moe_status backward_impl(const moe_config* c, const void* x, const void* w_router,
                          const float* logit_offset, const moe_expert_weights* w,
                          const int32_t* topk_idx, const float* topk_w, const void* dout,
@@ -408,28 +403,26 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
   const int32_t* offsets = at<int32_t>(fws, L.offsets);
   const int32_t* slot_pos = at<int32_t>(fws, L.slot_pos);
   const int32_t* perm_src = at<int32_t>(fws, L.perm_src);
-  const void* x_perm = at<void>(fws, L.x_perm);
   const void* h = at<void>(fws, L.h);
   const void* y_perm = at<void>(fws, L.y_perm);
   float* dw = at<float>(bws, B.dw);
   int32_t* poff = at<int32_t>(bws, B.poff);
   // combine: dw and the experts' output gradients
   MOE_TRY(moe::bwd_dy(dout, y_perm, slot_pos, topk_w, at<void>(bws, B.dy), dw, T, d, k, s));
-  // transposed weights (W2^T [E, F, d]; [W1^T | W3^T] [E, d, 2F])
-  MOE_TRY(moe::transpose_bf16(w->w2, E, d, F, at<void>(bws, B.w2t), d, 0, s));
-  MOE_TRY(moe::transpose_bf16(w->w1, E, F, d, at<void>(bws, B.w13t), 2 * F, 0, s));
-  MOE_TRY(moe::transpose_bf16(w->w3, E, F, d, at<void>(bws, B.w13t), 2 * F, F, s));
-  // dH = dY W2 ; G, U recomputed ; dG, dU ; dX = [dG | dU] [W1 ; W3]
-  MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dy), R, offsets, E, 0, at<void>(bws, B.w2t), F,
-                                 d, at<void>(bws, B.dh), status, s));
-  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w1, F, d, at<void>(bws, B.gb),
-                                 status, s));
-  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w3, F, d, at<void>(bws, B.ub),
-                                 status, s));
+  // dH = dY W2 ; G, U recomputed ; dG, dU ; dX = [dG | dU] [W1 ; W3].  The
+  // weights of dH and dX are read MN-major in place (no transposed copies).
+  MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dy), R, offsets, E, 0, w->w2, nullptr, d,
+                                     F, d, at<void>(bws, B.dh), status, s));
+  // G and U recomputed from x's rows gathered by the permutation (the
+  // forward may not have kept a permuted copy of x)
+  MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w1, F, d,
+                                        at<void>(bws, B.gb), status, s));
+  MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w3, F, d,
+                                        at<void>(bws, B.ub), status, s));
   MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.gb), at<void>(bws, B.ub), at<void>(bws, B.dh),
                           at<void>(bws, B.dgu), R, F, s));
-  MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, at<void>(bws, B.w13t),
-                                 d, 2 * F, at<void>(bws, B.dxp), status, s));
+  MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, w->w1, w->w3, F, d,
+                                     2 * F, at<void>(bws, B.dxp), status, s));
   // weight gradients over each expert's rows (transposed, padded operands)
   MOE_TRY(moe::pad_offsets(offsets, E, 0, poff, s));
   MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dy), d, offsets, E, 0, poff, nullptr,
@@ -451,20 +444,16 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
   if (c->n_shared) {
     const int Fs = c->d_ff_shared;
     int32_t* poff_sh = at<int32_t>(bws, B.poff_sh);
-    MOE_TRY(moe::transpose_bf16(w->ws2, 1, d, Fs, at<void>(bws, B.ws2t), d, 0, s));
-    MOE_TRY(moe::transpose_bf16(w->ws1, 1, Fs, d, at<void>(bws, B.ws13t), 2 * Fs, 0, s));
-    MOE_TRY(moe::transpose_bf16(w->ws3, 1, Fs, d, at<void>(bws, B.ws13t), 2 * Fs, Fs, s));
-    MOE_TRY(moe::grouped_down_bf16(dout, T, nullptr, 1, T, at<void>(bws, B.ws2t), Fs, d,
-                                   at<void>(bws, B.dh_sh), status, s));
+    MOE_TRY(moe::grouped_gemm_bmn_bf16(dout, T, nullptr, 1, T, w->ws2, nullptr, d, Fs, d,
+                                       at<void>(bws, B.dh_sh), status, s));
     MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws1, Fs, d, at<void>(bws, B.g_sh),
                                    status, s));
     MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws3, Fs, d, at<void>(bws, B.u_sh),
                                    status, s));
     MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.g_sh), at<void>(bws, B.u_sh),
                             at<void>(bws, B.dh_sh), at<void>(bws, B.dgu_sh), T, Fs, s));
-    MOE_TRY(moe::grouped_down_bf16(at<void>(bws, B.dgu_sh), T, nullptr, 1, T,
-                                   at<void>(bws, B.ws13t), d, 2 * Fs, at<void>(bws, B.dxs),
-                                   status, s));
+    MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu_sh), T, nullptr, 1, T, w->ws1,
+                                       w->ws3, Fs, d, 2 * Fs, at<void>(bws, B.dxs), status, s));
     dxs = at<void>(bws, B.dxs);
     MOE_TRY(moe::pad_offsets(nullptr, 1, T, poff_sh, s));
     const int tp = static_cast<int>(B.tp);

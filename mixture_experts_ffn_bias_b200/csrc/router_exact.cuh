@@ -6,8 +6,7 @@
 // fp32 key was within the margin of its (k+1)-th pick, which must contain the
 // exact top-k) or all experts.  Their exact logits are fp64 sums of exact
 // bf16 x bf16 products.  Selection uses the fp64 keys (ties to the lower
-// expert id); the weights are formed in fp32 from the exact logits.  One warp
-// handles one token.
+// expert id); the weights are formed in fp32 from the exact logits.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -133,44 +132,59 @@ __device__ __noinline__ void refine_select(const double* s_l, const int* s_e, in
 }
 
 
-// Exact logits of candidates s_e[0..n) of token row x_row (bf16, d
-// elements): s_l[c] = fp64 sum of the exact products (+ offset[e]).  Each
-// warp lane reads 16-byte pieces of x and of two router rows at a time.
-__device__ __noinline__ void exact_logits_warp(const __nv_bfloat16* __restrict__ x_row,
+// Exact logits of a batch of (token, expert) pairs, all the listed tokens of
+// a block at once: pair p is token row x + s_pt[p] * d and router row
+// s_pe[p]; s_pl[p] = fp64 sum of the exact bf16 x bf16 products (+
+// offset[e]).  Warp `first` of `step` warps takes pairs first, first + step,
+// ..., two at a time, with the 16-byte loads of four column steps of both
+// pairs issued before they are used: the rows come from L2, so the time is
+// load latency, and one round of it covers up to 512 columns of two pairs.
+__device__ __noinline__ void exact_pair_logits(const __nv_bfloat16* __restrict__ x,
                                                const __nv_bfloat16* __restrict__ wr,
                                                const float* __restrict__ offset, int d,
-                                               const int* s_e, int n, double* s_l) {
+                                               const int* s_pt, const int* s_pe, int npairs,
+                                               double* s_pl, int first, int step) {
   const int lane = threadIdx.x & 31;
-  const uint4* xr = reinterpret_cast<const uint4*>(x_row);
-  for (int c0 = 0; c0 < n; c0 += 2) {
-    const int c1 = c0 + 1;
-    const int e0 = s_e[c0], e1 = c1 < n ? s_e[c1] : e0;
-    const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
-    const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1) * d);
-    double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int col = lane * 8; col < d; col += 256) {
-      const uint4 ux = __ldg(xr + col / 8), u0 = __ldg(r0 + col / 8), u1 = __ldg(r1 + col / 8);
-      const __nv_bfloat16* hx = reinterpret_cast<const __nv_bfloat16*>(&ux);
-      const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
-      const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+  for (int p0 = first; p0 < npairs; p0 += 2 * step) {
+    const int p1 = p0 + step < npairs ? p0 + step : p0;
+    const uint4* xa = reinterpret_cast<const uint4*>(x + static_cast<size_t>(s_pt[p0]) * d);
+    const uint4* xb = reinterpret_cast<const uint4*>(x + static_cast<size_t>(s_pt[p1]) * d);
+    const uint4* wa = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(s_pe[p0]) * d);
+    const uint4* wb = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(s_pe[p1]) * d);
+    double sa = 0.0, sb = 0.0;
+    const int nv = d / 8;   // 16-byte pieces per row
+    for (int v0 = lane; v0 < nv; v0 += 4 * 32) {
+      uint4 ux[4], uw[4], vx[4], vw[4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        // bf16 x bf16 products are exact in fp32; the sums run in fp64
-        const float xv = __bfloat162float(hx[j]);
-        a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv);
-        b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv);
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + 32 * u;
+        const bool in = v < nv;
+        ux[u] = in ? __ldg(xa + v) : make_uint4(0u, 0u, 0u, 0u);
+        uw[u] = in ? __ldg(wa + v) : make_uint4(0u, 0u, 0u, 0u);
+        vx[u] = in ? __ldg(xb + v) : make_uint4(0u, 0u, 0u, 0u);
+        vw[u] = in ? __ldg(wb + v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat16* hx = reinterpret_cast<const __nv_bfloat16*>(&ux[u]);
+        const __nv_bfloat16* hw = reinterpret_cast<const __nv_bfloat16*>(&uw[u]);
+        const __nv_bfloat16* gx = reinterpret_cast<const __nv_bfloat16*>(&vx[u]);
+        const __nv_bfloat16* gw = reinterpret_cast<const __nv_bfloat16*>(&vw[u]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {   // exact fp32 products, fp64 sums
+          sa += static_cast<double>(__bfloat162float(hw[j]) * __bfloat162float(hx[j]));
+          sb += static_cast<double>(__bfloat162float(gw[j]) * __bfloat162float(gx[j]));
+        }
       }
     }
-    double s0 = (a[0] + a[1]) + (a[2] + a[3]);
-    double s1 = (b[0] + b[1]) + (b[2] + b[3]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      sa += __shfl_xor_sync(0xffffffffu, sa, o);
+      sb += __shfl_xor_sync(0xffffffffu, sb, o);
     }
     if (lane == 0) {
-      s_l[c0] = s0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
-      if (c1 < n) s_l[c1] = s1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+      s_pl[p0] = sa + (offset ? static_cast<double>(offset[s_pe[p0]]) : 0.0);
+      if (p1 != p0) s_pl[p1] = sb + (offset ? static_cast<double>(offset[s_pe[p1]]) : 0.0);
     }
   }
   __syncwarp();

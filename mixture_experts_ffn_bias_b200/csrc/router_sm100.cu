@@ -557,6 +557,7 @@ bool maps(const void* x, int T, const void* w_router, int E, int K, CUtensorMap*
 // Warp roles: warp 0 TMA producer, warp 1 TMEM owner and (rank 0) MMA
 // issuer, warps 2-5 epilogue.  No load uses cluster multicast.
 constexpr int PR_LIST_MAX = 128;
+constexpr int PR_PAIRS_MAX = 512;   // (token, candidate) pairs re-decided per batch
 
 struct PairRouterArgs {
   const __nv_bfloat16* x;     // [T, K] (exact re-decision reads its rows)
@@ -763,15 +764,17 @@ router_pair_kernel(const __grid_constant__ CUtensorMap tmX,
   uint64_t* sempty_bar = bars + 2 * C::STAGES + C::NSLOT;  // rank 0's copy, 8 arrivals
   uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_abort, s_epi_abort, s_nlist, s_last;
+  __shared__ int s_abort, s_epi_abort, s_nlist, s_last, s_nlist_batch;
   __shared__ __align__(16) float s_off[NSEL];
   __shared__ __align__(16) float s_bias[NSEL];
   __shared__ int s_sel[(KMAX_FUSED + 1) * 128];
   __shared__ uint32_t s_masks[NSEL][4];
   __shared__ int s_list[PR_LIST_MAX];
   __shared__ int s_cand[PR_LIST_MAX * kRefineCand];
-  __shared__ double s_rl[4][256];
-  __shared__ int s_re[4][256];
+  __shared__ double s_pl[PR_PAIRS_MAX];    // exact logits of the batch's pairs
+  __shared__ int s_pt[PR_PAIRS_MAX];       // their token rows
+  __shared__ int s_pe[PR_PAIRS_MAX];       // their experts
+  __shared__ int s_pbase[PR_LIST_MAX + 1]; // first pair of each listed token
   __shared__ int s_cnt[NSEL];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -941,29 +944,53 @@ router_pair_kernel(const __grid_constant__ CUtensorMap tmX,
         pair_route_row<NSEL>(acc, s_log, sel, s_off, s_bias, E, t, row, a, &s_nlist, s_list,
                              s_cand);
       epi_bar();
-      // exact re-decision of the listed tokens, one warp per token
+      // exact re-decision of the listed tokens: their (token, candidate)
+      // pairs in batches of up to PR_PAIRS_MAX, the exact logits of a batch
+      // by the four epilogue warps together, then one warp per token decides
       const int nlist = s_nlist;
       refined += nlist;
-      for (int i = ew; i < nlist; i += 4) {
-        const int r = s_list[i];
-        const int tt = b * a.tpc + r;
-        const int* cand = s_cand + i * kRefineCand;
-        const bool all = cand[0] == -2;
-        int n = E;
-        if (!all) {
-          n = 0;
-          while (n < kRefineCand && cand[n] >= 0) ++n;
+      for (int i0 = 0; i0 < nlist;) {
+        if (et == 0) {
+          int np = 0, i = i0;
+          for (; i < nlist; ++i) {
+            const int* cand = s_cand + i * kRefineCand;
+            int n = E;
+            if (cand[0] != -2) {
+              n = 0;
+              while (n < kRefineCand && cand[n] >= 0) ++n;
+            }
+            if (np + n > PR_PAIRS_MAX && i > i0) break;   // the next batch takes it
+            s_pbase[i - i0] = np;
+            np += n;
+          }
+          s_pbase[i - i0] = np;
+          s_nlist_batch = i - i0;
         }
-        for (int c = lane; c < 256; c += 32) s_re[ew][c] = all ? c : (c < n ? cand[c] : 0);
-        __syncwarp();
-        exact_logits_warp(a.x + static_cast<size_t>(tt) * a.K, a.wr, a.offset, a.K, s_re[ew], n,
-                          s_rl[ew]);
-        refine_select(s_rl[ew], s_re[ew], n, a.bias, a.k, a.gate, a.renorm, all, 0, nullptr,
-                      a.topk_idx + static_cast<size_t>(tt) * a.k,
-                      a.topk_w + static_cast<size_t>(tt) * a.k, s_sel + r, 128);
-        __syncwarp();
+        epi_bar();
+        const int nb = s_nlist_batch;
+        for (int q = et; q < s_pbase[nb]; q += 128) {
+          int i = 0;
+          while (s_pbase[i + 1] <= q) ++i;
+          const int* cand = s_cand + (i0 + i) * kRefineCand;
+          const int c = q - s_pbase[i];
+          s_pt[q] = b * a.tpc + s_list[i0 + i];
+          s_pe[q] = cand[0] == -2 ? c : cand[c];
+        }
+        epi_bar();
+        exact_pair_logits(a.x, a.wr, a.offset, a.K, s_pt, s_pe, s_pbase[nb], s_pl, ew, 4);
+        epi_bar();
+        for (int i = ew; i < nb; i += 4) {
+          const int r = s_list[i0 + i];
+          const int tt = b * a.tpc + r;
+          const bool all = s_cand[(i0 + i) * kRefineCand] == -2;
+          refine_select(s_pl + s_pbase[i], s_pe + s_pbase[i], s_pbase[i + 1] - s_pbase[i],
+                        a.bias, a.k, a.gate, a.renorm, all, 0, nullptr,
+                        a.topk_idx + static_cast<size_t>(tt) * a.k,
+                        a.topk_w + static_cast<size_t>(tt) * a.k, s_sel + r, 128);
+        }
+        epi_bar();
+        i0 += nb;
       }
-      epi_bar();
       // ranks inside the block: one bit per (expert, token)
       if (valid)
         for (int j = 0; j < a.k; ++j) atomicOr(&s_masks[sel[j * 128]][row >> 5], 1u << (row & 31));
@@ -1005,32 +1032,91 @@ router_pair_kernel(const __grid_constant__ CUtensorMap tmX,
     __threadfence();
     int* sb = reinterpret_cast<int*>(smem);   // the stage ring is idle now
     const int n = a.nblk * E;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) sb[i] = __ldcg(a.blk + i);
+    // 16-byte loads, eight in flight per thread (E a multiple of 4; the
+    // block counts start 256-byte aligned), then the rest one by one
+    const int n4 = E % 4 == 0 ? n / 4 : 0;
+    const int4* g4 = reinterpret_cast<const int4*>(a.blk);
+    int4* s4 = reinterpret_cast<int4*>(sb);
+    for (int i0 = threadIdx.x; i0 < n4; i0 += 8 * blockDim.x) {
+      int4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n4) v[u] = __ldcg(g4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n4) s4[i] = v[u];
+      }
+    }
+    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) sb[i] = __ldcg(a.blk + i);
     __syncthreads();
     if (threadIdx.x < E) {
-      const int e = threadIdx.x;
-      int run = 0;
-      for (int bb = 0; bb < a.nblk; ++bb) {
-        const int c = sb[bb * E + e];
-        sb[bb * E + e] = run;
-        run += c;
-      }
-      s_cnt[e] = run;
-      a.counts[e] = run;
+      // running sums over the blocks of expert e, four segments of blocks
+      // in flight at once
+      const int e = threadIdx.x, nb = a.nblk, seg = (nb + 3) / 4;
+      int sum[4] = {0, 0, 0, 0};
+      for (int j = 0; j < seg; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int bb = q * seg + j;
+          if (bb < nb) sum[q] += sb[bb * E + e];
+        }
+      int base[4] = {0, sum[0], sum[0] + sum[1], sum[0] + sum[1] + sum[2]};
+      for (int j = 0; j < seg; ++j)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int bb = q * seg + j;
+          if (bb < nb) {
+            const int c = sb[bb * E + e];
+            sb[bb * E + e] = base[q];
+            base[q] += c;
+          }
+        }
+      const int total = sum[0] + sum[1] + sum[2] + sum[3];
+      s_cnt[e] = total;
+      a.counts[e] = total;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int run = 0;
-      for (int e = 0; e < E; ++e) {
-        const int c = s_cnt[e];
-        s_cnt[e] = run;
-        a.offsets[e] = run;
-        run += c;
+    if (warp == 0) {
+      // exclusive prefix over the experts: eight consecutive experts per lane
+      int v[8], loc = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane * 8 + j;
+        v[j] = e < E ? s_cnt[e] : 0;
+        loc += v[j];
       }
-      a.offsets[E] = run;
+      int incl = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int run = incl - loc;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane * 8 + j;
+        if (e < E) {
+          s_cnt[e] = run;
+          a.offsets[e] = run;
+        }
+        run += v[j];
+      }
+      if (lane == 31) a.offsets[E] = incl;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) a.blk[i] = sb[i] + s_cnt[i % E];
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+      const int e0 = (4 * i) % E;
+      int4 v = s4[i];
+      v.x += s_cnt[e0];
+      v.y += s_cnt[e0 + 1];
+      v.z += s_cnt[e0 + 2];
+      v.w += s_cnt[e0 + 3];
+      reinterpret_cast<int4*>(a.blk)[i] = v;
+    }
+    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) a.blk[i] = sb[i] + s_cnt[i % E];
   }
   __syncthreads();
   cluster_sync_all();          // neither CTA leaves while the other still uses the pair

@@ -202,11 +202,28 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for an MN-major bf16 tile with the
+// 128-byte swizzle: the layout TMA tile loads with a 64-element inner box
+// along M/N write, one box per 64 M/N elements.  Inside a box each 128-byte
+// row holds 64 consecutive M/N elements of one k, eight rows (k) form a
+// 1024-byte swizzle atom, so the stride between 8-row groups along K is 1024
+// bytes (stride-dimension offset) and the stride between the 64-element
+// boxes along M/N is `box_bytes` (leading-dimension offset).
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t box_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((box_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B (format 1), f32 accumulator
-// (format 1), both K-major, dense, no negation; N >> 3 at bit 17, M >> 4 at
-// bit 24.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) |
+// (format 1), dense, no negation; N >> 3 at bit 17, M >> 4 at bit 24.  A and
+// B are K-major unless b_mn (bit 16: B is MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn ? (1u << 16) : 0u) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -238,6 +255,20 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];"
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32_rank0(bar)),
         "r"(x), "r"(y)
+      : "memory");
+}
+// Four rows gathered from a 2-D tensor (box 64 elements x 1 row) into four
+// consecutive 128-byte rows of this CTA's shared memory (512 bytes at dst),
+// completion counted on the pair's rank-0 barrier.  x is the inner
+// coordinate (element), r0..r3 the rows.  No multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                                 int32_t x, int32_t r0, int32_t r1, int32_t r2,
+                                                 int32_t r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32_rank0(bar)),
+        "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
 // Arrive on the rank-0 copy of a barrier.

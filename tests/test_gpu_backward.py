@@ -40,12 +40,15 @@ def _np(t):
     return t.detach().float().cpu().numpy()
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_backward_small_elementwise(name):
+@pytest.mark.parametrize("name,gather", [(n, False) for n in SMALL] +
+                         [("qwen3_small", True), ("skew_small", True)])
+def test_backward_small_elementwise(name, gather):
+    """gather: the forward ran with gathered gate/up rows (no permuted copy
+    of x kept); the backward gathers x's rows itself."""
     shape = SMALL[name]
     host = I.make_inputs(shape)
     layer = MoELayer(shape, host)
-    layer.forward()
+    layer.forward(gather_rows=gather)
     dout_h = I.round_to_bf16(np.random.default_rng(77).standard_normal(
         (shape.T, shape.d_model)).astype(np.float32))
     g = layer.backward(to_device(dout_h, torch.bfloat16, "cuda"))

@@ -116,11 +116,12 @@ def test_forward_full_size_every_token(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", ["page2_small", "qwen3_small", "skew_small"])
+@pytest.mark.parametrize("name", ["page2_small", "qwen3_small", "skew_small", "qwen3_30b"])
 def test_forward_with_gathered_gate_up_rows(name):
     """The alternative expert path (moe_forward_ex, gather_rows = 1) that
-    skips the permuted copy of x and gathers the gate/up GEMM's rows from x."""
-    shape = SMALL[name]
+    skips the permuted copy of x and gathers the gate/up GEMM's rows from x
+    (small shapes, and the full qwen3_30b workload on every token)."""
+    shape = SMALL[name] if name in SMALL else I.WORKLOADS[name]
     host = I.make_inputs(shape)
     layer = MoELayer(shape, host)
     layer.forward(gather_rows=True)
