@@ -15,9 +15,6 @@
 //            exclusive scan over experts (offsets).
 //   scatter  one warp per token: final row = base + rank, x row read once
 //            and written to its k rows with 16-byte vector accesses.
-// The forward's fused router (router_topk_pair) produces the ranks and block
-// counts itself, over blocks of its own size, and usually the scan as well;
-// the scatter then takes that block size.
 // Pairs with an expert id outside [0, E), or repeating an expert the token
 // already chose, are skipped (row -1) and flagged in the status word.
 #include <cuda_runtime.h>

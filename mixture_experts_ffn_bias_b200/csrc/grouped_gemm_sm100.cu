@@ -79,6 +79,9 @@ struct GemmArgs {
   int x_ldc;
   int gather_limit;            // GATHER: entries of gather_rows
   int gather_src_rows;         // GATHER: rows of gather_src
+  // GATHER: when set and zero on the device, the rows are read in tiles from
+  // the permuted copy (map tmA2, no extra group) instead of gathered
+  const uint32_t* gather_flag;
 };
 
 // Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
@@ -245,6 +248,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr uint32_t IDESC = idesc_bf16_f32(BM2, Cfg::N_MMA, BMN);
   constexpr int BOX_MN = 64 * 128;   // PLAIN_BMN: one 64-column box of 64 k-rows
 
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -323,6 +327,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     int stage = 0;
     uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
     bool ok = true;
+    const bool copy_a = GATHER && args.gather_flag != nullptr && __ldg(args.gather_flag) == 0u;
     // without gathers lane 0 alone drives the ring
     for (int tile = pair; tile < total_tiles && ok && (GATHER || lane == 0); tile += npairs) {
       const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
@@ -331,10 +336,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const int gbase = pt.x ? 0 : g * args.n_per_group;
       const int brow = SWIGLU ? gbase + n * BN_OUT
                               : gbase + n * BN_OUT + static_cast<int>(rank) * (BN_ACC / 2);
-      const CUtensorMap* ma = pt.x ? &tmA2 : &tmA;
+      const CUtensorMap* ma = (pt.x || copy_a) ? &tmA2 : &tmA;
       const CUtensorMap* mb = (SWIGLU && rank == 1) ? (pt.x ? &tmB1_2 : &tmB1)
                                                     : (pt.x ? &tmB0_2 : &tmB0);
-      const bool gathered = GATHER && !pt.x;
+      const bool gathered = GATHER && !pt.x && !copy_a;
       int tok[4] = {0, 0, 0, 0};
       if (gathered) {
 #pragma unroll
@@ -436,7 +441,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
-    const int row = q * 32 + lane;
     int it = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
       const int acc = it % NACC;
@@ -447,14 +451,16 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
       const int rows_g = pt.rows, n = pt.n;
       const int r0 = pt.m * BM2 + static_cast<int>(rank) * BM;   // first row (in group) of this CTA
-      const bool valid = (r0 + row) < rows_g;
+      const bool valid = (r0 + q * 32 + lane) < rows_g;
       const bool warp_full = (r0 + q * 32 + 32) <= rows_g;
       const int warp_row0 = pt.row0 + r0 + q * 32;
       uint8_t* stage_buf = smemEpi + (warp - 2) * (32 * 128);
       const CUtensorMap* mc = pt.x ? &tmC2 : &tmC;
       __nv_bfloat16* cbase = static_cast<__nv_bfloat16*>(pt.x ? args.x_C : args.C);
-      const size_t crow_off = static_cast<size_t>(pt.row0 + r0 + row) * (pt.x ? args.x_ldc : args.ldc);
+      const size_t crow_off =
+          static_cast<size_t>(warp_row0 + lane) * (pt.x ? args.x_ldc : args.ldc);
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
+      constexpr int UP = Cfg::N_MMA / 2;   // up columns follow the gate columns
 #pragma unroll 1
       for (int cb = 0; cb < BN_OUT / 64; ++cb) {
         // accumulator column of this 64-column chunk and its output column:
@@ -480,7 +486,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           uint32_t v[32];
           if (SWIGLU) {
             uint32_t u[32];
-            constexpr int UP = Cfg::N_MMA / 2;   // up columns follow the gate columns
             tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
             tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
             tmem_ld16(t_addr + UP + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
@@ -640,7 +645,7 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
       !make_map(&tb1, W3, b_rows, K, bh) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0};
+                0, 0, 0, nullptr, 0, 0, 0, nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, bh) ||
@@ -656,8 +661,8 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
     xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
   }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
-  return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args, rows_upper,
-                                            stream);
+  return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
+                                            rows_upper, stream);
 }
 
 // Gate/up pass whose A rows are gathered from X [x_rows, K]: output row r
@@ -675,7 +680,7 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
       !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, R, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows), nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, 128) ||
@@ -690,27 +695,36 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
   } else {
     xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
   }
-  return launch_pair<256, MODE_SWIGLU_BF16, true>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
-                                                  static_cast<int>(R), stream);
+  return launch_pair<256, MODE_SWIGLU_BF16, true>(ta, tb0, tb1, tc, xa, xb0, xb1, xc,
+                                                  args, static_cast<int>(R), stream);
 }
 
 // Y[r] = X[rows[r]] W[g]^T for the expert-contiguous rows r < R (A rows
-// gathered from X [x_rows, K] as above); Y is [R, N].
+// gathered from X [x_rows, K] as above); Y is [R, N].  When x_perm [R, K]
+// and flag are given, the kernel reads the flag on the device: zero means
+// x_perm holds the permuted rows, which are then read in tiles instead.
 cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
                                      const int32_t* offsets, int num_groups, const void* W, int N,
-                                     int K, void* Y, uint32_t* status, cudaStream_t stream) {
-  CUtensorMap ta, tb, tc;
+                                     int K, void* Y, uint32_t* status, cudaStream_t stream,
+                                     const void* x_perm, const uint32_t* flag) {
+  CUtensorMap ta, tb, tc, tp;
   const int64_t b_rows = static_cast<int64_t>(num_groups) * N;
   const int bn = (N % 256 == 0) ? 256 : 128;
   if (!make_map(&ta, X, x_rows, K, 1) || !make_map(&tb, W, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, R, N, 32))
     return cudaErrorInvalidValue;
+  if (x_perm != nullptr && flag != nullptr) {
+    if (!make_map(&tp, x_perm, R, K, BM)) return cudaErrorInvalidValue;
+  } else {
+    tp = ta;
+    flag = nullptr;
+  }
   GemmArgs args{offsets, num_groups, 0, N, K, Y, N, status, rows, X, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows), flag};
   if (bn == 256)
-    return launch_pair<256, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, ta, tb, tb, tc, args,
+    return launch_pair<256, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, tp, tb, tb, tc, args,
                                                    static_cast<int>(R), stream);
-  return launch_pair<128, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, ta, tb, tb, tc, args,
+  return launch_pair<128, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, tp, tb, tb, tc, args,
                                                  static_cast<int>(R), stream);
 }
 
@@ -733,7 +747,7 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0};
+                0, 0, 0, nullptr, 0, 0, 0, nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (extra->n != N || !make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb, extra->B0, N, extra->K, bn / 2) ||
@@ -749,13 +763,13 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (bn == 512)
-    return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
-                                             stream);
+    return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                             rows_upper, stream);
   if (bn == 256)
-    return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
-                                             stream);
-  return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args, rows_upper,
-                                           stream);
+    return launch_pair<256, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                             rows_upper, stream);
+  return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                           rows_upper, stream);
 }
 
 // Y[r] = A[r] B_g with B_g stored [K, N] (MN-major): its first b0_rows rows
@@ -776,16 +790,16 @@ cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* 
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
-                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0};
+                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (N % 512 == 0 && K >= 4096)
-    return launch_pair<512, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
-                                            stream);
+    return launch_pair<512, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args,
+                                            rows_upper, stream);
   if (N % 256 == 0)
-    return launch_pair<256, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
-                                            stream);
-  return launch_pair<128, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args, rows_upper,
-                                          stream);
+    return launch_pair<256, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args,
+                                            rows_upper, stream);
+  return launch_pair<128, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args,
+                                          rows_upper, stream);
 }
 
 }  // namespace moe

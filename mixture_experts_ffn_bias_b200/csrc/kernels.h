@@ -48,21 +48,6 @@ cudaError_t router_topk_tc(const void* x, int T, const void* w_router, int E, in
                            cudaStream_t stream);
 cudaError_t router_logits_tc(const void* x, int T, const void* w_router, int E, int K,
                              float* logits, uint32_t* status, cudaStream_t stream);
-// Fused router on CTA pairs (E <= 128, k <= 8): logits, selection, exact
-// re-decision of near ties inside the kernel, and the dispatch's per-block
-// ranks (rank_out [T, k]) and counts (blk [router_pair_blocks(T), E], blocks
-// of router_pair_block_tokens(T) tokens).  When *scan_fused comes back true
-// the last CTA has also turned blk into block bases and written counts and
-// offsets; otherwise dispatch_scan must follow.  done: a zeroed counter.
-constexpr int kRouterPairs = 74;   // CTA pairs the token tiles are sized for
-int router_pair_block_tokens(int T);
-int router_pair_blocks(int T);
-cudaError_t router_topk_pair(const void* x, int T, const void* w_router, int E, int K,
-                             const float* logit_offset, const float* sel_bias, int k, int gate,
-                             int renorm, int32_t* topk_idx, float* topk_w, int32_t* rank_out,
-                             int32_t* blk, int32_t* counts, int32_t* offsets,
-                             int32_t* refine_count, uint32_t* status, uint32_t* done,
-                             bool* scan_fused, cudaStream_t stream);
 cudaError_t router_select_fast(const float* logits, const float* logit_offset,
                                const float* sel_bias, int T, int E, int k, int gate, int renorm,
                                const KeyOpts& ko, int32_t* topk_idx, float* topk_w,
@@ -128,9 +113,13 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
                                               const GemmExtraGroup* extra = nullptr);
 // Y[r] = X[rows[r]] W[g]^T over the expert-contiguous rows r < R (A rows
 // gathered from X by the permutation; no permuted copy).
+// With x_perm [R, K] and flag: a zero flag on the device means x_perm holds
+// the permuted rows, read in tiles instead of gathered.
 cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
                                      const int32_t* offsets, int num_groups, const void* W, int N,
-                                     int K, void* Y, uint32_t* status, cudaStream_t stream);
+                                     int K, void* Y, uint32_t* status, cudaStream_t stream,
+                                     const void* x_perm = nullptr,
+                                     const uint32_t* flag = nullptr);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream,

@@ -15,8 +15,8 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
-  size_t status, blk, offsets, counts, slot_pos, perm_src, refine, refine_cand, stats, logits,
-      x_perm, h, y_perm, h_sh, y_sh, total;
+  size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, stats, logits, x_perm, h,
+      y_perm, h_sh, y_sh, total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -28,15 +28,10 @@ Layout layout(const moe_config& c) {
   Layout L{};
   size_t o = 0;
   // status area: word 0 device status, word 1 tokens re-decided by the
-  // router, word 2 the fused router's finished-CTA counter
-  L.status = o;   o += up(4 * sizeof(uint32_t));
-  // block counts: the rank kernel's blocks or the fused router's, whichever
-  // are more
-  const int nblk = moe::rank_blocks(c.T) > moe::router_pair_blocks(c.T)
-                       ? moe::rank_blocks(c.T) : moe::router_pair_blocks(c.T);
-  L.blk = o;      o += up(static_cast<size_t>(nblk) * E * 4);
+  // router
+  L.status = o;   o += up(3 * sizeof(uint32_t));
+  L.blk = o;      o += up(static_cast<size_t>(moe::rank_blocks(c.T)) * E * 4);
   L.offsets = o;  o += up((E + 1) * 4);
-  L.counts = o;   o += up(E * 4);
   L.slot_pos = o; o += up(R * 4);
   L.perm_src = o; o += up(R * 4);
   L.refine = o;   o += up(T * 4);
@@ -95,9 +90,10 @@ inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
   } while (0)
 
 // Word 0: device status flags; word 1: number of tokens the router listed
-// for exact re-decision; word 2: CTAs of the fused router that finished.
+// for exact re-decision; word 2: non-zero when the last forward kept no
+// permuted copy of x (gathered gate/up rows).
 moe_status clear_status(void* ws, cudaStream_t s) {
-  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, 4 * sizeof(uint32_t), s));
+  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, 3 * sizeof(uint32_t), s));
   return MOE_OK;
 }
 
@@ -108,38 +104,12 @@ int device_sms() {
   return n > 0 ? n : 148;
 }
 
-// What the router left for the dispatch: nothing, or (fused pair router) the
-// ranks in slot_pos and the block counts, and maybe the scan as well.
-struct RouterDispatch {
-  bool ranked = false;       // slot_pos holds ranks, blk the block counts
-  bool scanned = false;      // blk holds block bases; counts and offsets written
-  int blk_tokens = 0;        // tokens per block
-};
-
-// Router into caller buffers; logits scratch in ws.  counts: where the fused
-// router's scan writes the per-expert counts (ws scratch when null).
+// Router into caller buffers; logits scratch in ws.
 moe_status run_router(const moe_config* c, const void* x, const void* w_router,
                       const float* sel_bias, const float* logit_offset, int32_t* topk_idx,
                       float* topk_w, void* ws, cudaStream_t s,
-                      const moe::KeyOpts& ko = moe::KeyOpts{}, int32_t* counts = nullptr,
-                      RouterDispatch* rd = nullptr) {
+                      const moe::KeyOpts& ko = moe::KeyOpts{}) {
   const Layout L = layout(*c);
-  if (c->dtype == MOE_BF16 && ko.is_default() &&
-      moe::router_fused_supported(c->n_experts, c->top_k)) {
-    bool scanned = false;
-    MOE_TRY(moe::router_topk_pair(
-        x, c->T, w_router, c->n_experts, c->d_model, logit_offset, sel_bias, c->top_k, c->gate,
-        c->norm_topk_prob, topk_idx, topk_w, at<int32_t>(ws, L.slot_pos), at<int32_t>(ws, L.blk),
-        counts ? counts : at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
-        at<int32_t>(ws, L.status) + 1, at<uint32_t>(ws, L.status), at<uint32_t>(ws, L.status) + 2,
-        &scanned, s));
-    if (rd) {
-      rd->ranked = true;
-      rd->scanned = scanned;
-      rd->blk_tokens = moe::router_pair_block_tokens(c->T);
-    }
-    return MOE_OK;
-  }
   if (c->dtype == MOE_BF16) {
     float* logits = at<float>(ws, L.logits);
     int32_t* count = at<int32_t>(ws, L.status) + 1;
@@ -297,9 +267,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   const Marks mk{events, s};
   if ((st = clear_status(ws, s)) != MOE_OK) return st;
   if (!mk.rec(0)) return MOE_ERR_CUDA;
-  RouterDispatch rd;
-  if ((st = run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, s,
-                       moe::KeyOpts{}, counts, &rd)) != MOE_OK)
+  if ((st = run_router(cfg, x, w_router, sel_bias, logit_offset, topk_idx, topk_w, ws, s)) !=
+      MOE_OK)
     return st;
   if (!mk.rec(1)) return MOE_ERR_CUDA;
   int32_t* offsets = at<int32_t>(ws, L.offsets);
@@ -313,23 +282,10 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   // less memory but measured slower on B200 (each of an m-tile's n-tile CTAs
   // gathers the same rows again).
   int32_t* perm_src = at<int32_t>(ws, L.perm_src);
-  if (rd.ranked) {
-    // the fused router ranked every pair inside its block (and usually
-    // scanned the block counts): only the scan (if left) and the scatter
-    int32_t* blk = at<int32_t>(ws, L.blk);
-    if (!rd.scanned)
-      MOE_TRY(moe::dispatch_scan(blk, moe::router_pair_blocks(cfg->T), cfg->n_experts, counts,
-                                 offsets, s));
-    if (gather)
-      MOE_TRY(moe::dispatch_positions(topk_idx, blk, slot_pos, perm_src, cfg->T, cfg->top_k,
-                                      cfg->n_experts, rd.blk_tokens, s));
-    else
-      MOE_TRY(moe::dispatch_scatter(true, x, topk_idx, blk, slot_pos, perm_src, x_perm, cfg->T,
-                                    cfg->d_model, cfg->top_k, cfg->n_experts, rd.blk_tokens, s));
-  } else if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
-                               gather ? nullptr : x_perm, ws, s)) != MOE_OK) {
+  if (gather) MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, L.status) + 2, 0xff, sizeof(uint32_t), s));
+  if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
+                        gather ? nullptr : x_perm, ws, s)) != MOE_OK)
     return st;
-  }
   if (!mk.rec(2)) return MOE_ERR_CUDA;
   if ((st = run_experts(cfg, gather ? nullptr : x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk,
                         perm_src)) != MOE_OK)
@@ -389,7 +345,8 @@ BLayout blayout(const moe_config& c) {
 }
 
 // The layer's backward (bf16 layers).  fws holds the state of the forward:
-// offsets, slot_pos, perm_src, h, y_perm (and h_sh).
+// offsets, slot_pos, perm_src, x_perm (unless that forward gathered its rows:
+// status word 2), h, y_perm (and h_sh).
 moe_status backward_impl(const moe_config* c, const void* x, const void* w_router,
                          const float* logit_offset, const moe_expert_weights* w,
                          const int32_t* topk_idx, const float* topk_w, const void* dout,
@@ -413,12 +370,15 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
   // weights of dH and dX are read MN-major in place (no transposed copies).
   MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dy), R, offsets, E, 0, w->w2, nullptr, d,
                                      F, d, at<void>(bws, B.dh), status, s));
-  // G and U recomputed from x's rows gathered by the permutation (the
-  // forward may not have kept a permuted copy of x)
+  // G and U recomputed from the forward's permuted copy of x, or, when that
+  // forward gathered its rows instead (status word 2 set), from x's rows
+  // gathered by the permutation
+  const void* x_perm = at<void>(fws, L.x_perm);
+  const uint32_t* no_xperm = at<uint32_t>(fws, L.status) + 2;
   MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w1, F, d,
-                                        at<void>(bws, B.gb), status, s));
+                                        at<void>(bws, B.gb), status, s, x_perm, no_xperm));
   MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w3, F, d,
-                                        at<void>(bws, B.ub), status, s));
+                                        at<void>(bws, B.ub), status, s, x_perm, no_xperm));
   MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.gb), at<void>(bws, B.ub), at<void>(bws, B.dh),
                           at<void>(bws, B.dgu), R, F, s));
   MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, w->w1, w->w3, F, d,

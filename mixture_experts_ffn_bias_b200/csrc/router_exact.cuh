@@ -1,6 +1,5 @@
 // Exact re-decision of a router token whose fp32 selection keys hold a near
-// tie (two of its top-(k+1) keys closer than the router's margin), shared by
-// the separate refine kernel and the fused CTA-pair router.
+// tie (two of its top-(k+1) keys closer than the router's margin).
 //
 // The experts to decide over are the token's candidates (every expert whose
 // fp32 key was within the margin of its (k+1)-th pick, which must contain the
@@ -19,13 +18,10 @@ namespace {
 constexpr int kMaxPerLane = 8;   // E <= 256 = 8 x 32
 
 // Decision on exact logits s_l[0..n) of experts s_e[0..n) (shared memory),
-// written to idx_row / w_row (and, when sel_out is set, the picked ids to
-// sel_out[j * sel_stride]).
-__device__ __noinline__ void refine_select(const double* s_l, const int* s_e, int n,
-                                           const float* bias, int k, int gate, int renorm,
-                                           bool all_experts, int space, const float* noise_row,
-                                           int32_t* idx_row, float* w_row,
-                                           int* sel_out = nullptr, int sel_stride = 0) {
+// written to idx_row / w_row.
+__device__ void refine_select(const double* s_l, const int* s_e, int n, const float* bias,
+                              int k, int gate, int renorm, bool all_experts, int space,
+                              const float* noise_row, int32_t* idx_row, float* w_row) {
   const int lane = threadIdx.x & 31;
   double key[kMaxPerLane];
   float lf[kMaxPerLane];
@@ -127,68 +123,9 @@ __device__ __noinline__ void refine_select(const double* s_l, const int* s_e, in
   if (lane < k) {
     idx_row[lane] = my_idx;
     w_row[lane] = renorm ? my_s / (ssum + 1e-9f) : my_s;
-    if (sel_out) sel_out[lane * sel_stride] = my_idx;
   }
 }
 
-
-// Exact logits of a batch of (token, expert) pairs, all the listed tokens of
-// a block at once: pair p is token row x + s_pt[p] * d and router row
-// s_pe[p]; s_pl[p] = fp64 sum of the exact bf16 x bf16 products (+
-// offset[e]).  Warp `first` of `step` warps takes pairs first, first + step,
-// ..., two at a time, with the 16-byte loads of four column steps of both
-// pairs issued before they are used: the rows come from L2, so the time is
-// load latency, and one round of it covers up to 512 columns of two pairs.
-__device__ __noinline__ void exact_pair_logits(const __nv_bfloat16* __restrict__ x,
-                                               const __nv_bfloat16* __restrict__ wr,
-                                               const float* __restrict__ offset, int d,
-                                               const int* s_pt, const int* s_pe, int npairs,
-                                               double* s_pl, int first, int step) {
-  const int lane = threadIdx.x & 31;
-  for (int p0 = first; p0 < npairs; p0 += 2 * step) {
-    const int p1 = p0 + step < npairs ? p0 + step : p0;
-    const uint4* xa = reinterpret_cast<const uint4*>(x + static_cast<size_t>(s_pt[p0]) * d);
-    const uint4* xb = reinterpret_cast<const uint4*>(x + static_cast<size_t>(s_pt[p1]) * d);
-    const uint4* wa = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(s_pe[p0]) * d);
-    const uint4* wb = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(s_pe[p1]) * d);
-    double sa = 0.0, sb = 0.0;
-    const int nv = d / 8;   // 16-byte pieces per row
-    for (int v0 = lane; v0 < nv; v0 += 4 * 32) {
-      uint4 ux[4], uw[4], vx[4], vw[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + 32 * u;
-        const bool in = v < nv;
-        ux[u] = in ? __ldg(xa + v) : make_uint4(0u, 0u, 0u, 0u);
-        uw[u] = in ? __ldg(wa + v) : make_uint4(0u, 0u, 0u, 0u);
-        vx[u] = in ? __ldg(xb + v) : make_uint4(0u, 0u, 0u, 0u);
-        vw[u] = in ? __ldg(wb + v) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const __nv_bfloat16* hx = reinterpret_cast<const __nv_bfloat16*>(&ux[u]);
-        const __nv_bfloat16* hw = reinterpret_cast<const __nv_bfloat16*>(&uw[u]);
-        const __nv_bfloat16* gx = reinterpret_cast<const __nv_bfloat16*>(&vx[u]);
-        const __nv_bfloat16* gw = reinterpret_cast<const __nv_bfloat16*>(&vw[u]);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {   // exact fp32 products, fp64 sums
-          sa += static_cast<double>(__bfloat162float(hw[j]) * __bfloat162float(hx[j]));
-          sb += static_cast<double>(__bfloat162float(gw[j]) * __bfloat162float(gx[j]));
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sa += __shfl_xor_sync(0xffffffffu, sa, o);
-      sb += __shfl_xor_sync(0xffffffffu, sb, o);
-    }
-    if (lane == 0) {
-      s_pl[p0] = sa + (offset ? static_cast<double>(offset[s_pe[p0]]) : 0.0);
-      if (p1 != p0) s_pl[p1] = sb + (offset ? static_cast<double>(offset[s_pe[p1]]) : 0.0);
-    }
-  }
-  __syncwarp();
-}
 
 }  // namespace
 }  // namespace moe

@@ -37,7 +37,6 @@
 
 #include "kernels.h"
 #include "launch.cuh"
-#include "router_exact.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -83,18 +82,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;"
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
-        "r"(x), "r"(y), "l"(policy)
-      : "memory");
-}
-
-// tma_load_2d_pair with an L2 eviction-priority policy.
-__device__ __forceinline__ void tma_load_2d_pair_hint(void* dst, const CUtensorMap* map,
-                                                      uint64_t* bar, int32_t x, int32_t y,
-                                                      uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;"
-      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32_rank0(bar)),
         "r"(x), "r"(y), "l"(policy)
       : "memory");
 }
@@ -530,712 +517,7 @@ bool maps(const void* x, int T, const void* w_router, int E, int K, CUtensorMap*
   return map2d(mx, x, T, K, RBM) && map2d(mw, w_router, E, K, npad_for(E));
 }
 
-
-// ============================================================================
-// Fused router on CTA pairs: logits, selection, exact re-decision of near
-// ties, and the per-block ranks and counts of the dispatch, in one kernel.
-//
-// A pair of CTAs (cluster of two) takes a tile of 2 * tpc tokens; tpc <= 128
-// tokens per CTA is chosen on the host so that the tiles fill the pairs of
-// the GPU in whole waves.  tcgen05.mma.cta_group::2 with M = 256, N = NMMA:
-// CTA r holds rows [0, tpc) of its own 128-row A tile (its tokens; the rows
-// past tpc are never read out) and the router rows [r NMMA/2, (r+1) NMMA/2),
-// so every SM streams only its own tokens and half of the router weight.
-// Each 128-wide K chunk accumulates in a fresh TMEM slot; the epilogue thread
-// of a token adds the chunks in fp32 registers.  After a tile's logits:
-//   1. select: each token's thread forms keys = logit + bias and picks the
-//      top-(k+1) (descending, ties to the lower id), or lists the token with
-//      its candidate experts when two of those keys lie within the margin;
-//   2. exact re-decision of the listed tokens on fp64 logit sums, one
-//      epilogue warp per token (router_exact.cuh);
-//   3. ranks: a bitmask per expert over the CTA's tokens; a pair's rank in
-//      its block is a popcount, written to rank_out; the block's count per
-//      expert goes to blk[b, e] (b = block of tpc tokens).
-// The last CTA to finish (a counter in the status area, zeroed by every
-// call) turns the block counts into block bases, counts and offsets (the
-// dispatch scan), so the kernel after this one is the row scatter.
-// Warp roles: warp 0 TMA producer, warp 1 TMEM owner and (rank 0) MMA
-// issuer, warps 2-5 epilogue.  No load uses cluster multicast.
-constexpr int PR_LIST_MAX = 128;
-constexpr int PR_PAIRS_MAX = 512;   // (token, candidate) pairs re-decided per batch
-
-struct PairRouterArgs {
-  const __nv_bfloat16* x;     // [T, K] (exact re-decision reads its rows)
-  const __nv_bfloat16* wr;    // [E, K]
-  const float* offset;        // [E] or null
-  const float* bias;          // [E] or null
-  int T, K, E, k, gate, renorm;
-  int tpc, ntiles, nblk, fuse_scan;
-  int32_t* topk_idx;          // [T, k]
-  float* topk_w;              // [T, k]
-  int32_t* rank_out;          // [T, k] rank of each pair inside its block
-  int32_t* blk;               // [nblk, E] counts; bases when the scan is fused
-  int32_t* counts;            // [E]      (fused scan)
-  int32_t* offsets;           // [E + 1]  (fused scan)
-  int32_t* refine_count;      // tokens re-decided (diagnostic)
-  uint32_t* status;
-  uint32_t* done;             // CTAs finished (zero at launch)
-};
-
-template <int NSEL>
-struct PCfg {
-  static constexpr int NMMA = NSEL < 64 ? 64 : NSEL;
-  static constexpr int A_BYTES = 128 * RBK * 2;
-  static constexpr int B_BYTES = (NMMA / 2) * RBK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int LOGIT_BYTES = NSEL * 128 * 4;
-  static constexpr int STAGE_BUDGET = 190464 - LOGIT_BYTES;   // 186 KB of dynamic smem
-  static constexpr int STAGES =
-      (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
-  static constexpr int NSLOT = (512 / NMMA) > 8 ? 8 : (512 / NMMA);
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LOGIT_BYTES + 1024 + 1024;
-  static constexpr int SCAN_INTS = STAGES * STAGE_BYTES / 4;   // fused-scan staging
-  static_assert(NSLOT * NMMA <= TMEM_COLS, "TMEM slots");
-};
-
-__device__ __forceinline__ void epi_bar() {
-  asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-// Selection of one token from its fp32 logits (fused path).  acc[i] holds
-// the logit of expert i (+ offset); the logits are kept in the thread's
-// shared-memory column s_log[i * 128].  Picks go to s_sel[j * 128] (j <= k).
-// Returns true when the token was decided here; false when it holds a near
-// tie: then it is appended to the CTA's list with its candidate experts.
-template <int COLS>
-__device__ __forceinline__ bool pair_route_row(float (&acc)[COLS], float* s_log, int* s_sel,
-                                               const float* s_off, const float* s_bias, int E,
-                                               int t, int row, const PairRouterArgs& a,
-                                               int* s_nlist, int* s_list, int* s_cand) {
-  float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-  for (int i = 0; i < COLS; i += 4) {
-    const float4 f = *reinterpret_cast<const float4*>(s_off + i);
-    const float ov[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float l = i + q < E ? acc[i + q] + ov[q] : -INFINITY;
-      acc[i + q] = l;
-      mx[q] = fmaxf(mx[q], l);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < COLS; ++i) s_log[i * 128] = acc[i];
-#pragma unroll
-  for (int i = 0; i < COLS; i += 4) {
-    const float4 f = *reinterpret_cast<const float4*>(s_bias + i);
-    const float bv[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) acc[i + q] = i + q < E ? acc[i + q] + bv[q] : -INFINITY;
-  }
-  const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-  float S = 1.0f;
-  if (a.gate == 0 && !a.renorm) {
-    float sp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-    for (int i = 0; i < COLS; i += 4) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sp[q] += expf(s_log[(i + q) * 128] - m);
-    }
-    S = (sp[0] + sp[1]) + (sp[2] + sp[3]);
-  }
-  constexpr int GS = COLS >= 64 ? 8 : 4;
-  constexpr int NG = COLS / GS;
-  constexpr int NONE = 0x7fffffff;
-  float gv[NG];
-  int gi[NG];
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    gv[g] = acc[g * GS];
-    gi[g] = g * GS;
-#pragma unroll
-    for (int s = 1; s < GS; ++s) {
-      const bool take = acc[g * GS + s] > gv[g];
-      gv[g] = take ? acc[g * GS + s] : gv[g];
-      gi[g] = take ? g * GS + s : gi[g];
-    }
-  }
-  const int rounds = a.k < E ? a.k + 1 : a.k;
-  float pv = INFINITY;
-  int pi = -1;
-  float min_gap = INFINITY;
-#pragma unroll 1
-  for (int j = 0; j < rounds; ++j) {
-    float bv = gv[0];
-    int bi = gi[0], bg = 0;
-#pragma unroll
-    for (int g = 1; g < NG; ++g) {
-      const bool take = (gi[g] != NONE) & ((bi == NONE) | (gv[g] > bv));
-      bv = take ? gv[g] : bv;
-      bi = take ? gi[g] : bi;
-      bg = take ? g : bg;
-    }
-    min_gap = j > 0 ? fminf(min_gap, pv - bv) : min_gap;
-    pv = bv;
-    pi = bi;
-    s_sel[j * 128] = bi;
-    float vv[GS];
-#pragma unroll
-    for (int s = 0; s < GS; ++s) {
-      const int i = bg * GS + s;
-      vv[s] = i < E ? s_log[i * 128] + s_bias[i] : -INFINITY;
-    }
-    float nv = -INFINITY;
-    int ni = NONE;
-#pragma unroll
-    for (int s = 0; s < GS; ++s) {
-      const int i = bg * GS + s;
-      const bool after = (vv[s] < pv) | ((vv[s] == pv) & (i > pi));
-      const bool take = after & ((vv[s] > nv) | (ni == NONE));
-      nv = take ? vv[s] : nv;
-      ni = take ? i : ni;
-    }
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      gv[g] = g == bg ? nv : gv[g];
-      gi[g] = g == bg ? ni : gi[g];
-    }
-  }
-  if (min_gap < kRefineMargin) {
-    const int slot = atomicAdd(s_nlist, 1);   // < 128: one entry per token of the CTA
-    s_list[slot] = row;
-    int* cand = s_cand + slot * kRefineCand;
-    const float lo = pv - kRefineMargin;
-    int n = (a.gate == 0 && !a.renorm) ? kRefineCand + 1 : 0;
-#pragma unroll 1
-    for (int i = 0; i < E; ++i) {
-      if (s_log[i * 128] + s_bias[i] >= lo) {
-        if (n < kRefineCand) cand[n] = i;
-        ++n;
-      }
-    }
-    if (n > kRefineCand) {
-      cand[0] = -2;
-      n = 1;
-    }
-    for (int c = n; c < kRefineCand; ++c) cand[c] = -1;
-    return false;
-  }
-  float sc[KMAX_FUSED];
-  int sid[KMAX_FUSED];
-  float ssum = 0.f;
-#pragma unroll
-  for (int j = 0; j < KMAX_FUSED; ++j) {
-    sc[j] = 0.f;
-    sid[j] = 0;
-    if (j < a.k) {
-      sid[j] = s_sel[j * 128];
-      const float l = s_log[sid[j] * 128];
-      sc[j] = a.gate == 1 ? 1.0f / (1.0f + expf(-l)) : expf(l - m) / S;
-      ssum += sc[j];
-    }
-  }
-  int32_t* irow = a.topk_idx + static_cast<size_t>(t) * a.k;
-  float* wrow = a.topk_w + static_cast<size_t>(t) * a.k;
-#pragma unroll
-  for (int j = 0; j < KMAX_FUSED; ++j) {
-    if (j < a.k) {
-      irow[j] = sid[j];
-      wrow[j] = a.renorm ? sc[j] / (ssum + 1e-9f) : sc[j];
-    }
-  }
-  return true;
-}
-
-template <int NSEL>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-router_pair_kernel(const __grid_constant__ CUtensorMap tmX,
-                   const __grid_constant__ CUtensorMap tmW, const PairRouterArgs a) {
-  using C = PCfg<NSEL>;
-  constexpr int NMMA = C::NMMA;
-  constexpr uint32_t IDESC = idesc_bf16_f32(256, NMMA);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  float* s_logits = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* bars =
-      reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::LOGIT_BYTES);
-  uint64_t* full_bar = bars;                               // rank 0's copy counts both CTAs
-  uint64_t* empty_bar = bars + C::STAGES;                  // both copies
-  uint64_t* sfull_bar = bars + 2 * C::STAGES;              // both copies
-  uint64_t* sempty_bar = bars + 2 * C::STAGES + C::NSLOT;  // rank 0's copy, 8 arrivals
-  uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
-  __shared__ uint32_t s_tmem;
-  __shared__ int s_abort, s_epi_abort, s_nlist, s_last, s_nlist_batch;
-  __shared__ __align__(16) float s_off[NSEL];
-  __shared__ __align__(16) float s_bias[NSEL];
-  __shared__ int s_sel[(KMAX_FUSED + 1) * 128];
-  __shared__ uint32_t s_masks[NSEL][4];
-  __shared__ int s_list[PR_LIST_MAX];
-  __shared__ int s_cand[PR_LIST_MAX * kRefineCand];
-  __shared__ double s_pl[PR_PAIRS_MAX];    // exact logits of the batch's pairs
-  __shared__ int s_pt[PR_PAIRS_MAX];       // their token rows
-  __shared__ int s_pe[PR_PAIRS_MAX];       // their experts
-  __shared__ int s_pbase[PR_LIST_MAX + 1]; // first pair of each listed token
-  __shared__ int s_cnt[NSEL];
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int kblocks = a.K / RBK;
-  const int chunks = (kblocks + KCH - 1) / KCH;
-  const int E = a.E;
-
-  if (threadIdx.x == 0) {
-    s_abort = 0;
-    s_epi_abort = 0;
-    s_nlist = 0;
-    s_last = 0;
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
-    }
-    for (int s = 0; s < C::NSLOT; ++s) {
-      mbar_init(&sfull_bar[s], 1);
-      mbar_init(&sempty_bar[s], 8);
-    }
-    mbar_init(drain_bar, 1);
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmW);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(&s_tmem, C::TMEM_COLS);
-    tmem_relinquish_pair();
-  }
-  pdl_wait();   // everything above touches no global memory
-  if (warp >= 2) {
-    for (int e = threadIdx.x - 64; e < NSEL; e += 128) {
-      s_off[e] = (e < E && a.offset) ? a.offset[e] : 0.f;
-      s_bias[e] = (e < E && a.bias) ? a.bias[e] : 0.f;
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();          // both CTAs' barriers are initialised
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  volatile int* abort_flag = &s_abort;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
-      bool ok = true;
-      const uint64_t keep_x = l2_evict_last_policy();
-      // a box that would lie wholly outside the tensor is pointed at row 0
-      // instead (its rows are never read out)
-      int wrow = static_cast<int>(rank) * (NMMA / 2);
-      if (wrow >= E) wrow = 0;
-      for (int tile = pair; tile < a.ntiles && ok; tile += npairs) {
-        int xrow = tile * 2 * a.tpc + static_cast<int>(rank) * a.tpc;
-        if (xrow >= a.T) xrow = 0;
-        for (int kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          if (rank == 0)
-            mbar_arrive_expect_tx(&full_bar[stage], 2u * (a.tpc * 128u + C::B_BYTES));
-          tma_load_2d_pair_hint(sA + stage * C::A_BYTES, &tmX, &full_bar[stage], kb * RBK, xrow,
-                                keep_x);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmW, &full_bar[stage], kb * RBK, wrow);
-          issued_mask |= 1u << stage;
-          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-        }
-      }
-      pdl_trigger();   // all loads issued: the next kernel may launch
-      if (!ok && rank == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
-          if (!(issued_mask & (1u << s))) continue;
-          const unsigned long long t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full_bar[s], (issued_phase >> s) & 1u))
-            if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------- MMA issuer (rank 0)
-    if (lane == 0 && rank == 0) {
-      int stage = 0, cc = 0;
-      uint32_t phase = 0;
-      bool ok = true, issued = false;
-      for (int tile = pair; tile < a.ntiles && ok; tile += npairs) {
-        for (int ch = 0; ch < chunks && ok; ++ch, ++cc) {
-          const int slot = cc % C::NSLOT;
-          const uint32_t sph = (cc / C::NSLOT) & 1;
-          if (!mbar_wait(&sempty_bar[slot], sph ^ 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem + slot * NMMA;
-          const int kb_end = (ch + 1) * KCH < kblocks ? (ch + 1) * KCH : kblocks;
-          for (int kb = ch * KCH; kb < kb_end; ++kb) {
-            if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t sa = smem_u32(sA + stage * C::A_BYTES);
-            const uint32_t sb = smem_u32(sB + stage * C::B_BYTES);
-#pragma unroll
-            for (int kk = 0; kk < RBK / 16; ++kk)
-              tc_mma_f16_pair(d, smem_desc_sw128(sa + kk * 32), smem_desc_sw128(sb + kk * 32),
-                              IDESC, (kb > ch * KCH || kk > 0) ? 1u : 0u);
-            issued = true;
-            tc_commit_pair(&empty_bar[stage]);
-            if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
-          }
-          if (!ok) break;
-          tc_commit_pair(&sfull_bar[slot]);
-        }
-      }
-      if (!ok && issued) {
-        tc_commit_pair(drain_bar);
-        const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0))
-          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int ew = warp - 2;               // epilogue warp 0..3
-    const int q = warp & 3;                // TMEM lane quadrant of this warp
-    const int row = q * 32 + lane;         // token row of this thread in the CTA's block
-    const int et = threadIdx.x - 64;       // 0..127
-    float* s_log = s_logits + et;
-    int* sel = s_sel + row;
-    int cc = 0;
-    int refined = 0;
-    for (int tile = pair; tile < a.ntiles; tile += npairs) {
-      float acc[NSEL];
-#pragma unroll
-      for (int i = 0; i < NSEL; ++i) acc[i] = 0.f;
-      bool ok = true;
-      for (int ch = 0; ch < chunks; ++ch, ++cc) {
-        if (!ok) continue;
-        const int slot = cc % C::NSLOT;
-        const uint32_t sph = (cc / C::NSLOT) & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[slot], sph, abort_flag));
-        if (!ok) continue;
-        tc_fence_after();
-        const uint32_t taddr = tmem + slot * NMMA + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll
-        for (int c = 0; c < NSEL / 16; ++c) {
-          uint32_t v[16];
-          tmem_ld16(taddr + c * 16, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[c * 16 + i] += __uint_as_float(v[i]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_rank0(&sempty_bar[slot]);
-      }
-      // one decision for the four epilogue warps: all go on, or all stop
-      if (!ok && lane == 0) s_epi_abort = 1;
-      for (int i = et; i < NSEL * 4; i += 128) (&s_masks[0][0])[i] = 0u;
-      if (et == 0) s_nlist = 0;
-      epi_bar();
-      if (s_epi_abort) break;
-      const int b = tile * 2 + static_cast<int>(rank);        // block of tpc tokens
-      const int t = b * a.tpc + row;
-      const bool valid = row < a.tpc && t < a.T;
-      if (valid)
-        pair_route_row<NSEL>(acc, s_log, sel, s_off, s_bias, E, t, row, a, &s_nlist, s_list,
-                             s_cand);
-      epi_bar();
-      // exact re-decision of the listed tokens: their (token, candidate)
-      // pairs in batches of up to PR_PAIRS_MAX, the exact logits of a batch
-      // by the four epilogue warps together, then one warp per token decides
-      const int nlist = s_nlist;
-      refined += nlist;
-      for (int i0 = 0; i0 < nlist;) {
-        if (et == 0) {
-          int np = 0, i = i0;
-          for (; i < nlist; ++i) {
-            const int* cand = s_cand + i * kRefineCand;
-            int n = E;
-            if (cand[0] != -2) {
-              n = 0;
-              while (n < kRefineCand && cand[n] >= 0) ++n;
-            }
-            if (np + n > PR_PAIRS_MAX && i > i0) break;   // the next batch takes it
-            s_pbase[i - i0] = np;
-            np += n;
-          }
-          s_pbase[i - i0] = np;
-          s_nlist_batch = i - i0;
-        }
-        epi_bar();
-        const int nb = s_nlist_batch;
-        for (int q = et; q < s_pbase[nb]; q += 128) {
-          int i = 0;
-          while (s_pbase[i + 1] <= q) ++i;
-          const int* cand = s_cand + (i0 + i) * kRefineCand;
-          const int c = q - s_pbase[i];
-          s_pt[q] = b * a.tpc + s_list[i0 + i];
-          s_pe[q] = cand[0] == -2 ? c : cand[c];
-        }
-        epi_bar();
-        exact_pair_logits(a.x, a.wr, a.offset, a.K, s_pt, s_pe, s_pbase[nb], s_pl, ew, 4);
-        epi_bar();
-        for (int i = ew; i < nb; i += 4) {
-          const int r = s_list[i0 + i];
-          const int tt = b * a.tpc + r;
-          const bool all = s_cand[(i0 + i) * kRefineCand] == -2;
-          refine_select(s_pl + s_pbase[i], s_pe + s_pbase[i], s_pbase[i + 1] - s_pbase[i],
-                        a.bias, a.k, a.gate, a.renorm, all, 0, nullptr,
-                        a.topk_idx + static_cast<size_t>(tt) * a.k,
-                        a.topk_w + static_cast<size_t>(tt) * a.k, s_sel + r, 128);
-        }
-        epi_bar();
-        i0 += nb;
-      }
-      // ranks inside the block: one bit per (expert, token)
-      if (valid)
-        for (int j = 0; j < a.k; ++j) atomicOr(&s_masks[sel[j * 128]][row >> 5], 1u << (row & 31));
-      epi_bar();
-      if (valid) {
-        const uint32_t below = (1u << (row & 31)) - 1u;
-        const int w = row >> 5;
-        for (int j = 0; j < a.k; ++j) {
-          const int e = sel[j * 128];
-          int r = __popc(s_masks[e][w] & below);
-          for (int ww = 0; ww < w; ++ww) r += __popc(s_masks[e][ww]);
-          a.rank_out[static_cast<size_t>(t) * a.k + j] = r;
-        }
-      }
-      if (b < a.nblk)
-        for (int e = et; e < E; e += 128)
-          a.blk[static_cast<size_t>(b) * E + e] = __popc(s_masks[e][0]) + __popc(s_masks[e][1]) +
-                                                   __popc(s_masks[e][2]) + __popc(s_masks[e][3]);
-      __threadfence();   // block counts visible before this CTA counts itself done
-      epi_bar();
-    }
-    if (et == 0 && refined > 0) atomicAdd(a.refine_count, refined);
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    if (s_abort || s_epi_abort) atomicOr(a.status, kDevTimeout);
-    if (a.fuse_scan) {
-      __threadfence();
-      s_last = atomicAdd(a.done, 1u) == gridDim.x - 1 ? 1 : 0;
-    }
-  }
-  __syncthreads();
-  if (s_last) {
-    // the dispatch scan over every block's counts (all CTAs have finished
-    // writing them): per-expert running sums over blocks, then the
-    // exclusive prefix over experts
-    __threadfence();
-    int* sb = reinterpret_cast<int*>(smem);   // the stage ring is idle now
-    const int n = a.nblk * E;
-    // 16-byte loads, eight in flight per thread (E a multiple of 4; the
-    // block counts start 256-byte aligned), then the rest one by one
-    const int n4 = E % 4 == 0 ? n / 4 : 0;
-    const int4* g4 = reinterpret_cast<const int4*>(a.blk);
-    int4* s4 = reinterpret_cast<int4*>(sb);
-    for (int i0 = threadIdx.x; i0 < n4; i0 += 8 * blockDim.x) {
-      int4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n4) v[u] = __ldcg(g4 + i);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n4) s4[i] = v[u];
-      }
-    }
-    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) sb[i] = __ldcg(a.blk + i);
-    __syncthreads();
-    if (threadIdx.x < E) {
-      // running sums over the blocks of expert e, four segments of blocks
-      // in flight at once
-      const int e = threadIdx.x, nb = a.nblk, seg = (nb + 3) / 4;
-      int sum[4] = {0, 0, 0, 0};
-      for (int j = 0; j < seg; ++j)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int bb = q * seg + j;
-          if (bb < nb) sum[q] += sb[bb * E + e];
-        }
-      int base[4] = {0, sum[0], sum[0] + sum[1], sum[0] + sum[1] + sum[2]};
-      for (int j = 0; j < seg; ++j)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int bb = q * seg + j;
-          if (bb < nb) {
-            const int c = sb[bb * E + e];
-            sb[bb * E + e] = base[q];
-            base[q] += c;
-          }
-        }
-      const int total = sum[0] + sum[1] + sum[2] + sum[3];
-      s_cnt[e] = total;
-      a.counts[e] = total;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // exclusive prefix over the experts: eight consecutive experts per lane
-      int v[8], loc = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane * 8 + j;
-        v[j] = e < E ? s_cnt[e] : 0;
-        loc += v[j];
-      }
-      int incl = loc;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      int run = incl - loc;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane * 8 + j;
-        if (e < E) {
-          s_cnt[e] = run;
-          a.offsets[e] = run;
-        }
-        run += v[j];
-      }
-      if (lane == 31) a.offsets[E] = incl;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < n4; i += blockDim.x) {
-      const int e0 = (4 * i) % E;
-      int4 v = s4[i];
-      v.x += s_cnt[e0];
-      v.y += s_cnt[e0 + 1];
-      v.z += s_cnt[e0 + 2];
-      v.w += s_cnt[e0 + 3];
-      reinterpret_cast<int4*>(a.blk)[i] = v;
-    }
-    for (int i = 4 * n4 + threadIdx.x; i < n; i += blockDim.x) a.blk[i] = sb[i] + s_cnt[i % E];
-  }
-  __syncthreads();
-  cluster_sync_all();          // neither CTA leaves while the other still uses the pair
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc_pair(tmem, C::TMEM_COLS);
-  }
-}
-
-template <int NSEL>
-cudaError_t launch_router_pair(const CUtensorMap& mx, const CUtensorMap& mw,
-                               const PairRouterArgs& a, cudaStream_t stream) {
-  using C = PCfg<NSEL>;
-  auto kern = router_pair_kernel<NSEL>;
-  static unsigned long long attr_done = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_done & bit)) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done |= bit;
-  }
-  int sms = 0;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int max_pairs = sms >= 2 ? sms / 2 : 1;
-  const int pairs = a.ntiles < max_pairs ? a.ntiles : max_pairs;
-  return launch_pdl(kern, dim3(2 * pairs), dim3(192), C::SMEM_BYTES, stream, mx, mw, a);
-}
-
-template <int NSEL>
-int pair_scan_capacity() {
-  return PCfg<NSEL>::SCAN_INTS;
-}
-
-int nsel_for(int E) {
-  int n = 16;
-  while (n < E) n *= 2;
-  return n;
-}
-
 }  // namespace
-
-// Tokens per CTA block of the fused pair router: the tiles of 2 * tpc tokens
-// fill kRouterPairs CTA pairs in whole waves (tpc <= 128, at least 32, a
-// multiple of 8).  A function of T alone, so the workspace layout does not
-// depend on the device.
-int router_pair_block_tokens(int T) {
-  const long long per_wave = 2LL * kRouterPairs * 128;
-  const long long w = (T + per_wave - 1) / per_wave;
-  long long tpc = (T + 2LL * kRouterPairs * w - 1) / (2LL * kRouterPairs * w);
-  tpc = (tpc + 7) / 8 * 8;
-  if (tpc < 32) tpc = 32;
-  if (tpc > 128) tpc = 128;
-  return static_cast<int>(tpc);
-}
-
-int router_pair_blocks(int T) {
-  const int tpc = router_pair_block_tokens(T);
-  return (T + tpc - 1) / tpc;
-}
-
-cudaError_t router_topk_pair(const void* x, int T, const void* w_router, int E, int K,
-                             const float* logit_offset, const float* sel_bias, int k, int gate,
-                             int renorm, int32_t* topk_idx, float* topk_w, int32_t* rank_out,
-                             int32_t* blk, int32_t* counts, int32_t* offsets,
-                             int32_t* refine_count, uint32_t* status, uint32_t* done,
-                             bool* scan_fused, cudaStream_t stream) {
-  *scan_fused = false;
-  if (T <= 0) return cudaSuccess;
-  if (!router_fused_supported(E, k)) return cudaErrorInvalidValue;
-  const int nsel = nsel_for(E);
-  const int nmma = nsel < 64 ? 64 : nsel;
-  PairRouterArgs a{};
-  a.x = static_cast<const __nv_bfloat16*>(x);
-  a.wr = static_cast<const __nv_bfloat16*>(w_router);
-  a.offset = logit_offset;
-  a.bias = sel_bias;
-  a.T = T;
-  a.K = K;
-  a.E = E;
-  a.k = k;
-  a.gate = gate;
-  a.renorm = renorm;
-  a.tpc = router_pair_block_tokens(T);
-  a.ntiles = (T + 2 * a.tpc - 1) / (2 * a.tpc);
-  a.nblk = (T + a.tpc - 1) / a.tpc;
-  int cap = 0;
-  switch (nsel) {
-    case 16: cap = pair_scan_capacity<16>(); break;
-    case 32: cap = pair_scan_capacity<32>(); break;
-    case 64: cap = pair_scan_capacity<64>(); break;
-    default: cap = pair_scan_capacity<128>(); break;
-  }
-  a.fuse_scan = static_cast<long long>(a.nblk) * E <= cap ? 1 : 0;
-  a.topk_idx = topk_idx;
-  a.topk_w = topk_w;
-  a.rank_out = rank_out;
-  a.blk = blk;
-  a.counts = counts;
-  a.offsets = offsets;
-  a.refine_count = refine_count;
-  a.status = status;
-  a.done = done;
-  CUtensorMap mx, mw;
-  if (!map2d(&mx, x, T, K, a.tpc) || !map2d(&mw, w_router, E, K, nmma / 2))
-    return cudaErrorInvalidValue;
-  cudaError_t err;
-  switch (nsel) {
-    case 16: err = launch_router_pair<16>(mx, mw, a, stream); break;
-    case 32: err = launch_router_pair<32>(mx, mw, a, stream); break;
-    case 64: err = launch_router_pair<64>(mx, mw, a, stream); break;
-    default: err = launch_router_pair<128>(mx, mw, a, stream); break;
-  }
-  if (err == cudaSuccess) *scan_fused = a.fuse_scan != 0;
-  return err;
-}
 
 bool router_fused_supported(int E, int k) { return npad_for(E) <= 128 && k <= KMAX_FUSED; }
 
