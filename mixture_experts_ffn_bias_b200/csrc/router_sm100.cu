@@ -47,25 +47,34 @@ constexpr int RBK = 64;
 constexpr int KCH = 2;                       // k-blocks per accumulation chunk
 constexpr int R_A_BYTES = RBM * RBK * 2;
 
+constexpr int KMAX_FUSED = 8;
+constexpr int PICKS = KMAX_FUSED + 2;        // a part's picks (k + 1 at most) and an end mark
+constexpr int kSelectParts = 4;              // fused select over 128 experts: 4 x 32 keys
+
 template <int NPAD, bool FUSED = false>
 struct RCfg {
-  static constexpr int EPI_WG = NPAD > 128 ? 2 : 1;
+  // Epilogue warpgroups: each holds NPAD / EPI_WG accumulator columns of
+  // every row.  The fused select over 128 experts splits a token's keys
+  // between kSelectParts threads, which divides the serial per-thread work
+  // and gives each SM sub-partition more warps to interleave; the first
+  // warpgroup merges the partial rankings.
+  static constexpr int EPI_WG = (FUSED && NPAD == 128) ? kSelectParts : (NPAD > 128 ? 2 : 1);
   static constexpr int COLS = NPAD / EPI_WG;           // columns per epilogue thread
   static constexpr int THREADS = 64 + 128 * EPI_WG;
   static constexpr int B_BYTES = NPAD * RBK * 2;
   static constexpr int STAGE_BYTES = R_A_BYTES + B_BYTES;
-  // fused select keeps each token's logits in a shared-memory column
+  // fused select keeps each token's logits in a shared-memory column, and
+  // each warpgroup's partial ranking (values and ids) in two more
   static constexpr int LOGIT_BYTES = FUSED ? NPAD * 128 * 4 : 0;
-  static constexpr int STAGE_BUDGET = 212992 - LOGIT_BYTES;   // 208 KB of stages + logit column
+  static constexpr int PICK_BYTES = FUSED ? EPI_WG * PICKS * 128 * 8 : 0;
+  static constexpr int STAGE_BUDGET = 226304 - LOGIT_BYTES - PICK_BYTES;   // of 227 KB
   static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 8 ? 8 : (STAGE_BUDGET / STAGE_BYTES);
   static constexpr int NSLOT = (512 / NPAD) > 8 ? 8 : (512 / NPAD);
   static constexpr int TMEM_RAW = NSLOT * NPAD;
   static constexpr int TMEM_COLS = TMEM_RAW <= 32 ? 32 : TMEM_RAW <= 64 ? 64
                                    : TMEM_RAW <= 128 ? 128 : TMEM_RAW <= 256 ? 256 : 512;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LOGIT_BYTES + 1024 + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + LOGIT_BYTES + PICK_BYTES + 1024 + 1024;
 };
-
-constexpr int KMAX_FUSED = 8;
 
 // TMA tile load with an L2 eviction-priority policy (the router's x tiles
 // are marked evict-last, so the dispatch scatter that re-reads x right after
@@ -86,6 +95,13 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Prefetch of one tile box into L2 (x aligned as for a tile load); no
+// completion is tracked.
+__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
+}
+
 struct RouterOut {
   float* logits;                 // unfused: [T, E] fp32
   const float* offset;           // fused: per-expert logit offset or null
@@ -99,83 +115,71 @@ struct RouterOut {
   uint32_t* status;
 };
 
-// Routing decision for one token from its logits held in registers (fused
-// select).  acc[i] = logit of expert i (i < E), overwritten with the
-// selection keys; the logits (with the per-expert offset) are kept in the
-// thread's shared-memory column s_log[i * 128], so the weights use them
-// exactly and the per-round re-scan can index them.  One thread owns a token
-// and only four warps run this per SM, so the code is written for
-// instruction-level parallelism: no branches inside the loops (even a
-// warp-uniform branch splits the unrolled loop into blocks that cannot be
-// interleaved), selects instead of short-circuit conditions, four partial
-// maxima and sums, and loads kept apart from stores.
+// Fused select, part 1, run by every epilogue thread for its token over the
+// experts [base, base + COLS) whose logits it holds in acc[] (i < E only).
+// The logits (with the per-expert offset) go to the token's shared-memory
+// column s_log[e * 128], acc[] becomes the selection keys (logit + bias),
+// and the best min(rounds, experts here) keys in (descending key, ascending
+// id) order go to pv/pi[j * 128] with an end mark after them.  Returns the
+// largest logit of the part.
+//
+// One thread owns a (token, part) and only a few warps run this per SM, so
+// the code is written for instruction-level parallelism: no branches inside
+// the loops (even a warp-uniform branch splits an unrolled loop into blocks
+// that cannot be interleaved), selects instead of short-circuit conditions,
+// four partial maxima and sums, loads kept apart from stores.  The ranking
+// splits the part into NG groups of GS consecutive ids, each holding its
+// best key not yet picked; a round takes the best group head and re-scans
+// only that group (keys re-formed from the logit column and the bias: the
+// same fp32 sums as acc[]).
 template <int COLS>
-__device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int* s_seli,
-                                          const float* s_off, const float* s_bias, int E, int t,
-                                          const RouterOut& o) {
+__device__ __forceinline__ float route_part(float (&acc)[COLS], float* s_log, const float* s_off,
+                                            const float* s_bias, int base, int E, int rounds,
+                                            float* pv, int* pi) {
+  constexpr int NONE = 0x7fffffff;
   float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int i = 0; i < COLS; i += 4) {
-    const float4 f = *reinterpret_cast<const float4*>(s_off + i);
+    const float4 f = *reinterpret_cast<const float4*>(s_off + base + i);
     const float ov[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float l = i + q < E ? acc[i + q] + ov[q] : -INFINITY;
+      const float l = base + i + q < E ? acc[i + q] + ov[q] : -INFINITY;
       acc[i + q] = l;
       mx[q] = fmaxf(mx[q], l);
     }
   }
 #pragma unroll
-  for (int i = 0; i < COLS; ++i) s_log[i * 128] = acc[i];
+  for (int i = 0; i < COLS; ++i) s_log[(base + i) * 128] = acc[i];
 #pragma unroll
   for (int i = 0; i < COLS; i += 4) {
-    const float4 f = *reinterpret_cast<const float4*>(s_bias + i);
+    const float4 f = *reinterpret_cast<const float4*>(s_bias + base + i);
     const float bv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) acc[i + q] = i + q < E ? acc[i + q] + bv[q] : -INFINITY;
+    for (int q = 0; q < 4; ++q)
+      acc[i + q] = base + i + q < E ? acc[i + q] + bv[q] : -INFINITY;
   }
   const float m = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-  // The softmax denominator is needed only without renormalisation: with
-  // it, the weights exp(l_j - m) / sum over the picks are the renormalised
-  // probabilities (the 1e-9 guard then scales with the denominator).
-  float S = 1.0f;
-  if (o.gate == 0 && !o.renorm) {
-    float sp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-    for (int i = 0; i < COLS; i += 4) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sp[q] += expf(s_log[(i + q) * 128] - m);   // exp(-inf) = 0 past E
-    }
-    S = (sp[0] + sp[1]) + (sp[2] + sp[3]);
-  }
-  // top-(k+1) keys in (descending key, ascending expert id) order.  The
-  // experts are split into NG groups of GS consecutive ids; each group holds
-  // its best key not yet picked.  A round takes the best group head and
-  // re-scans only that group (keys re-formed from the shared-memory logit
-  // column and the bias: the same fp32 sums as acc[]) for its best key after
-  // the pick.  Picks go to the thread's shared-memory column s_seli.
   constexpr int GS = COLS >= 64 ? 8 : 4;
   constexpr int NG = COLS / GS;
-  constexpr int NONE = 0x7fffffff;
   float gv[NG];
   int gi[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     gv[g] = acc[g * GS];
-    gi[g] = g * GS;
+    gi[g] = base + g * GS;
 #pragma unroll
     for (int s = 1; s < GS; ++s) {
       const bool take = acc[g * GS + s] > gv[g];
       gv[g] = take ? acc[g * GS + s] : gv[g];
-      gi[g] = take ? g * GS + s : gi[g];
+      gi[g] = take ? base + g * GS + s : gi[g];
     }
+    gi[g] = base + g * GS < E ? gi[g] : NONE;   // a group wholly past E holds nothing
   }
-  const int rounds = o.k < E ? o.k + 1 : o.k;
-  float pv = INFINITY;
-  int pi = -1;
-  float min_gap = INFINITY;
+  const int here = E - base < COLS ? (E - base > 0 ? E - base : 0) : COLS;
+  const int n = rounds < here ? rounds : here;
 #pragma unroll 1
-  for (int j = 0; j < rounds; ++j) {
+  for (int j = 0; j < n; ++j) {
     // groups are in id order, so on equal heads the earlier group wins
     float bv = gv[0];
     int bi = gi[0], bg = 0;
@@ -186,23 +190,21 @@ __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int*
       bi = take ? gi[g] : bi;
       bg = take ? g : bg;
     }
-    min_gap = j > 0 ? fminf(min_gap, pv - bv) : min_gap;
-    pv = bv;
-    pi = bi;
-    s_seli[j * 128] = bi;
+    pv[j * 128] = bv;
+    pi[j * 128] = bi;
     float vv[GS];
 #pragma unroll
     for (int s = 0; s < GS; ++s) {
-      const int i = bg * GS + s;
+      const int i = base + bg * GS + s;
       vv[s] = i < E ? s_log[i * 128] + s_bias[i] : -INFINITY;
     }
     float nv = -INFINITY;
     int ni = NONE;
 #pragma unroll
     for (int s = 0; s < GS; ++s) {
-      const int i = bg * GS + s;
-      const bool after = (vv[s] < pv) | ((vv[s] == pv) & (i > pi));
-      const bool take = after & ((vv[s] > nv) | (ni == NONE));
+      const int i = base + bg * GS + s;
+      const bool after = (vv[s] < bv) | ((vv[s] == bv) & (i > bi));
+      const bool take = (i < E) & after & ((vv[s] > nv) | (ni == NONE));
       nv = take ? vv[s] : nv;
       ni = take ? i : ni;
     }
@@ -212,6 +214,50 @@ __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int*
       gi[g] = g == bg ? ni : gi[g];
     }
   }
+  pv[n * 128] = -INFINITY;   // end mark
+  pi[n * 128] = NONE;
+  return m;
+}
+
+// Fused select, part 2, for one token: merge the NP partial rankings (part p
+// holds lower expert ids than part p + 1, so equal keys take the earlier
+// part) into the top-(k+1) keys, then either list the token for exact
+// re-decision (two of those keys closer than kRefineMargin) with its
+// candidate experts, or write its k experts and weights.  m_part[128 p]:
+// the parts' largest logits.
+template <int NP>
+__device__ __forceinline__ void route_finish(const float* pv, const int* pi, int pstride,
+                                             const float* m_part, const float* s_log,
+                                             const float* s_bias, int E, int t,
+                                             const RouterOut& o) {
+  constexpr int NONE = 0x7fffffff;
+  const int rounds = o.k < E ? o.k + 1 : o.k;
+  int head[NP];
+#pragma unroll
+  for (int p = 0; p < NP; ++p) head[p] = 0;
+  int sid[KMAX_FUSED];
+  float prev = 0.f, min_gap = INFINITY;
+#pragma unroll
+  for (int j = 0; j < KMAX_FUSED + 1; ++j) {
+    if (j < rounds) {
+      float bv = pv[head[0] * 128];
+      int bi = pi[head[0] * 128], bp = 0;
+#pragma unroll
+      for (int p = 1; p < NP; ++p) {
+        const float v = pv[p * pstride + head[p] * 128];
+        const int i = pi[p * pstride + head[p] * 128];
+        const bool take = (i != NONE) & ((bi == NONE) | (v > bv));
+        bv = take ? v : bv;
+        bi = take ? i : bi;
+        bp = take ? p : bp;
+      }
+#pragma unroll
+      for (int p = 0; p < NP; ++p) head[p] += p == bp ? 1 : 0;
+      min_gap = j > 0 ? fminf(min_gap, prev - bv) : min_gap;
+      prev = bv;
+      if (j < KMAX_FUSED) sid[j] = bi;
+    }
+  }
   if (min_gap < kRefineMargin) {
     // list the token with its candidate experts: every expert whose key is
     // within the margin of the last pick (the exact top-k is among them);
@@ -219,32 +265,58 @@ __device__ __forceinline__ void route_row(float (&acc)[COLS], float* s_log, int*
     const int slot = atomicAdd(o.refine_count, 1);
     o.refine_list[slot] = t;
     int32_t* cand = o.refine_cand + static_cast<size_t>(slot) * kRefineCand;
-    const float lo = pv - kRefineMargin;
-    int n = (o.gate == 0 && !o.renorm) ? kRefineCand + 1 : 0;
-#pragma unroll 1
-    for (int i = 0; i < E; ++i) {
-      if (s_log[i * 128] + s_bias[i] >= lo) {   // the key, as in acc[]
-        if (n < kRefineCand) cand[n] = i;
-        ++n;
+    const float lo = prev - kRefineMargin;
+    uint32_t msk[4];   // E <= 128 here
+    int n = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint32_t b = 0;
+#pragma unroll
+      for (int u = 0; u < 32; ++u) {
+        const int i = w * 32 + u;
+        const float v = i < E ? s_log[i * 128] + s_bias[i] : -INFINITY;   // the key, as in the parts
+        b |= (v >= lo ? 1u : 0u) << u;
       }
+      msk[w] = b;
+      n += __popc(b);
     }
-    if (n > kRefineCand) {
+    if (n > kRefineCand || (o.gate == 0 && !o.renorm)) {
       cand[0] = -2;
       n = 1;
+    } else {
+      n = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        for (uint32_t b = msk[w]; b != 0u; b &= b - 1u) cand[n++] = w * 32 + __ffs(b) - 1;
+      }
     }
     for (int c = n; c < kRefineCand; ++c) cand[c] = -1;
     return;
   }
+  float m = m_part[0];
+#pragma unroll
+  for (int p = 1; p < NP; ++p) m = fmaxf(m, m_part[p * 128]);
+  // The softmax denominator is needed only without renormalisation: with
+  // it, the weights exp(l_j - m) / sum over the picks are the renormalised
+  // probabilities (the 1e-9 guard then scales with the denominator).
+  float S = 1.0f;
+  if (o.gate == 0 && !o.renorm) {
+    float sp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int i = 0; i < E; i += 4) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        sp[q] += i + q < E ? expf(s_log[(i + q) * 128] - m) : 0.f;
+    }
+    S = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+  }
   float sc[KMAX_FUSED];
-  int sid[KMAX_FUSED];
   float ssum = 0.f;
 #pragma unroll
   for (int j = 0; j < KMAX_FUSED; ++j) {
     sc[j] = 0.f;
-    sid[j] = 0;
     if (j < o.k) {
-      sid[j] = s_seli[j * 128];
-      const float l = s_log[sid[j] * 128];
+      const float l = s_log[(sid[j] < E ? sid[j] : 0) * 128];   // a pick is an id < E unless keys are NaN
       sc[j] = o.gate == 1 ? 1.0f / (1.0f + expf(-l)) : expf(l - m) / S;
       ssum += sc[j];
     }
@@ -272,18 +344,26 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * R_A_BYTES;
   float* s_logits = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* bars =
-      reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::LOGIT_BYTES);
+  // fused select: part p's ranking of row r, entry j at [p * PSTRIDE + j * 128 + r]
+  constexpr int PSTRIDE = PICKS * 128;
+  float* s_pv = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + C::LOGIT_BYTES);
+  int* s_pi = reinterpret_cast<int*>(s_pv + C::EPI_WG * PSTRIDE * (FUSED ? 1 : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES +
+                                               C::LOGIT_BYTES + C::PICK_BYTES);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + C::STAGES;
   uint64_t* sfull_bar = bars + 2 * C::STAGES;
   uint64_t* sempty_bar = bars + 2 * C::STAGES + C::NSLOT;
   uint64_t* drain_bar = bars + 2 * C::STAGES + 2 * C::NSLOT;
+  // fused select in parts: the other warpgroups' rankings are ready (xfull),
+  // the first has merged them and they may be overwritten (xfree)
+  uint64_t* xfull_bar = drain_bar + 1;
+  uint64_t* xfree_bar = drain_bar + 2;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   __shared__ __align__(16) float s_off[NPAD];
   __shared__ __align__(16) float s_bias[NPAD];
-  __shared__ int s_sel[FUSED ? (KMAX_FUSED + 1) * 128 : 1];
+  __shared__ float s_mpart[FUSED ? C::EPI_WG * 128 : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles = (T + RBM - 1) / RBM;
@@ -301,6 +381,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       mbar_init(&sempty_bar[s], 4 * C::EPI_WG);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(xfull_bar, 128 * (C::EPI_WG > 1 ? C::EPI_WG - 1 : 1));
+    mbar_init(xfree_bar, 128);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -331,6 +413,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       bool ok = true;
       const uint64_t keep_x = l2_evict_last_policy();
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        // Ask L2 for every x box of the tile up front, in k-block order:
+        // the tile loads of the ring can hold only a few stages of this
+        // HBM stream in flight, the prefetches all of it.
+        for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmX, kb * RBK, tile * RBM);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
@@ -391,12 +477,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     }
   } else {
     const int ew = warp - 2;                 // epilogue warp 0 .. 4*EPI_WG-1
-    const int wg = ew >> 2;                  // column half for NPAD = 256
+    const int wg = ew >> 2;                  // column part of this warpgroup
     const int q = warp & 3;                  // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;
-    int cc = 0;
+    int cc = 0, it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++it) {
       float acc[C::COLS];
 #pragma unroll
       for (int i = 0; i < C::COLS; ++i) acc[i] = 0.f;
@@ -422,11 +508,32 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       }
       if (!ok) break;
       const int t = tile * RBM + row;
-      if (t >= T) continue;
       if constexpr (FUSED) {
-        route_row<C::COLS>(acc, s_logits + (threadIdx.x - 64), s_sel + (threadIdx.x - 64),
-                           s_off, s_bias, E, t, out);
+        // every thread ranks its part of the row (rows past T too, so that
+        // all take part in the exchange); the first warpgroup merges
+        const int rounds = out.k < E ? out.k + 1 : out.k;
+        if (C::EPI_WG > 1 && wg > 0 && it > 0) {
+          // the first warpgroup must have merged the previous tile
+          ok = __all_sync(0xffffffffu, mbar_wait(xfree_bar, (it - 1) & 1, abort_flag));
+          if (!ok) break;
+        }
+        s_mpart[wg * 128 + row] =
+            route_part<C::COLS>(acc, s_logits + row, s_off, s_bias, wg * C::COLS, E, rounds,
+                                s_pv + wg * PSTRIDE + row, s_pi + wg * PSTRIDE + row);
+        if (C::EPI_WG > 1) {
+          if (wg > 0) {
+            mbar_arrive(xfull_bar);
+            continue;
+          }
+          ok = __all_sync(0xffffffffu, mbar_wait(xfull_bar, it & 1, abort_flag));
+          if (!ok) break;
+        }
+        if (t < T)
+          route_finish<C::EPI_WG>(s_pv + row, s_pi + row, PSTRIDE, s_mpart + row,
+                                  s_logits + row, s_bias, E, t, out);
+        if (C::EPI_WG > 1) mbar_arrive(xfree_bar);
       } else {
+        if (t >= T) continue;
         float* dst = out.logits + static_cast<size_t>(t) * E + wg * C::COLS;
         const int ncol = E - wg * C::COLS;
         if ((E & 3) == 0 && ncol >= C::COLS) {
