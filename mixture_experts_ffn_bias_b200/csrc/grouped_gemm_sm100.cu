@@ -94,7 +94,11 @@ struct PairTile {
   int kblocks;
 };
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+// silu(g) = g / (1 + e^-g) with the fast exponential and the fast divide
+// (a reciprocal and a multiply, no IEEE slow path): a few ulp of fp32, far
+// below the bf16 rounding of h that follows.  For g < -87, e^-g overflows
+// and the quotient is 0, the limit of silu.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -209,7 +213,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_of
   PairTile t;
   if (tile >= s_prefix[G]) {
     const int local = tile - s_prefix[G];
-    const int xn = a.x_n / BN_OUT;
+    const int xn = (a.x_n + BN_OUT - 1) / BN_OUT;
     t.x = true;
     t.g = 0;
     t.m = local / xn;
@@ -272,7 +276,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1;
   const int npairs = gridDim.x >> 1;
-  const int n_tiles = args.n_per_group / BN_OUT;
+  const int n_tiles = (args.n_per_group + BN_OUT - 1) / BN_OUT;   // a last tile may be partial
   const int G = args.offsets == nullptr ? 1 : args.num_groups;
 
   if (threadIdx.x == 0) {
@@ -312,7 +316,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int x_tiles = args.x_rows > 0 ? (args.x_rows + BM2 - 1) / BM2 * (args.x_n / BN_OUT) : 0;
+  const int x_tiles =
+      args.x_rows > 0 ? (args.x_rows + BM2 - 1) / BM2 * ((args.x_n + BN_OUT - 1) / BN_OUT) : 0;
   const int total_tiles = s_prefix[G] + x_tiles;
   volatile int* abort_flag = &s_abort;
 
@@ -461,6 +466,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           static_cast<size_t>(warp_row0 + lane) * (pt.x ? args.x_ldc : args.ldc);
       const uint32_t t_addr = tmem_base + acc * BN_ACC + (static_cast<uint32_t>(q * 32) << 16);
       constexpr int UP = Cfg::N_MMA / 2;   // up columns follow the gate columns
+      // output columns of the group: a last partial n-tile (plain mode, the
+      // columns a multiple of 64) skips its 64-column chunks past them
+      const int ncols = pt.x ? args.x_n : args.n_per_group;
 #pragma unroll 1
       for (int cb = 0; cb < BN_OUT / 64; ++cb) {
         // accumulator column of this 64-column chunk and its output column:
@@ -479,6 +487,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           ocol = n * BN_ACC + (jj / (Cfg::N_MMA / 2)) * (BN_ACC / 2) + sub * (Cfg::N_MMA / 2) +
                  jj % (Cfg::N_MMA / 2);
         }
+        if (ocol >= ncols) continue;   // warp-uniform
         uint32_t packed[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -615,9 +624,10 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
                          args.K * 2.0;
   a2r.m_fastest = b_bytes > 32.0 * 1024 * 1024 ? 1 : 0;
   const long long m_tiles_upper = (rows_upper + BM2 - 1) / BM2 + (G > 1 ? G : 0);
-  long long tiles_upper = m_tiles_upper * (args.n_per_group / BN_OUT);
+  long long tiles_upper = m_tiles_upper * ((args.n_per_group + BN_OUT - 1) / BN_OUT);
   if (args.x_rows > 0)
-    tiles_upper += static_cast<long long>((args.x_rows + BM2 - 1) / BM2) * (args.x_n / BN_OUT);
+    tiles_upper += static_cast<long long>((args.x_rows + BM2 - 1) / BM2) *
+                   ((args.x_n + BN_OUT - 1) / BN_OUT);
   if (tiles_upper <= 0) return cudaSuccess;
   const int max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles_upper < max_pairs ? tiles_upper : max_pairs);
@@ -741,7 +751,11 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
   // exposed epilogue is a small part of a tile: measured on B200, wide's
   // down GEMM (K = 4352) 0.616 -> 0.551 ms, but qwen3_30b's (K = 768) 0.33 ->
   // 0.38 ms
-  const int bn = (N % 512 == 0 && K >= 4096) ? 512 : (N % 256 == 0) ? 256 : 128;
+  // N a multiple of 128 but not of 256 (page-2 shape, d = 640): 256-column
+  // tiles with a half-empty last one beat 128-column tiles, whose A tile
+  // is streamed twice as often per MMA flop.
+  const int bn = (N % 512 == 0 && K >= 4096) ? 512
+                 : (N % 256 == 0 || (N % 128 == 0 && N > 256)) ? 256 : 128;
   // each CTA of the pair loads half of the B tile
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, c_rows, N, 32))

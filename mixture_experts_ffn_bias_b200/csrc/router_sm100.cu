@@ -95,13 +95,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-// Prefetch of one tile box into L2 (x aligned as for a tile load); no
-// completion is tracked.
-__device__ __forceinline__ void tma_prefetch_l2(const CUtensorMap* map, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y) : "memory");
-}
-
 struct RouterOut {
   float* logits;                 // unfused: [T, E] fp32
   const float* offset;           // fused: per-expert logit offset or null
@@ -413,10 +406,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       bool ok = true;
       const uint64_t keep_x = l2_evict_last_policy();
       for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        // Ask L2 for every x box of the tile up front, in k-block order:
-        // the tile loads of the ring can hold only a few stages of this
-        // HBM stream in flight, the prefetches all of it.
-        for (int kb = 0; kb < kblocks; ++kb) tma_prefetch_l2(&tmX, kb * RBK, tile * RBM);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
