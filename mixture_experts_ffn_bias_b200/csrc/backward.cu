@@ -10,9 +10,12 @@
 //   swiglu_bwd_kernel   dG = dH * U * silu'(G), dU = dH * silu(G)
 //   dx_gather_kernel    dx[t] = sum_j dX[slot(t, j)] + dx_router[t] (+ dx_shared[t])
 //   router_dlogits_kernel  dlogits from dw through the (renormalised) gate
-//   sgemm_kernel        fp32 CUDA-core GEMM for the router gradients (the
-//                       router runs in fp32: "moe-200m-qwen3-100b" README,
+//   router_grad_split_kernel  dlogits (fp32) as three bf16 terms, in the two
+//                       layouts the router-gradient GEMMs read (the router
+//                       runs in fp32: "moe-200m-qwen3-100b" README,
 //                       "Per-layer numerics")
+//   router_grad_reduce_kernel  dW_router = sum of the per-slice, per-term
+//                       fp32 partial products, in a fixed order
 // The chain rule is that of the layer in the "moe-200m-qwen3-100b" README
 // ("Architecture diagram", SigmoidRouter forward): out = shared(x) +
 // sum_j w_j expert_j(x), w = gate scores of the picked experts, renormalised.
@@ -312,122 +315,74 @@ router_dlogits_kernel(const float* __restrict__ logits, const float* __restrict_
 }
 
 // fp32 CUDA-core GEMM, split over K: part[z][m][n] = sum_{k in slice z} A(m, k) B(k, n).
-// A(m, k) = a[m * lda + k] (A_T: a[k * lda + m]), fp32; B(k, n) = b[k * ldb + n], bf16.
-// 128 x 128 tile per block, K in steps of 8 through shared memory, 256
-// threads with an 8 x 8 register tile each (rows ty + 16 i, columns
-// 4 tx + 64 j + q, so the shared-memory reads are float4 and conflict free).
-// N a multiple of 128, any M and K (rows past M and k past the slice read
-// as zero); kslice a multiple of 8.
-constexpr int SG_T = 128, SG_K = 8;
-
-template <bool A_T>
+// The router gradients dW_router = dlogits^T x and dx_router = dlogits Wr
+// run on the tensor cores.  x and Wr are bf16; dlogits (fp32) is written as
+// h1 + h2 + h3 with h1 = bf16(v), h2 = bf16(v - h1), h3 = bf16(v - h1 - h2)
+// (each difference exact in fp32), which represents v to within fp32
+// rounding (2^-24 relative); every product with a bf16 value is exact in
+// fp32, so the tensor cores' fp32 sums are the rounding, as in an fp32 GEMM.  Term j of expert e sits at index
+// j * Ep + e (Ep = E rounded up to 64, zeros past E):
+//   adx [T, 3 Ep]            row t: the terms of dlogits[t, :]   (dx GEMM, K = 3 Ep)
+//   adw [G, 3 Ep, Ks]        slice g of the tokens, transposed:  (dW GEMM, K = Ks
+//                            per slice, zeros past T)
+// goff[g] = g * 3 Ep are the row groups of adw (one GEMM group per slice).
+// Block b takes tokens [32 b, 32 b + 32), which lie in one slice.
 __global__ void __launch_bounds__(256)
-sgemm_kernel(const float* __restrict__ a, int lda, const __nv_bfloat16* __restrict__ b, int ldb,
-             int M, int N, int K, int kslice, float* __restrict__ part) {
+router_grad_split_kernel(const float* __restrict__ dlogits, int T, int E, int Ep, int Ks, int G,
+                         __nv_bfloat16* __restrict__ adx, __nv_bfloat16* __restrict__ adw,
+                         int32_t* __restrict__ goff) {
   pdl_trigger();
   pdl_wait();
-  __shared__ __align__(16) float As[SG_K][SG_T];
-  __shared__ __align__(16) float Bs[SG_K][SG_T];
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const int m0 = blockIdx.y * SG_T, n0 = blockIdx.x * SG_T;
-  const int kbeg = blockIdx.z * kslice, kend = min(K, kbeg + kslice);
-  const bool vec = (lda & 3) == 0;   // 16-byte aligned rows of A
-  float acc[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int k0 = kbeg; k0 < kend; k0 += SG_K) {
-    // A tile: 8 x 128 floats = 256 float4
-    if (A_T) {
-      const int kk = tid >> 5, mm = (tid & 31) * 4;   // row kk, columns mm..mm+3
-      const int k = k0 + kk, m = m0 + mm;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (k < kend) {
-        const float* src = a + static_cast<size_t>(k) * lda + m;
-        if (vec && m + 3 < M) {
-          v = *reinterpret_cast<const float4*>(src);
-        } else {
-          v.x = m < M ? src[0] : 0.f;
-          v.y = m + 1 < M ? src[1] : 0.f;
-          v.z = m + 2 < M ? src[2] : 0.f;
-          v.w = m + 3 < M ? src[3] : 0.f;
-        }
-      }
-      *reinterpret_cast<float4*>(&As[kk][mm]) = v;
-    } else {
-      const int mm = tid >> 1, kk = (tid & 1) * 4;     // row mm, k columns kk..kk+3
-      const int m = m0 + mm, k = k0 + kk;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (m < M) {
-        const float* src = a + static_cast<size_t>(m) * lda + k;
-        if (vec && k + 3 < kend) {
-          v = *reinterpret_cast<const float4*>(src);
-        } else {
-          v.x = k < kend ? src[0] : 0.f;
-          v.y = k + 1 < kend ? src[1] : 0.f;
-          v.z = k + 2 < kend ? src[2] : 0.f;
-          v.w = k + 3 < kend ? src[3] : 0.f;
-        }
-      }
-      As[kk][mm] = v.x;
-      As[kk + 1][mm] = v.y;
-      As[kk + 2][mm] = v.z;
-      As[kk + 3][mm] = v.w;
-    }
-    // B tile: 8 x 128 bf16 = 128 x 16 bytes
-    if (tid < 128) {
-      const int kk = tid >> 4, nn = (tid & 15) * 8;
-      const int k = k0 + kk, n = n0 + nn;
-      float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      if (k < kend && n + 7 < N) {
-        const uint4 u = *reinterpret_cast<const uint4*>(b + static_cast<size_t>(k) * ldb + n);
-        unpack8(u, f);
-      }
-      *reinterpret_cast<float4*>(&Bs[kk][nn]) = make_float4(f[0], f[1], f[2], f[3]);
-      *reinterpret_cast<float4*>(&Bs[kk][nn + 4]) = make_float4(f[4], f[5], f[6], f[7]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < SG_K; ++kk) {
-      float av[8], bv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) av[i] = As[kk][ty + 16 * i];
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][4 * tx + 64]);
-      bv[0] = b0.x; bv[1] = b0.y; bv[2] = b0.z; bv[3] = b0.w;
-      bv[4] = b1.x; bv[5] = b1.y; bv[6] = b1.z; bv[7] = b1.w;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
+  extern __shared__ float s_v[];            // [32][E + 1]
+  const int ld = E + 1;
+  const int t0 = blockIdx.x * 32;
+  if (blockIdx.x == 0)
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) goff[g] = g * 3 * Ep;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) {
+    const int r = i / E, e = i - r * E;
+    s_v[r * ld + e] = t0 + r < T ? dlogits[static_cast<size_t>(t0 + r) * E + e] : 0.f;
   }
-  float* out = part + static_cast<size_t>(blockIdx.z) * M * N;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int m = m0 + ty + 16 * i;
-    if (m >= M) continue;
-    float* row = out + static_cast<size_t>(m) * N + n0 + 4 * tx;
-    *reinterpret_cast<float4*>(row) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-    *reinterpret_cast<float4*>(row + 64) =
-        make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+  __syncthreads();
+  const int C3 = 3 * Ep;
+  auto term = [](float v, int j) {
+    const __nv_bfloat16 h1 = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(h1);
+    if (j == 0) return h1;
+    const __nv_bfloat16 h2 = __float2bfloat16_rn(r1);
+    if (j == 1) return h2;
+    return __float2bfloat16_rn(r1 - __bfloat162float(h2));
+  };
+  for (int i = threadIdx.x; i < 32 * C3; i += blockDim.x) {
+    const int r = i / C3, c = i - r * C3;
+    if (t0 + r >= T) continue;
+    const int j = c / Ep, e = c - j * Ep;
+    adx[static_cast<size_t>(t0 + r) * C3 + c] = term(e < E ? s_v[r * ld + e] : 0.f, j);
+  }
+  const int g = t0 / Ks, k0 = t0 - g * Ks;
+  for (int i = threadIdx.x; i < C3 * 32; i += blockDim.x) {
+    const int row = i >> 5, r = i & 31;
+    const int j = row / Ep, e = row - j * Ep;
+    adw[(static_cast<size_t>(g) * C3 + row) * Ks + k0 + r] =
+        term(e < E ? s_v[r * ld + e] : 0.f, j);
   }
 }
 
-// out[i] = sum_z part[z][i] (fixed order)
+// out[e, n] = sum_g sum_j part[g * 3 Ep + j * Ep + e, n]  (g, then j: a fixed
+// order)
 __global__ void __launch_bounds__(256)
-sum_slices_kernel(const float* __restrict__ part, int slices, long long n,
-                  float* __restrict__ out) {
+router_grad_reduce_kernel(const float* __restrict__ part, int G, int E, int Ep, int d,
+                          float* __restrict__ out) {
   pdl_trigger();
   pdl_wait();
+  const long long n = static_cast<long long>(E) * d;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    float s = 0.f;
-    for (int z = 0; z < slices; ++z) s += part[z * n + i];
-    out[i] = s;
+    const long long e = i / d, c = i - e * d;
+    float acc = 0.f;
+    for (int g = 0; g < G; ++g)
+      for (int j = 0; j < 3; ++j)
+        acc += part[(static_cast<long long>(g) * 3 * Ep + j * Ep + e) * d + c];
+    out[i] = acc;
   }
 }
 
@@ -488,27 +443,37 @@ cudaError_t router_dlogits(const float* logits, const float* offset, const int32
                     dlogits);
 }
 
-int sgemm_slices(int K) {
-  int s = (K + 1023) / 1024;
-  return s < 1 ? 1 : (s > 16 ? 16 : s);
+RouterGradShape router_grad_shape(int T, int E) {
+  RouterGradShape r;
+  r.Ep = (E + 63) / 64 * 64;
+  // token slices of the dW GEMM: about 16, each a multiple of 64 tokens
+  r.Ks = ((T + 15) / 16 + 63) / 64 * 64;
+  if (r.Ks < 64) r.Ks = 64;
+  r.G = (T + r.Ks - 1) / r.Ks;
+  return r;
 }
 
-cudaError_t sgemm_f32(bool a_t, const float* a, int lda, const void* b, int ldb, int M, int N,
-                      int K, float* part, float* out, cudaStream_t stream) {
-  if (N % SG_T || ldb % 8) return cudaErrorInvalidValue;
-  const int slices = sgemm_slices(K);
-  const int kslice = ((K + slices - 1) / slices + SG_K - 1) / SG_K * SG_K;
-  const dim3 grid(N / SG_T, (M + SG_T - 1) / SG_T, slices);
-  if (slices == 1) part = out;   // one slice: the partial sum is the result
-  cudaError_t e =
-      a_t ? launch_pdl(sgemm_kernel<true>, grid, dim3(256), 0, stream, a, lda,
-                       static_cast<const __nv_bfloat16*>(b), ldb, M, N, K, kslice, part)
-          : launch_pdl(sgemm_kernel<false>, grid, dim3(256), 0, stream, a, lda,
-                       static_cast<const __nv_bfloat16*>(b), ldb, M, N, K, kslice, part);
-  if (e != cudaSuccess || slices == 1) return e;
-  const long long n = static_cast<long long>(M) * N;
-  return launch_pdl(sum_slices_kernel, dim3(grid_1d(n)), dim3(256), 0, stream, part, slices, n,
-                    out);
+cudaError_t router_grad_split(const float* dlogits, int T, int E, const RouterGradShape& r,
+                              void* adx, void* adw, int32_t* goff, cudaStream_t stream) {
+  const size_t smem = static_cast<size_t>(32) * (E + 1) * sizeof(float);
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(router_grad_split_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  // every column of every slice is written, zeros past T
+  const int blocks = r.G * r.Ks / 32;
+  return launch_pdl(router_grad_split_kernel, dim3(blocks), dim3(256), smem, stream, dlogits, T,
+                    E, r.Ep, r.Ks, r.G, static_cast<__nv_bfloat16*>(adx),
+                    static_cast<__nv_bfloat16*>(adw), goff);
+}
+
+cudaError_t router_grad_reduce(const float* part, const RouterGradShape& r, int E, int d,
+                               float* out, cudaStream_t stream) {
+  const long long n = static_cast<long long>(E) * d;
+  return launch_pdl(router_grad_reduce_kernel, dim3(grid_1d(n)), dim3(256), 0, stream, part,
+                    r.G, E, r.Ep, d, out);
 }
 
 }  // namespace moe

@@ -54,6 +54,9 @@ constexpr int MODE_SWIGLU_BF16 = 1;   // C = silu(A B0^T) * (A B1^T), rounded to
 // bf16; the K rows of a group come from B0 (the first kb_split k-blocks) and
 // then from B1, so [W1; W3] needs no concatenated copy.
 constexpr int MODE_PLAIN_BMN = 2;
+// As MODE_PLAIN_BMN with fp32 output, stored row by row from the registers
+// (the router's gradient products, whose sums stay in fp32).
+constexpr int MODE_PLAIN_BMN_F32 = 3;
 
 struct GemmArgs {
   const int32_t* offsets;  // [G+1] device, or nullptr: one group [0, rows_single)
@@ -245,7 +248,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   using Cfg = PairCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
-  constexpr bool BMN = MODE == MODE_PLAIN_BMN;
+  constexpr bool BMN = MODE == MODE_PLAIN_BMN || MODE == MODE_PLAIN_BMN_F32;
+  constexpr bool OUT_F32 = MODE == MODE_PLAIN_BMN_F32;
   constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
   constexpr int NSUB = Cfg::NSUB;
   constexpr int NACC = Cfg::NACC;
@@ -511,12 +515,25 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             tmem_ld16(t_addr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
             tmem_ld16(t_addr + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&v[16]));
             tmem_ld_wait();
+            if constexpr (OUT_F32) {
+              if (valid) {
+                float4* dst = reinterpret_cast<float4*>(
+                    static_cast<float*>(pt.x ? args.x_C : args.C) + crow_off + ocol + half * 32);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              packed[half * 16 + i] =
-                  pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                for (int i = 0; i < 8; ++i)
+                  dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                       __uint_as_float(v[4 * i + 2]),
+                                       __uint_as_float(v[4 * i + 3]));
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                packed[half * 16 + i] =
+                    pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
           }
         }
+        if constexpr (OUT_F32) continue;   // stored above
         if (warp_full) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -784,6 +801,29 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
                                              rows_upper, stream);
   return launch_pair<128, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args,
                                            rows_upper, stream);
+}
+
+// Y [rows, N] fp32 = A B_g over the groups of A's rows, B_g the rows
+// [g b0_rows, g b0_rows + K) of B0 [b0_total_rows, N] (MN-major; rows past
+// b0_total_rows read as zero).  K = b0_rows, a multiple of 64; N a multiple
+// of 128.
+cudaError_t grouped_gemm_bmn_f32out(const void* A, int64_t a_rows, const int32_t* offsets,
+                                    int num_groups, int rows_single, const void* B0,
+                                    int b0_rows, int64_t b0_total_rows, int N, float* Y,
+                                    uint32_t* status, cudaStream_t stream) {
+  const int K = b0_rows;
+  if (K % BK || K <= 0 || N % 128 || b0_total_rows <= 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb0;
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, B0, b0_total_rows, N, BK))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
+                K / BK, K, 0, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
+  const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (N % 256 == 0)
+    return launch_pair<256, MODE_PLAIN_BMN_F32>(ta, tb0, tb0, ta, ta, tb0, tb0, ta, args,
+                                                rows_upper, stream);
+  return launch_pair<128, MODE_PLAIN_BMN_F32>(ta, tb0, tb0, ta, ta, tb0, tb0, ta, args,
+                                              rows_upper, stream);
 }
 
 // Y[r] = A[r] B_g with B_g stored [K, N] (MN-major): its first b0_rows rows

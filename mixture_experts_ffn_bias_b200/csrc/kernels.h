@@ -130,6 +130,12 @@ cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* 
                                   int num_groups, int rows_single, const void* B0,
                                   const void* B1, int b0_rows, int N, int K, void* Y,
                                   uint32_t* status, cudaStream_t stream);
+// fp32 output variant, all K rows from B0 (group g: rows [g K, g K + K),
+// rows at or past b0_total_rows read as zero).
+cudaError_t grouped_gemm_bmn_f32out(const void* A, int64_t a_rows, const int32_t* offsets,
+                                    int num_groups, int rows_single, const void* B0,
+                                    int b0_rows, int64_t b0_total_rows, int N, float* Y,
+                                    uint32_t* status, cudaStream_t stream);
 cudaError_t grouped_swiglu_gateup_f32(const float* A, int64_t a_rows, const int32_t* offsets,
                                       int num_groups, int rows_single, const float* W1,
                                       const float* W3, int F, int K, float* H,
@@ -159,11 +165,18 @@ cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr
 cudaError_t router_dlogits(const float* logits, const float* offset, const int32_t* topk_idx,
                            const float* topk_w, const float* dw, int T, int E, int k, int gate,
                            int renorm, float* dlogits, cudaStream_t stream);
-int sgemm_slices(int K);
-// out [M, N] fp32 = A B with A(m, k) fp32 (a_t: stored [K, M]) and B [K, N] bf16;
-// part holds sgemm_slices(K) x M x N partial sums (unused when that is 1).
-cudaError_t sgemm_f32(bool a_t, const float* a, int lda, const void* b, int ldb, int M, int N,
-                      int K, float* part, float* out, cudaStream_t stream);
+// Router gradients on the tensor cores: dlogits split into three bf16 terms
+// (exact), Ep = E rounded up to 64, G token slices of Ks tokens for dW.
+struct RouterGradShape {
+  int Ep, Ks, G;
+};
+RouterGradShape router_grad_shape(int T, int E);
+// adx [T, 3 Ep] and adw [G, 3 Ep, Ks] bf16, goff [G + 1] = g * 3 Ep.
+cudaError_t router_grad_split(const float* dlogits, int T, int E, const RouterGradShape& r,
+                              void* adx, void* adw, int32_t* goff, cudaStream_t stream);
+// out [E, d] fp32 = sum over slices and terms of part [G, 3 Ep, d].
+cudaError_t router_grad_reduce(const float* part, const RouterGradShape& r, int E, int d,
+                               float* out, cudaStream_t stream);
 
 // Combine / bias ---------------------------------------------------------------
 cudaError_t combine(bool bf16, const void* y_perm, const int32_t* slot_pos, const float* topk_w,

@@ -298,7 +298,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
 
 // Workspace of moe_backward (separate from the forward's, which it reads).
 struct BLayout {
-  size_t status, dw, logits, dlogits, part, dxr, poff, poff_sh, dy, dh, gb, ub, dgu, dxp, dyT,
+  size_t status, dw, logits, dlogits, adx, adw, wr3, pdw, goff, dxr, poff, poff_sh, dy, dh, gb,
+      ub, dgu, dxp, dyT,
       hT, dguT, xT, dh_sh, g_sh, u_sh, dgu_sh, dxs, doutT, hshT, dgushT, xTs, total;
   int64_t kp, tp;
 };
@@ -317,7 +318,13 @@ BLayout blayout(const moe_config& c) {
   B.dw = o;      o += up(R * 4);
   B.logits = o;  o += up(T * E * 4);
   B.dlogits = o; o += up(T * E * 4);
-  B.part = o;    o += up(static_cast<size_t>(moe::sgemm_slices(c.T)) * E * d * 4);
+  const moe::RouterGradShape rg = moe::router_grad_shape(c.T, c.n_experts);
+  const size_t C3 = 3 * static_cast<size_t>(rg.Ep), Gs = rg.G, Ks = rg.Ks;
+  B.adx = o;     o += up(T * C3 * 2);
+  B.adw = o;     o += up(Gs * C3 * Ks * 2);
+  B.wr3 = o;     o += up(C3 * d * 2);
+  B.pdw = o;     o += up(Gs * C3 * d * 4);
+  B.goff = o;    o += up((Gs + 1) * 4);
   B.dxr = o;     o += up(T * d * 4);
   B.poff = o;    o += up((E + 1) * 4);
   B.poff_sh = o; o += up(2 * 4);
@@ -433,16 +440,33 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
                                     at<void>(bws, B.xTs), tp, poff_sh, 1, Fs, d, g->dws3, status,
                                     s));
   }
-  // router (fp32): recomputed logits, dlogits, dW_router = dlogits^T x,
-  // dx_router = dlogits W_router
+  // router (fp32): recomputed logits, dlogits, then on the tensor cores
+  // with dlogits as three exact bf16 terms: dx_router = dlogits Wr (K = 3 Ep,
+  // Wr repeated per term) and dW_router = dlogits^T x (G token slices as
+  // GEMM groups, fp32 partials summed in a fixed order)
   float* logits = at<float>(bws, B.logits);
   float* dlogits = at<float>(bws, B.dlogits);
   MOE_TRY(moe::router_logits_tc(x, T, w_router, E, d, logits, status, s));
   MOE_TRY(moe::router_dlogits(logits, logit_offset, topk_idx, topk_w, dw, T, E, k, c->gate,
                               c->norm_topk_prob, dlogits, s));
-  MOE_TRY(moe::sgemm_f32(true, dlogits, E, x, d, E, d, T, at<float>(bws, B.part), dw_router, s));
-  MOE_TRY(moe::sgemm_f32(false, dlogits, E, w_router, d, T, d, E, at<float>(bws, B.part),
-                         at<float>(bws, B.dxr), s));
+  const moe::RouterGradShape rg = moe::router_grad_shape(T, E);
+  const int C3 = 3 * rg.Ep;
+  uint8_t* wr3 = at<uint8_t>(bws, B.wr3);
+  const size_t wr_bytes = static_cast<size_t>(E) * d * 2;
+  for (int j = 0; j < 3; ++j) {
+    uint8_t* dst = wr3 + static_cast<size_t>(j) * rg.Ep * d * 2;
+    MOE_TRY(cudaMemcpyAsync(dst, w_router, wr_bytes, cudaMemcpyDeviceToDevice, s));
+    if (rg.Ep > E)
+      MOE_TRY(cudaMemsetAsync(dst + wr_bytes, 0, static_cast<size_t>(rg.Ep - E) * d * 2, s));
+  }
+  MOE_TRY(moe::router_grad_split(dlogits, T, E, rg, at<void>(bws, B.adx), at<void>(bws, B.adw),
+                                 at<int32_t>(bws, B.goff), s));
+  MOE_TRY(moe::grouped_gemm_bmn_f32out(at<void>(bws, B.adx), T, nullptr, 1, T, wr3, C3, C3, d,
+                                       at<float>(bws, B.dxr), status, s));
+  MOE_TRY(moe::grouped_gemm_bmn_f32out(at<void>(bws, B.adw), static_cast<int64_t>(rg.G) * C3,
+                                       at<int32_t>(bws, B.goff), rg.G, 0, x, rg.Ks, T, d,
+                                       at<float>(bws, B.pdw), status, s));
+  MOE_TRY(moe::router_grad_reduce(at<float>(bws, B.pdw), rg, E, d, dw_router, s));
   MOE_TRY(moe::dx_gather(at<void>(bws, B.dxp), slot_pos, at<float>(bws, B.dxr), dxs, dx, T, d, k,
                          s));
   return MOE_OK;
