@@ -83,6 +83,105 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
   }
 }
 
+// The rank kernel with the scan folded in: each block, once its counts are
+// out, takes a ticket; the last block to finish turns all block counts into
+// block bases, counts and offsets (the same arithmetic as the scan kernel
+// below), then puts the ticket counter back to zero.  done: zero at launch.
+__global__ void __launch_bounds__(kRankBlock)
+dispatch_rank_scan_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
+                          int32_t* __restrict__ blk, int32_t* __restrict__ rank_out,
+                          int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                          uint32_t* __restrict__ status, uint32_t* __restrict__ done) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ uint32_t masks[kMaxE][kWords];
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, word = tid >> 5;
+  const int t = blockIdx.x * kRankBlock + tid;
+  for (int i = tid; i < E * kWords; i += kRankBlock) masks[i / kWords][i % kWords] = 0u;
+  __syncthreads();
+  const int32_t* row = topk_idx + static_cast<size_t>(t) * k;
+  bool bad = false;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      if (pair_valid(row, j, E))
+        atomicOr(&masks[row[j]][word], 1u << lane);
+      else
+        bad = true;
+    }
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      int r = -1;
+      if (pair_valid(row, j, E)) {
+        const int e = row[j];
+        r = __popc(masks[e][word] & below);
+        for (int w = 0; w < word; ++w) r += __popc(masks[e][w]);
+      }
+      rank_out[static_cast<size_t>(t) * k + j] = r;
+    }
+  }
+  if (bad) atomicOr(status, kDevBadIndex);
+  for (int e = tid; e < E; e += kRankBlock) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWords; ++w) c += __popc(masks[e][w]);
+    blk[static_cast<size_t>(blockIdx.x) * E + e] = c;
+  }
+  __threadfence();   // this block's counts are visible before its ticket
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(done, 1u) == gridDim.x - 1 ? 1 : 0;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // the scan: thread e walks expert e's column of block counts (read from
+  // L2, sixteen loads in flight), then a block scan over the experts
+  const int nblk = gridDim.x;
+  int* s = reinterpret_cast<int*>(masks);   // kMaxE ints of the mask space
+  const int e = tid;
+  int run = 0;
+  if (e < E) {
+    for (int b0 = 0; b0 < nblk; b0 += 16) {
+      int c[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        c[u] = b0 + u < nblk ? __ldcg(blk + static_cast<size_t>(b0 + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) run += c[u];
+    }
+    counts[e] = run;
+  }
+  s[e] = e < E ? run : 0;
+  __syncthreads();
+  for (int o = 1; o < kMaxE; o <<= 1) {          // inclusive Hillis-Steele scan
+    const int v = (e >= o) ? s[e - o] : 0;
+    __syncthreads();
+    s[e] += v;
+    __syncthreads();
+  }
+  const int excl = s[e] - (e < E ? run : 0);
+  if (e < E) offsets[e] = excl;
+  if (e == kMaxE - 1) offsets[E] = s[e];
+  if (e < E) {
+    int base = excl;
+    for (int b0 = 0; b0 < nblk; b0 += 16) {
+      int c[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        c[u] = b0 + u < nblk ? __ldcg(blk + static_cast<size_t>(b0 + u) * E + e) : 0;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        if (b0 + u < nblk) blk[static_cast<size_t>(b0 + u) * E + e] = base;
+        base += c[u];
+      }
+    }
+  }
+  if (tid == 0) *done = 0u;
+}
+
 // Block counts [nblk, E] -> block bases (in place), counts and offsets.  The
 // counts are staged in shared memory when they fit (kScanSmemInts), so the
 // per-expert running sums walk shared memory instead of global memory.
@@ -212,6 +311,14 @@ cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t*
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream) {
   return launch_pdl(dispatch_rank_kernel, dim3(rank_blocks(T)), dim3(kRankBlock), 0, stream,
                     topk_idx, T, k, E, blk_counts, rank_out, status);
+}
+
+cudaError_t dispatch_rank_scan(const int32_t* topk_idx, int T, int k, int E, int32_t* blk,
+                               int32_t* rank_out, int32_t* counts, int32_t* offsets,
+                               uint32_t* status, uint32_t* done, cudaStream_t stream) {
+  if (E > kMaxE || kRankBlock != kMaxE) return cudaErrorInvalidValue;
+  return launch_pdl(dispatch_rank_scan_kernel, dim3(rank_blocks(T)), dim3(kRankBlock), 0, stream,
+                    topk_idx, T, k, E, blk, rank_out, counts, offsets, status, done);
 }
 
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,

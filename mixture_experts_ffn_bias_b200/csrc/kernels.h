@@ -76,6 +76,11 @@ constexpr int kRankBlock = 256;   // tokens per histogram block
 inline int rank_blocks(int T) { return (T + kRankBlock - 1) / kRankBlock; }
 cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream);
+// dispatch_rank followed by dispatch_scan in one launch (the last block to
+// finish scans); done: a zeroed counter, zero again when the kernel ends.
+cudaError_t dispatch_rank_scan(const int32_t* topk_idx, int T, int k, int E, int32_t* blk,
+                               int32_t* rank_out, int32_t* counts, int32_t* offsets,
+                               uint32_t* status, uint32_t* done, cudaStream_t stream);
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream);
 // slot_pos (in: rank inside its block of blk_tokens tokens, out: row) and

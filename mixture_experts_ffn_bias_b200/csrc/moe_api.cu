@@ -27,9 +27,8 @@ Layout layout(const moe_config& c) {
   const size_t Fs = c.n_shared ? static_cast<size_t>(c.d_ff_shared) : 0;
   Layout L{};
   size_t o = 0;
-  // status area: word 0 device status, word 1 tokens re-decided by the
-  // router
-  L.status = o;   o += up(3 * sizeof(uint32_t));
+  // status area: four words (see clear_status)
+  L.status = o;   o += up(4 * sizeof(uint32_t));
   L.blk = o;      o += up(static_cast<size_t>(moe::rank_blocks(c.T)) * E * 4);
   L.offsets = o;  o += up((E + 1) * 4);
   L.slot_pos = o; o += up(R * 4);
@@ -91,9 +90,10 @@ inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Word 0: device status flags; word 1: number of tokens the router listed
 // for exact re-decision; word 2: non-zero when the last forward kept no
-// permuted copy of x (gathered gate/up rows).
+// permuted copy of x (gathered gate/up rows); word 3: the rank kernel's
+// count of finished blocks.
 moe_status clear_status(void* ws, cudaStream_t s) {
-  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, 3 * sizeof(uint32_t), s));
+  MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, 0), 0, 4 * sizeof(uint32_t), s));
   return MOE_OK;
 }
 
@@ -148,9 +148,8 @@ moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void*
   const Layout L = layout(*c);
   int32_t* blk = at<int32_t>(ws, L.blk);
   uint32_t* status = at<uint32_t>(ws, L.status);
-  const int nblk = moe::rank_blocks(c->T);
-  MOE_TRY(moe::dispatch_rank(topk_idx, c->T, c->top_k, c->n_experts, blk, slot_pos, status, s));
-  MOE_TRY(moe::dispatch_scan(blk, nblk, c->n_experts, counts, offsets, s));
+  MOE_TRY(moe::dispatch_rank_scan(topk_idx, c->T, c->top_k, c->n_experts, blk, slot_pos, counts,
+                                  offsets, status, status + 3, s));
   if (x_perm == nullptr) {   // rows only; the experts gather x through perm_src
     MOE_TRY(moe::dispatch_positions(topk_idx, blk, slot_pos, perm_src, c->T, c->top_k,
                                     c->n_experts, moe::kRankBlock, s));

@@ -369,9 +369,12 @@ router_select_fast_kernel(const float* __restrict__ logits, const float* __restr
   }
 }
 
-// Exact re-decision of listed tokens: one block per listed token, x staged
-// in shared memory as fp32, each warp reading two router rows at a time
-// (the decision itself is refine_select of router_exact.cuh).
+// Exact re-decision of listed tokens: one block per listed token.  The
+// chain of dependent memory accesses is kept short: the list length, then the
+// token and its candidate experts together, then the x row and the router
+// rows together (every warp loads the token's x row into registers and each
+// of its candidates' rows in full before it multiplies), then the decision
+// (refine_select of router_exact.cuh) by warp 0.
 __global__ void __launch_bounds__(256)
 router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
                      const float* __restrict__ offset, const float* __restrict__ bias, int d,
@@ -382,62 +385,60 @@ router_refine_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* _
                      float* __restrict__ topk_w) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float4 s_x4[];          // d floats
-  float* s_x = reinterpret_cast<float*>(s_x4);
+  constexpr int kVecs = 8;                  // 16-byte pieces of a row per lane held at once
   __shared__ double s_l[256];
   __shared__ int s_e[256];
-  __shared__ int s_n;
+  __shared__ int s_n, s_t, s_all;
   const int n_list = *refine_count;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nv = d / 8;                     // 16-byte pieces of a row
   for (int i = blockIdx.x; i < n_list; i += gridDim.x) {
-    const int t = refine_list[i];
-    const int32_t* cand = refine_cand ? refine_cand + static_cast<size_t>(i) * kRefineCand : nullptr;
-    const bool all = cand == nullptr || cand[0] == -2;
-    if (threadIdx.x == 0) {
-      int n = E;
-      if (!all) {
-        n = 0;
-        while (n < kRefineCand && cand[n] >= 0) ++n;
+    if (warp == 0) {
+      // the token and its candidates (a prefix of the list row, -1 after it;
+      // -2 first: all experts) are read together
+      const int t = refine_list[i];
+      int ce = -1;
+      if (refine_cand && lane < kRefineCand) ce = refine_cand[static_cast<size_t>(i) * kRefineCand + lane];
+      const bool all = refine_cand == nullptr || __shfl_sync(0xffffffffu, ce, 0) == -2;
+      const int n = all ? E : __popc(__ballot_sync(0xffffffffu, ce >= 0));
+      if (!all && lane < kRefineCand) s_e[lane] = ce;
+      if (lane == 0) {
+        s_n = n;
+        s_t = t;
+        s_all = all ? 1 : 0;
       }
-      s_n = n;
     }
-    for (int c = threadIdx.x; c < 256; c += blockDim.x)
-      s_e[c] = all ? c : (c < kRefineCand ? cand[c] : -1);
-    for (int c = threadIdx.x; c < d; c += blockDim.x)
-      s_x[c] = __bfloat162float(x[static_cast<size_t>(t) * d + c]);
     __syncthreads();
-    const int n = s_n;
-    const float4* sx4 = reinterpret_cast<const float4*>(s_x);
-    for (int c0 = warp; c0 < n; c0 += 16) {
-      const int c1 = c0 + 8;
-      const int e0 = s_e[c0], e1 = c1 < n ? s_e[c1] : e0;
-      const uint4* r0 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e0) * d);
-      const uint4* r1 = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e1) * d);
-      double a[4] = {0.0, 0.0, 0.0, 0.0}, b[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-      for (int col = lane * 8; col < d; col += 256) {
-        const uint4 u0 = __ldg(r0 + col / 8), u1 = __ldg(r1 + col / 8);
-        const float4 xa = sx4[col / 4], xb = sx4[col / 4 + 1];
-        const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        const __nv_bfloat16* h0 = reinterpret_cast<const __nv_bfloat16*>(&u0);
-        const __nv_bfloat16* h1 = reinterpret_cast<const __nv_bfloat16*>(&u1);
+    const int n = s_n, t = s_t;
+    const bool all = s_all != 0;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+    for (int c = warp; c < n; c += 8) {
+      const int e = all ? c : s_e[c];
+      const uint4* wrow = reinterpret_cast<const uint4*>(wr + static_cast<size_t>(e) * d);
+      double a[4] = {0.0, 0.0, 0.0, 0.0};
+      for (int v0 = lane; v0 < nv; v0 += 32 * kVecs) {
+        uint4 ux[kVecs], uw[kVecs];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // bf16 x bf16 products are exact in fp32; the sums run in fp64
-          a[j & 3] += static_cast<double>(__bfloat162float(h0[j]) * xv[j]);
-          b[j & 3] += static_cast<double>(__bfloat162float(h1[j]) * xv[j]);
+        for (int u = 0; u < kVecs; ++u) {
+          const int v = v0 + 32 * u;
+          ux[u] = v < nv ? __ldg(xr + v) : make_uint4(0u, 0u, 0u, 0u);
+          uw[u] = v < nv ? __ldg(wrow + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kVecs; ++u) {
+          const __nv_bfloat16* hx = reinterpret_cast<const __nv_bfloat16*>(&ux[u]);
+          const __nv_bfloat16* hw = reinterpret_cast<const __nv_bfloat16*>(&uw[u]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)   // bf16 x bf16 products are exact in fp32; fp64 sums
+            a[j & 3] += static_cast<double>(__bfloat162float(hw[j]) * __bfloat162float(hx[j]));
         }
       }
-      double s0 = (a[0] + a[1]) + (a[2] + a[3]);
-      double s1 = (b[0] + b[1]) + (b[2] + b[3]);
+      double sum = (a[0] + a[1]) + (a[2] + a[3]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      }
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (lane == 0) {
-        s_l[c0] = s0 + (offset ? static_cast<double>(offset[e0]) : 0.0);
-        if (c1 < n) s_l[c1] = s1 + (offset ? static_cast<double>(offset[e1]) : 0.0);
+        s_l[c] = sum + (offset ? static_cast<double>(offset[e]) : 0.0);
+        if (all) s_e[c] = c;
       }
     }
     __syncthreads();
@@ -507,14 +508,7 @@ cudaError_t router_refine(const void* x, const void* w_router, const float* logi
   int grid = 2 * sms;
   if (grid > T) grid = T;
   if (grid < 1) grid = 1;
-  const size_t smem = static_cast<size_t>(d) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(router_refine_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  return launch_pdl(router_refine_kernel, dim3(grid), dim3(256), smem, stream,
+  return launch_pdl(router_refine_kernel, dim3(grid), dim3(256), 0, stream,
                     static_cast<const __nv_bfloat16*>(x),
                     static_cast<const __nv_bfloat16*>(w_router), logit_offset, sel_bias, d, E, k,
                     gate, renorm, ko.space, ko.noise, refine_count, refine_list, refine_cand,
