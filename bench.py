@@ -53,6 +53,26 @@ def layer_flops(s: I.MoEShape) -> dict:
     }
 
 
+# DRAM bytes per launch of the routed gate/up GEMM, from the ncu capture in
+# profiles/grouped_gemm_gateup_qwen3_30b.md, and the kernel source it was
+# taken on (sha256 of csrc/grouped_gemm_sm100.cu, first 16 hex digits).
+GATEUP_TRAFFIC = {"qwen3_30b": (1537016064, "8281548d44192e04")}
+
+
+def traffic_note(s: I.MoEShape) -> str:
+    import hashlib
+    src = os.path.join(ROOT, "mixture_experts_ffn_bias_b200", "csrc", "grouped_gemm_sm100.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if s.name not in GATEUP_TRAFFIC:
+        return "not measured in this run; no ncu capture of this workload's gate/up launch"
+    nbytes, at = GATEUP_TRAFFIC[s.name]
+    same = "the same source" if sha == at else f"an older source (now {sha})"
+    return (f"not measured in this run; {nbytes} DRAM bytes per launch in the ncu capture of "
+            f"profiles/grouped_gemm_gateup_qwen3_30b.md, taken on kernel source {at} "
+            f"({same})")
+
+
 def describe(s: I.MoEShape) -> str:
     gate = "softmax" if s.gate == I.GATE_SOFTMAX else "sigmoid"
     dt = "bf16" if s.dtype == I.DTYPE_BF16 else "fp32"
@@ -483,8 +503,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
                          "frac_of_sustained": achieved / sus,
                          "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
                          "traffic": None,
-                         "traffic_note": "not measured in this run; per-launch DRAM bytes of "
-                                         "an ncu capture are in profiles/"},
+                         "traffic_note": traffic_note(shape)},
             "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": layer.x.numel() * layer.x.element_size(),
                     "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size(),
