@@ -378,13 +378,17 @@ const char* moe_status_string(moe_status s);
  * topk_w (as moe_forward returned them) and dout [T, d] act.  fws is the
  * workspace of that moe_forward (or moe_forward_ex) call, unchanged since
  * (the backward reads the routed order and the saved activations h and y
- * from it; x's rows are gathered again by the permutation).  bws: backward scratch of moe_backward_workspace_size(cfg) bytes,
+ * from it, and x_perm unless that forward gathered its rows).  bws:
+ * backward scratch of moe_backward_workspace_size(cfg) bytes,
  * 256-byte aligned; its first word is a device status word read with
  * moe_device_status(bws, ...).
  * Outputs: dx [T, d] act; dw_router [E, d] fp32; g->dw1, dw3 [E, F, d],
  * dw2 [E, d, F] act (and the shared expert's).  Activation gradients are
- * bf16 between the steps, the contractions accumulate in fp32 (tensor cores;
- * the router's on CUDA cores in fp32). */
+ * bf16 between the steps, the contractions accumulate in fp32 on the tensor
+ * cores.  The router's dlogits stay fp32: its two products run with dlogits
+ * written as three bf16 terms whose sum is the fp32 value to within fp32
+ * rounding, so every product with the bf16 x or w_router is exact and the
+ * fp32 accumulation is the only rounding. */
 size_t moe_backward_workspace_size(const moe_config* cfg);
 moe_status moe_backward(const moe_config* cfg, const void* x, const void* w_router,
                         const float* logit_offset, const moe_expert_weights* w,
