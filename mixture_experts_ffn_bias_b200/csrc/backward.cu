@@ -4,9 +4,6 @@
 // GEMM of grouped_gemm_wgrad_sm100.cu for the weight gradients); this file
 // holds what feeds and finishes them:
 //   bwd_dy_kernel       dw[t, j] = <dout[t], y_perm[slot]>, dY[slot] = w[t, j] dout[t]
-//   gtranspose_kernel   rows of each group -> padded columns (the K-grouped
-//                       operands), zeros in the padding
-//   pad_offsets_kernel  padded column offsets of the groups
 //   swiglu_bwd_kernel   dG = dH * U * silu'(G), dU = dH * silu(G)
 //   dx_gather_kernel    dx[t] = sum_j dX[slot(t, j)] + dx_router[t] (+ dx_shared[t])
 //   router_dlogits_kernel  dlogits from dw through the (renormalised) gate
@@ -84,98 +81,6 @@ bwd_dy_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y_perm,
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     if (lane == 0) dw[p] = dot;
   }
-}
-
-// Transposes move 64 x 64 bf16 tiles through shared memory: 16-byte global
-// loads of the source rows (a warp reads four full 128-byte rows), and
-// 128-byte output rows written as bf16 pairs by a warp.  The tile's rows are
-// 66 elements apart (33 words), so the column reads hit at most two lanes
-// per bank.  All dimensions here are multiples of 64 (bf16 layers have d, F
-// multiples of 128; padded column counts are multiples of 64).
-constexpr int TT = 64;
-constexpr int TROW = TT + 2;
-
-// Loads source rows src_row(i), i < 64 (negative: zeros), columns [c0, c0+64).
-__device__ __forceinline__ void load_tile(uint16_t (*tile)[TROW], const __nv_bfloat16* in,
-                                          int cols, int c0, const int* src_row) {
-  for (int idx = threadIdx.x; idx < TT * 8; idx += blockDim.x) {
-    const int i = idx >> 3, v = idx & 7;
-    const int src = src_row[i];
-    uint4 u = make_uint4(0u, 0u, 0u, 0u);
-    if (src >= 0)
-      u = *reinterpret_cast<const uint4*>(in + static_cast<size_t>(src) * cols + c0 + v * 8);
-    uint32_t* t = reinterpret_cast<uint32_t*>(&tile[i][v * 8]);
-    t[0] = u.x; t[1] = u.y; t[2] = u.z; t[3] = u.w;
-  }
-}
-
-// Writes out[(c0 + c) * ldo + base + i] = tile[i][c] for c, i < 64.
-__device__ __forceinline__ void store_tile_t(const uint16_t (*tile)[TROW], __nv_bfloat16* out,
-                                             long long ldo, long long base, int c0) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int c = warp; c < TT; c += nw) {
-    const uint32_t lo = tile[2 * lane][c], hi = tile[2 * lane + 1][c];
-    reinterpret_cast<uint32_t*>(out + (c0 + c) * ldo + base)[lane] = lo | (hi << 16);
-  }
-}
-
-// out[b][c][col_off + r] = in[b][r][c] for r < rows, c < cols.
-// Padded column offsets: poff[g + 1] = poff[g] + roundup(rows_g, 64).
-// offsets null: one group of rows_single rows.
-__global__ void pad_offsets_kernel(const int32_t* __restrict__ offsets, int G, int rows_single,
-                                   int32_t* __restrict__ poff) {
-  pdl_trigger();
-  pdl_wait();
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int run = 0;
-  poff[0] = 0;
-  for (int g = 0; g < G; ++g) {
-    const int rows = offsets ? offsets[g + 1] - offsets[g] : rows_single;
-    run += (rows + 63) / 64 * 64;
-    poff[g + 1] = run;
-  }
-}
-
-// out [cols, kp]: column p of out is row src(p) of in [rows, cols], where
-// p = poff[g] + i < poff[g] + rows_g maps to row offsets[g] + i (gathered
-// through `gather` when not null), and every other p is zero.  The grid
-// covers kp x cols in 64 x 64 tiles; the group offsets are staged in shared
-// memory for the per-position search.
-__global__ void __launch_bounds__(256)
-gtranspose_kernel(const __nv_bfloat16* __restrict__ in, int cols,
-                  const int32_t* __restrict__ offsets, int G, int rows_single,
-                  const int32_t* __restrict__ poff, const int32_t* __restrict__ gather,
-                  __nv_bfloat16* __restrict__ out, int kp) {
-  pdl_trigger();
-  pdl_wait();
-  __shared__ __align__(16) uint16_t tile[TT][TROW];
-  __shared__ int s_poff[258];
-  __shared__ int s_off[258];
-  __shared__ int s_src[TT];
-  const int p0 = blockIdx.x * TT, c0 = blockIdx.y * TT;
-  for (int g = threadIdx.x; g <= G; g += blockDim.x) {
-    s_poff[g] = poff[g];
-    s_off[g] = offsets ? offsets[g] : (g == 0 ? 0 : rows_single);
-  }
-  __syncthreads();
-  if (threadIdx.x < TT) {
-    const int p = p0 + static_cast<int>(threadIdx.x);
-    int src = -1;
-    if (p < s_poff[G]) {
-      int lo = 0, hi = G - 1;   // last g with poff[g] <= p
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_poff[mid] <= p) lo = mid; else hi = mid - 1;
-      }
-      const int i = p - s_poff[lo];
-      if (i < s_off[lo + 1] - s_off[lo]) src = gather ? gather[s_off[lo] + i] : s_off[lo] + i;
-    }
-    s_src[threadIdx.x] = src;
-  }
-  __syncthreads();
-  load_tile(tile, in, cols, c0, s_src);
-  __syncthreads();
-  store_tile_t(tile, out, kp, p0, c0);
 }
 
 // dGU [n, 2F]: columns [0, F) = dG, [F, 2F) = dU; G, U, dH [n, F].  fq = F / 8.
@@ -315,6 +220,31 @@ router_dlogits_kernel(const float* __restrict__ logits, const float* __restrict_
 }
 
 // fp32 CUDA-core GEMM, split over K: part[z][m][n] = sum_{k in slice z} A(m, k) B(k, n).
+// x's rows in expert order, for a forward that gathered them instead of
+// writing x_perm (flag set): x_perm[r] = x[perm_src[r]], one warp per row
+// (grid-stride); a row whose source is out of range (a skipped pair) is
+// zeroed.  With the flag clear the forward's x_perm is already there and
+// nothing is done.
+__global__ void __launch_bounds__(256)
+fill_xperm_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_src,
+                  const uint32_t* __restrict__ flag, uint4* __restrict__ x_perm, long long R,
+                  int T, int vecs) {
+  pdl_trigger();
+  pdl_wait();
+  if (*flag == 0u) return;
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long r = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < R; r += warps) {
+    const int t = perm_src[r];
+    const bool ok = t >= 0 && t < T;
+    uint4* dst = x_perm + r * vecs;
+    const uint4* src = x + static_cast<long long>(ok ? t : 0) * vecs;
+    for (int c = lane; c < vecs; c += 32)
+      dst[c] = ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 // The router gradients dW_router = dlogits^T x and dx_router = dlogits Wr
 // run on the tensor cores.  x and Wr are bf16; dlogits (fp32) is written as
 // h1 + h2 + h3 with h1 = bf16(v), h2 = bf16(v - h1), h3 = bf16(v - h1 - h2)
@@ -402,22 +332,6 @@ cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos
                     topk_w, static_cast<uint4*>(dy), dw, T, d / 8, k);
 }
 
-cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,
-                        cudaStream_t stream) {
-  return launch_pdl(pad_offsets_kernel, dim3(1), dim3(32), 0, stream, offsets, G, rows_single,
-                    poff);
-}
-
-cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,
-                            int rows_single, const int32_t* poff, const int32_t* gather,
-                            void* out, int kp, cudaStream_t stream) {
-  if (kp % TT || cols % TT || G > 257) return cudaErrorInvalidValue;
-  const dim3 grid(kp / TT, cols / TT);
-  return launch_pdl(gtranspose_kernel, grid, dim3(256), 0, stream,
-                    static_cast<const __nv_bfloat16*>(in), cols, offsets, G, rows_single, poff,
-                    gather, static_cast<__nv_bfloat16*>(out), kp);
-}
-
 cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
                        int F, cudaStream_t stream) {
   const long long n8 = n * (F / 8);
@@ -441,6 +355,17 @@ cudaError_t router_dlogits(const float* logits, const float* offset, const int32
   return launch_pdl(router_dlogits_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0,
                     stream, logits, offset, topk_idx, topk_w, dw, T, E, k, gate, renorm,
                     dlogits);
+}
+
+cudaError_t fill_xperm(const void* x, const int32_t* perm_src, const uint32_t* flag,
+                       void* x_perm, long long R, int T, int d, cudaStream_t stream) {
+  const int warps = 8;
+  long long blocks = (R + warps - 1) / warps;
+  if (blocks > 1184) blocks = 1184;   // 8 per SM; rows are taken grid-stride
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(fill_xperm_kernel, dim3(static_cast<unsigned>(blocks)), dim3(warps * 32), 0,
+                    stream, static_cast<const uint4*>(x), perm_src, flag,
+                    static_cast<uint4*>(x_perm), R, T, d / 8);
 }
 
 RouterGradShape router_grad_shape(int T, int E) {

@@ -82,9 +82,6 @@ struct GemmArgs {
   int x_ldc;
   int gather_limit;            // GATHER: entries of gather_rows
   int gather_src_rows;         // GATHER: rows of gather_src
-  // GATHER: when set and zero on the device, the rows are read in tiles from
-  // the permuted copy (map tmA2, no extra group) instead of gathered
-  const uint32_t* gather_flag;
 };
 
 // Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
@@ -336,7 +333,6 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     int stage = 0;
     uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
     bool ok = true;
-    const bool copy_a = GATHER && args.gather_flag != nullptr && __ldg(args.gather_flag) == 0u;
     // without gathers lane 0 alone drives the ring
     for (int tile = pair; tile < total_tiles && ok && (GATHER || lane == 0); tile += npairs) {
       const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
@@ -345,10 +341,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const int gbase = pt.x ? 0 : g * args.n_per_group;
       const int brow = SWIGLU ? gbase + n * BN_OUT
                               : gbase + n * BN_OUT + static_cast<int>(rank) * (BN_ACC / 2);
-      const CUtensorMap* ma = (pt.x || copy_a) ? &tmA2 : &tmA;
+      const CUtensorMap* ma = pt.x ? &tmA2 : &tmA;
       const CUtensorMap* mb = (SWIGLU && rank == 1) ? (pt.x ? &tmB1_2 : &tmB1)
                                                     : (pt.x ? &tmB0_2 : &tmB0);
-      const bool gathered = GATHER && !pt.x && !copy_a;
+      const bool gathered = GATHER && !pt.x;
       int tok[4] = {0, 0, 0, 0};
       if (gathered) {
 #pragma unroll
@@ -672,7 +668,7 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
       !make_map(&tb1, W3, b_rows, K, bh) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0, nullptr};
+                0, 0, 0, nullptr, 0, 0, 0};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, bh) ||
@@ -707,7 +703,7 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
       !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, R, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows), nullptr};
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, 128) ||
@@ -724,35 +720,6 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
   }
   return launch_pair<256, MODE_SWIGLU_BF16, true>(ta, tb0, tb1, tc, xa, xb0, xb1, xc,
                                                   args, static_cast<int>(R), stream);
-}
-
-// Y[r] = X[rows[r]] W[g]^T for the expert-contiguous rows r < R (A rows
-// gathered from X [x_rows, K] as above); Y is [R, N].  When x_perm [R, K]
-// and flag are given, the kernel reads the flag on the device: zero means
-// x_perm holds the permuted rows, which are then read in tiles instead.
-cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
-                                     const int32_t* offsets, int num_groups, const void* W, int N,
-                                     int K, void* Y, uint32_t* status, cudaStream_t stream,
-                                     const void* x_perm, const uint32_t* flag) {
-  CUtensorMap ta, tb, tc, tp;
-  const int64_t b_rows = static_cast<int64_t>(num_groups) * N;
-  const int bn = (N % 256 == 0) ? 256 : 128;
-  if (!make_map(&ta, X, x_rows, K, 1) || !make_map(&tb, W, b_rows, K, bn / 2) ||
-      !make_map(&tc, Y, R, N, 32))
-    return cudaErrorInvalidValue;
-  if (x_perm != nullptr && flag != nullptr) {
-    if (!make_map(&tp, x_perm, R, K, BM)) return cudaErrorInvalidValue;
-  } else {
-    tp = ta;
-    flag = nullptr;
-  }
-  GemmArgs args{offsets, num_groups, 0, N, K, Y, N, status, rows, X, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows), flag};
-  if (bn == 256)
-    return launch_pair<256, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, tp, tb, tb, tc, args,
-                                                   static_cast<int>(R), stream);
-  return launch_pair<128, MODE_PLAIN_BF16, true>(ta, tb, tb, tc, tp, tb, tb, tc, args,
-                                                 static_cast<int>(R), stream);
 }
 
 // Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.  extra: one
@@ -778,7 +745,7 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0, nullptr};
+                0, 0, 0, nullptr, 0, 0, 0};
   if (extra != nullptr && extra->rows > 0) {
     if (extra->n != N || !make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb, extra->B0, N, extra->K, bn / 2) ||
@@ -817,7 +784,7 @@ cudaError_t grouped_gemm_bmn_f32out(const void* A, int64_t a_rows, const int32_t
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, B0, b0_total_rows, N, BK))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
-                K / BK, K, 0, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
+                K / BK, K, 0, 0, 0, 0, nullptr, 0, 0, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (N % 256 == 0)
     return launch_pair<256, MODE_PLAIN_BMN_F32>(ta, tb0, tb0, ta, ta, tb0, tb0, ta, args,
@@ -844,7 +811,7 @@ cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* 
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
-                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
+                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (N % 512 == 0 && K >= 4096)
     return launch_pair<512, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args,

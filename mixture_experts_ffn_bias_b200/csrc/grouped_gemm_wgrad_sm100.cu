@@ -1,22 +1,28 @@
 // K-grouped GEMM on tcgen05 tensor cores: the weight gradients of the
 // grouped experts.
 //
-// For every group (expert) g:   C_g [M, N] = A_g B_g^T,   bf16 in, fp32
+// For every group (expert) g:   C_g [M, N] = A_g^T B_g,   bf16 in, fp32
 // accumulate in TMEM, bf16 out, C stored as [G, M, N].
-// A_g and B_g are the columns [poff[g], poff[g+1]) of A [M, Kp] and B [N, Kp]
-// (row-major, so the reduction dimension is contiguous: K-major operands).
-// They are the transposed activations of the expert's rows: for the down
-// projection dW2[g] = dY_g^T H_g uses A = dY^T, B = H^T; for the gate/up
-// projections dW1[g] = dG_g^T X_g uses A = dG^T, B = X^T.  Each group's
-// column range is padded with zeros to a multiple of 64, so a k-block never
-// straddles two groups; an expert with no rows gets C_g = 0 (written by the
-// epilogue without touching the accumulator ring).
+// A_g and B_g are the rows [off[g], off[g+1]) of A [R, lda] (columns
+// [a_col0, a_col0 + M)) and B [R, ldb] (columns [b_col0, b_col0 + N)): the
+// activations of the expert's rows as the forward and backward keep them, so
+// the reduction dimension (rows) is the strided one and both operands are
+// read MN-major, with no transposed copy.  For the down projection
+// dW2[g] = dY_g^T H_g (A = dY, B = H); for the gate/up projections
+// dW1[g] = dG_g^T X_g and dW3[g] = dU_g^T X_g (A = [dG | dU] from column 0
+// or F, B = X's rows in expert order).  A group's rows start anywhere; its
+// last 64-row k-block may reach into the next group's rows, which are zeroed
+// in the A tile in shared memory before the MMAs read it, so they add
+// nothing.  An expert with no rows gets C_g = 0 (written by the epilogue
+// without touching the accumulator ring).
 //
 // Structure (one CTA per SM, persistent over (g, m, n) tiles, n fastest):
-//   warp 0      TMA producer: A tile 128 x 64, B tile BN x 64 per stage
-//   warp 1      TMEM allocation; one lane issues tcgen05.mma (M = 128,
-//               N = BN, K = 16 per instruction) into a double-buffered
-//               accumulator
+//   warp 0      TMA producer: A tile 64 k x 128 m (two 64-column boxes),
+//               B tile 64 k x BN n per stage, 128-byte swizzle
+//   warp 1      TMEM allocation; zeroes the rows past a group in its last
+//               A tile; one lane issues tcgen05.mma (M = 128, N = BN, K =
+//               16 per instruction, both operands MN-major) into a
+//               double-buffered accumulator
 //   warps 2..5  epilogue: TMEM -> registers -> bf16, staged 32 rows x 64
 //               columns per warp in shared memory, TMA tensor stores
 // Every wait is bounded; a wait that gives up aborts the CTA and sets the
@@ -52,11 +58,15 @@ struct WCfg {
 };
 
 struct WgradArgs {
-  const int32_t* poff;   // [G+1] padded column offsets
+  const int32_t* offsets;  // [G+1] row offsets of the groups, or null: one group of rows_single
+  int rows_single;
   int G, M, N;
-  __nv_bfloat16* C;      // [G, M, N]
+  int a_col0, b_col0;      // first column of A and of B taken
+  __nv_bfloat16* C;        // [G, M, N]
   uint32_t* status;
 };
+
+constexpr int W_BOX = 64 * 128;   // one 64-column x 64-row box of an MN-major operand
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -69,7 +79,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
              const __grid_constant__ CUtensorMap tmC, const WgradArgs args) {
   using Cfg = WCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
-  constexpr uint32_t IDESC = idesc_bf16_f32(WBM, BN);
+  constexpr uint32_t IDESC = idesc_bf16_f32(WBM, BN, true, true);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -82,7 +92,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
   uint64_t* tfull_bar = bars + 2 * STAGES;
   uint64_t* tempty_bar = bars + 2 * STAGES + 2;
   uint64_t* drain_bar = bars + 2 * STAGES + 4;
-  __shared__ int s_poff[W_MAX_GROUPS + 1];
+  __shared__ int s_off[W_MAX_GROUPS + 1];
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
@@ -113,8 +123,14 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     tmem_relinquish();
   }
   pdl_wait();   // everything above touches no global memory
-  if (warp == 2)
-    for (int i = lane; i <= args.G; i += 32) s_poff[i] = args.poff[i];
+  if (warp == 2) {
+    if (args.offsets)
+      for (int i = lane; i <= args.G; i += 32) s_off[i] = args.offsets[i];
+    else if (lane == 0) {
+      s_off[0] = 0;
+      s_off[1] = args.rows_single;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -130,12 +146,19 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         const int g = tile / (MT * NT);
         const int rem = tile - g * MT * NT;
         const int m = rem / NT, n = rem - (rem / NT) * NT;
-        const int k0 = s_poff[g], kbs = (s_poff[g + 1] - k0) / WBK;
+        const int k0 = s_off[g], kbs = (s_off[g + 1] - k0 + WBK - 1) / WBK;
         for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
-          tma_load_2d(sA + stage * W_A_BYTES, &tmA, &full_bar[stage], k0 + kb * WBK, m * WBM);
-          tma_load_2d(sB + stage * Cfg::B_BYTES, &tmB, &full_bar[stage], k0 + kb * WBK, n * BN);
+          const int krow = k0 + kb * WBK;
+#pragma unroll
+          for (int j = 0; j < WBM / 64; ++j)
+            tma_load_2d(sA + stage * W_A_BYTES + j * W_BOX, &tmA, &full_bar[stage],
+                        args.a_col0 + m * WBM + j * 64, krow);
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sB + stage * Cfg::B_BYTES + j * W_BOX, &tmB, &full_bar[stage],
+                        args.b_col0 + n * BN + j * 64, krow);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -152,42 +175,65 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      int stage = 0, it = 0;
-      uint32_t phase = 0;
-      bool ok = true, issued = false;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const int g = tile / (MT * NT);
-        const int kbs = (s_poff[g + 1] - s_poff[g]) / WBK;
-        if (kbs == 0) continue;   // empty group: the epilogue writes zeros, no accumulator
-        const int acc = it & 1;
-        if (!mbar_wait(&tempty_bar[acc], ((it >> 1) & 1) ^ 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d = tmem + acc * BN;
-        for (int kb = 0; kb < kbs; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+    // the whole warp follows the tiles: lane 0 issues the MMAs, all lanes
+    // zero the rows past a group in its last A tile
+    int stage = 0, it = 0;
+    uint32_t phase = 0;
+    bool ok = true, issued = false;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int g = tile / (MT * NT);
+      const int rows_g = s_off[g + 1] - s_off[g];
+      const int kbs = (rows_g + WBK - 1) / WBK;
+      if (kbs == 0) continue;   // empty group: the epilogue writes zeros, no accumulator
+      const int acc = it & 1;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&tempty_bar[acc], ((it >> 1) & 1) ^ 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * BN;
+      for (int kb = 0; kb < kbs; ++kb) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&full_bar[stage], phase, abort_flag));
+        if (!ok) break;
+        const int valid = rows_g - kb * WBK;   // rows of this k-block in the group
+        if (valid < WBK) {
+          // rows [valid, 64) of both A boxes belong to the next group (or
+          // lie past the tensor): zero them, 16 bytes per lane per store;
+          // each row of a box is 128 contiguous bytes whatever the swizzle
+          uint8_t* a_st = sA + stage * W_A_BYTES;
+          const int per_box = (WBK - valid) * 8;
+          for (int i = lane; i < 2 * per_box; i += 32) {
+            const int box = i / per_box, c = i - box * per_box;
+            *reinterpret_cast<uint4*>(a_st + box * W_BOX + valid * 128 + c * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_async_shared();   // visible to the tensor cores' reads
+        }
+        __syncwarp();
+        if (lane == 0) {
           tc_fence_after();
           const uint32_t a = smem_u32(sA + stage * W_A_BYTES);
           const uint32_t b = smem_u32(sB + stage * Cfg::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < WBK / 16; ++kk)
-            tc_mma_f16(d, smem_desc_sw128(a + kk * 32), smem_desc_sw128(b + kk * 32), IDESC,
+            tc_mma_f16(d, smem_desc_sw128_mn(a + kk * 16 * 128, W_BOX),
+                       smem_desc_sw128_mn(b + kk * 16 * 128, W_BOX), IDESC,
                        (kb | kk) != 0 ? 1u : 0u);
-          issued = true;
           tc_commit(&empty_bar[stage]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
-        tc_commit(&tfull_bar[acc]);
-        ++it;
+        issued = true;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
-      if (!ok && issued) {
-        tc_commit(drain_bar);
-        const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0))
-          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
-      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(&tfull_bar[acc]);
+      ++it;
     }
+    if (!ok && issued && lane == 0) {
+      tc_commit(drain_bar);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain_bar, 0))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+    __syncwarp();
   } else {
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -199,7 +245,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       uint4* dst = reinterpret_cast<uint4*>(
           args.C + (static_cast<size_t>(g) * args.M + m * WBM + row) * args.N +
           static_cast<size_t>(n) * BN);
-      if (s_poff[g + 1] == s_poff[g]) {   // empty group: C_g = 0, no accumulator used
+      if (s_off[g + 1] == s_off[g]) {   // empty group: C_g = 0, no accumulator used
         for (int c = 0; c < BN / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
         continue;
       }
@@ -316,16 +362,20 @@ cudaError_t launch_wgrad(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
 
 }  // namespace
 
-cudaError_t grouped_wgrad_bf16(const void* A, const void* B, int64_t kp, const int32_t* poff,
-                               int G, int M, int N, void* C, uint32_t* status,
-                               cudaStream_t stream) {
-  if (M % WBM || N % 128 || G > W_MAX_GROUPS - 1 || kp % WBK) return cudaErrorInvalidValue;
+cudaError_t grouped_wgrad_bf16(const void* A, int lda, int a_col0, const void* B, int ldb,
+                               int b_col0, int64_t rows, const int32_t* offsets, int G, int M,
+                               int N, void* C, uint32_t* status, cudaStream_t stream) {
+  if (M % WBM || N % 128 || G > W_MAX_GROUPS - 1 || a_col0 % 64 || b_col0 % 64 ||
+      a_col0 + M > lda || b_col0 + N > ldb || (offsets == nullptr && G != 1) ||
+      rows > 0x7fffffff)
+    return cudaErrorInvalidValue;
   const int bn = (N % 256 == 0) ? 256 : 128;
   CUtensorMap ta, tb, tc;
-  if (!map_rows(&ta, A, M, kp, WBM) || !map_rows(&tb, B, N, kp, bn) ||
+  if (!map_rows(&ta, A, rows, lda, WBK) || !map_rows(&tb, B, rows, ldb, WBK) ||
       !map_rows(&tc, C, static_cast<int64_t>(G) * M, N, 32))
     return cudaErrorInvalidValue;
-  WgradArgs a{poff, G, M, N, static_cast<__nv_bfloat16*>(C), status};
+  WgradArgs a{offsets, static_cast<int>(rows), G, M, N, a_col0, b_col0,
+              static_cast<__nv_bfloat16*>(C), status};
   if (bn == 256) return launch_wgrad<256>(ta, tb, tc, a, stream);
   return launch_wgrad<128>(ta, tb, tc, a, stream);
 }

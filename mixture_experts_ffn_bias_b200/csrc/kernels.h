@@ -116,15 +116,6 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
                                               const void* W1, const void* W3, int F, int K,
                                               void* H, uint32_t* status, cudaStream_t stream,
                                               const GemmExtraGroup* extra = nullptr);
-// Y[r] = X[rows[r]] W[g]^T over the expert-contiguous rows r < R (A rows
-// gathered from X by the permutation; no permuted copy).
-// With x_perm [R, K] and flag: a zero flag on the device means x_perm holds
-// the permuted rows, read in tiles instead of gathered.
-cudaError_t grouped_gemm_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows, int64_t R,
-                                     const int32_t* offsets, int num_groups, const void* W, int N,
-                                     int K, void* Y, uint32_t* status, cudaStream_t stream,
-                                     const void* x_perm = nullptr,
-                                     const uint32_t* flag = nullptr);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream,
@@ -150,19 +141,16 @@ cudaError_t grouped_down_f32(const float* A, int64_t a_rows, const int32_t* offs
                              float* Y, cudaStream_t stream);
 
 // Backward -------------------------------------------------------------------
-// K-grouped weight gradient C_g [M, N] = A_g B_g^T over the padded column
-// ranges [poff[g], poff[g+1]) of A [M, kp] and B [N, kp]; C [G, M, N] bf16.
-cudaError_t grouped_wgrad_bf16(const void* A, const void* B, int64_t kp, const int32_t* poff,
-                               int G, int M, int N, void* C, uint32_t* status,
-                               cudaStream_t stream);
+// K-grouped weight gradient C_g [M, N] = A_g^T B_g over the rows
+// [offsets[g], offsets[g+1]) (offsets null: one group of `rows` rows) of
+// A [rows, lda] (columns a_col0 ..) and B [rows, ldb] (columns b_col0 ..),
+// both read MN-major; C [G, M, N] bf16.
+cudaError_t grouped_wgrad_bf16(const void* A, int lda, int a_col0, const void* B, int ldb,
+                               int b_col0, int64_t rows, const int32_t* offsets, int G, int M,
+                               int N, void* C, uint32_t* status, cudaStream_t stream);
 cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos,
                    const float* topk_w, void* dy, float* dw, int T, int d, int k,
                    cudaStream_t stream);
-cudaError_t pad_offsets(const int32_t* offsets, int G, int rows_single, int32_t* poff,
-                        cudaStream_t stream);
-cudaError_t gtranspose_bf16(const void* in, int cols, const int32_t* offsets, int G,
-                            int rows_single, const int32_t* poff, const int32_t* gather,
-                            void* out, int kp, cudaStream_t stream);
 cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
                        int F, cudaStream_t stream);
 cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr, const void* dxs,
@@ -170,6 +158,10 @@ cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr
 cudaError_t router_dlogits(const float* logits, const float* offset, const int32_t* topk_idx,
                            const float* topk_w, const float* dw, int T, int E, int k, int gate,
                            int renorm, float* dlogits, cudaStream_t stream);
+// x_perm[r] = x[perm_src[r]] for r < R when *flag is non-zero (a forward
+// that gathered its rows); nothing otherwise.  bf16 rows of d elements.
+cudaError_t fill_xperm(const void* x, const int32_t* perm_src, const uint32_t* flag,
+                       void* x_perm, long long R, int T, int d, cudaStream_t stream);
 // Router gradients on the tensor cores: dlogits split into three bf16 terms
 // (exact), Ep = E rounded up to 64, G token slices of Ks tokens for dW.
 struct RouterGradShape {

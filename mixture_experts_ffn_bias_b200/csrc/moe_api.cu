@@ -297,10 +297,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
 
 // Workspace of moe_backward (separate from the forward's, which it reads).
 struct BLayout {
-  size_t status, dw, logits, dlogits, adx, adw, wr3, pdw, goff, dxr, poff, poff_sh, dy, dh, gb,
-      ub, dgu, dxp, dyT,
-      hT, dguT, xT, dh_sh, g_sh, u_sh, dgu_sh, dxs, doutT, hshT, dgushT, xTs, total;
-  int64_t kp, tp;
+  size_t status, dw, logits, dlogits, adx, adw, wr3, pdw, goff, dxr, dy, dh, gb, ub, dgu, dxp,
+      dh_sh, g_sh, u_sh, dgu_sh, dxs, total;
 };
 
 BLayout blayout(const moe_config& c) {
@@ -308,10 +306,6 @@ BLayout blayout(const moe_config& c) {
                k = c.top_k, R = T * k;
   const size_t Fs = c.n_shared ? static_cast<size_t>(c.d_ff_shared) : 0;
   BLayout B{};
-  // every group's column range is padded to a multiple of 64
-  B.kp = static_cast<int64_t>((R + 63 * E + 63) / 64 * 64);
-  B.tp = static_cast<int64_t>((T + 63) / 64 * 64);
-  const size_t kp = static_cast<size_t>(B.kp), tp = static_cast<size_t>(B.tp);
   size_t o = 0;
   B.status = o;  o += up(2 * sizeof(uint32_t));
   B.dw = o;      o += up(R * 4);
@@ -325,27 +319,17 @@ BLayout blayout(const moe_config& c) {
   B.pdw = o;     o += up(Gs * C3 * d * 4);
   B.goff = o;    o += up((Gs + 1) * 4);
   B.dxr = o;     o += up(T * d * 4);
-  B.poff = o;    o += up((E + 1) * 4);
-  B.poff_sh = o; o += up(2 * 4);
   B.dy = o;      o += up(R * d * 2);
   B.dh = o;      o += up(R * F * 2);
   B.gb = o;      o += up(R * F * 2);
   B.ub = o;      o += up(R * F * 2);
   B.dgu = o;     o += up(R * 2 * F * 2);
   B.dxp = o;     o += up(R * d * 2);
-  B.dyT = o;     o += up(d * kp * 2);
-  B.hT = o;      o += up(F * kp * 2);
-  B.dguT = o;    o += up(2 * F * kp * 2);
-  B.xT = o;      o += up(d * kp * 2);
   B.dh_sh = o;   o += up(T * Fs * 2);
   B.g_sh = o;    o += up(T * Fs * 2);
   B.u_sh = o;    o += up(T * Fs * 2);
   B.dgu_sh = o;  o += up(T * 2 * Fs * 2);
   B.dxs = o;     o += up(Fs ? T * d * 2 : 0);
-  B.doutT = o;   o += up(Fs ? d * tp * 2 : 0);
-  B.hshT = o;    o += up(Fs * tp * 2);
-  B.dgushT = o;  o += up(2 * Fs * tp * 2);
-  B.xTs = o;     o += up(Fs ? d * tp * 2 : 0);
   B.total = o;
   return B;
 }
@@ -369,47 +353,37 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
   const void* h = at<void>(fws, L.h);
   const void* y_perm = at<void>(fws, L.y_perm);
   float* dw = at<float>(bws, B.dw);
-  int32_t* poff = at<int32_t>(bws, B.poff);
   // combine: dw and the experts' output gradients
   MOE_TRY(moe::bwd_dy(dout, y_perm, slot_pos, topk_w, at<void>(bws, B.dy), dw, T, d, k, s));
   // dH = dY W2 ; G, U recomputed ; dG, dU ; dX = [dG | dU] [W1 ; W3].  The
   // weights of dH and dX are read MN-major in place (no transposed copies).
   MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dy), R, offsets, E, 0, w->w2, nullptr, d,
                                      F, d, at<void>(bws, B.dh), status, s));
-  // G and U recomputed from the forward's permuted copy of x, or, when that
-  // forward gathered its rows instead (status word 2 set), from x's rows
-  // gathered by the permutation
-  const void* x_perm = at<void>(fws, L.x_perm);
-  const uint32_t* no_xperm = at<uint32_t>(fws, L.status) + 2;
-  MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w1, F, d,
-                                        at<void>(bws, B.gb), status, s, x_perm, no_xperm));
-  MOE_TRY(moe::grouped_gemm_gather_bf16(x, T, perm_src, R, offsets, E, w->w3, F, d,
-                                        at<void>(bws, B.ub), status, s, x_perm, no_xperm));
+  // x's rows in expert order: the forward's x_perm, written here from x by
+  // the permutation when that forward gathered its rows instead (status
+  // word 2 set).  G and U are recomputed from it.
+  void* x_perm = at<void>(fws, L.x_perm);
+  MOE_TRY(moe::fill_xperm(x, perm_src, at<uint32_t>(fws, L.status) + 2, x_perm, R, T, d, s));
+  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w1, F, d, at<void>(bws, B.gb),
+                                 status, s));
+  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w3, F, d, at<void>(bws, B.ub),
+                                 status, s));
   MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.gb), at<void>(bws, B.ub), at<void>(bws, B.dh),
                           at<void>(bws, B.dgu), R, F, s));
   MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, w->w1, w->w3, F, d,
                                      2 * F, at<void>(bws, B.dxp), status, s));
-  // weight gradients over each expert's rows (transposed, padded operands)
-  MOE_TRY(moe::pad_offsets(offsets, E, 0, poff, s));
-  MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dy), d, offsets, E, 0, poff, nullptr,
-                               at<void>(bws, B.dyT), static_cast<int>(B.kp), s));
-  MOE_TRY(moe::gtranspose_bf16(h, F, offsets, E, 0, poff, nullptr, at<void>(bws, B.hT),
-                               static_cast<int>(B.kp), s));
-  MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dgu), 2 * F, offsets, E, 0, poff, nullptr,
-                               at<void>(bws, B.dguT), static_cast<int>(B.kp), s));
-  MOE_TRY(moe::gtranspose_bf16(x, d, offsets, E, 0, poff, perm_src, at<void>(bws, B.xT),
-                               static_cast<int>(B.kp), s));
-  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dyT), at<void>(bws, B.hT), B.kp, poff, E, d, F,
+  // weight gradients over each expert's rows, the row-major activations
+  // read MN-major: dW2 = dY^T h, dW1 = dG^T x_perm, dW3 = dU^T x_perm
+  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dy), d, 0, h, F, 0, R, offsets, E, d, F,
                                   g->dw2, status, s));
-  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dguT), at<void>(bws, B.xT), B.kp, poff, E, F,
+  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgu), 2 * F, 0, x_perm, d, 0, R, offsets, E, F,
                                   d, g->dw1, status, s));
-  MOE_TRY(moe::grouped_wgrad_bf16(at<uint8_t>(bws, B.dguT) + static_cast<size_t>(F) * B.kp * 2,
-                                  at<void>(bws, B.xT), B.kp, poff, E, F, d, g->dw3, status, s));
+  MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgu), 2 * F, F, x_perm, d, 0, R, offsets, E, F,
+                                  d, g->dw3, status, s));
   // shared expert (weight 1, all tokens)
   const void* dxs = nullptr;
   if (c->n_shared) {
     const int Fs = c->d_ff_shared;
-    int32_t* poff_sh = at<int32_t>(bws, B.poff_sh);
     MOE_TRY(moe::grouped_gemm_bmn_bf16(dout, T, nullptr, 1, T, w->ws2, nullptr, d, Fs, d,
                                        at<void>(bws, B.dh_sh), status, s));
     MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws1, Fs, d, at<void>(bws, B.g_sh),
@@ -421,23 +395,12 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
     MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu_sh), T, nullptr, 1, T, w->ws1,
                                        w->ws3, Fs, d, 2 * Fs, at<void>(bws, B.dxs), status, s));
     dxs = at<void>(bws, B.dxs);
-    MOE_TRY(moe::pad_offsets(nullptr, 1, T, poff_sh, s));
-    const int tp = static_cast<int>(B.tp);
-    MOE_TRY(moe::gtranspose_bf16(dout, d, nullptr, 1, T, poff_sh, nullptr,
-                                 at<void>(bws, B.doutT), tp, s));
-    MOE_TRY(moe::gtranspose_bf16(at<void>(fws, L.h_sh), Fs, nullptr, 1, T, poff_sh, nullptr,
-                                 at<void>(bws, B.hshT), tp, s));
-    MOE_TRY(moe::gtranspose_bf16(at<void>(bws, B.dgu_sh), 2 * Fs, nullptr, 1, T, poff_sh,
-                                 nullptr, at<void>(bws, B.dgushT), tp, s));
-    MOE_TRY(moe::gtranspose_bf16(x, d, nullptr, 1, T, poff_sh, nullptr, at<void>(bws, B.xTs), tp,
-                                 s));
-    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.doutT), at<void>(bws, B.hshT), tp, poff_sh,
-                                    1, d, Fs, g->dws2, status, s));
-    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgushT), at<void>(bws, B.xTs), tp, poff_sh,
-                                    1, Fs, d, g->dws1, status, s));
-    MOE_TRY(moe::grouped_wgrad_bf16(at<uint8_t>(bws, B.dgushT) + static_cast<size_t>(Fs) * tp * 2,
-                                    at<void>(bws, B.xTs), tp, poff_sh, 1, Fs, d, g->dws3, status,
-                                    s));
+    MOE_TRY(moe::grouped_wgrad_bf16(dout, d, 0, at<void>(fws, L.h_sh), Fs, 0, T, nullptr, 1, d,
+                                    Fs, g->dws2, status, s));
+    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgu_sh), 2 * Fs, 0, x, d, 0, T, nullptr, 1,
+                                    Fs, d, g->dws1, status, s));
+    MOE_TRY(moe::grouped_wgrad_bf16(at<void>(bws, B.dgu_sh), 2 * Fs, Fs, x, d, 0, T, nullptr, 1,
+                                    Fs, d, g->dws3, status, s));
   }
   // router (fp32): recomputed logits, dlogits, then on the tensor cores
   // with dlogits as three exact bf16 terms: dx_router = dlogits Wr (K = 3 Ep,

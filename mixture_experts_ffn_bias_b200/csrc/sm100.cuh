@@ -221,10 +221,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t 
 
 // Instruction descriptor, kind::f16: bf16 A and B (format 1), f32 accumulator
 // (format 1), dense, no negation; N >> 3 at bit 17, M >> 4 at bit 24.  A and
-// B are K-major unless b_mn (bit 16: B is MN-major).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn = false) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn ? (1u << 16) : 0u) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+// B are K-major unless b_mn (bit 16: B is MN-major) or a_mn (bit 15: A is
+// MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn = false,
+                                                      bool a_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn ? (1u << 15) : 0u) |
+         (b_mn ? (1u << 16) : 0u) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // ------------------------------------------------- CTA pairs (cta_group::2) --
