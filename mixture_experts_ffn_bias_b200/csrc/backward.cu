@@ -1,10 +1,10 @@
 // Backward pass of the MoE layer: the memory-bound steps and the fp32 router
 // gradient.  The contractions of the experts run on the tensor cores (the
-// plain grouped GEMM of grouped_gemm_sm100.cu for dH and dX, the K-grouped
-// GEMM of grouped_gemm_wgrad_sm100.cu for the weight gradients); this file
-// holds what feeds and finishes them:
+// grouped GEMM of grouped_gemm_sm100.cu for dH and dX and for the recomputed
+// gate/up pass whose epilogue forms dG and dU, the K-grouped GEMM of
+// grouped_gemm_wgrad_sm100.cu for the weight gradients); this file holds
+// what feeds and finishes them:
 //   bwd_dy_kernel       dw[t, j] = <dout[t], y_perm[slot]>, dY[slot] = w[t, j] dout[t]
-//   swiglu_bwd_kernel   dG = dH * U * silu'(G), dU = dH * silu(G)
 //   dx_gather_kernel    dx[t] = sum_j dX[slot(t, j)] + dx_router[t] (+ dx_shared[t])
 //   router_dlogits_kernel  dlogits from dw through the (renormalised) gate
 //   router_grad_split_kernel  dlogits (fp32) as three bf16 terms, in the two
@@ -80,31 +80,6 @@ bwd_dy_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y_perm,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
     if (lane == 0) dw[p] = dot;
-  }
-}
-
-// dGU [n, 2F]: columns [0, F) = dG, [F, 2F) = dU; G, U, dH [n, F].  fq = F / 8.
-__global__ void __launch_bounds__(256)
-swiglu_bwd_kernel(const uint4* __restrict__ G, const uint4* __restrict__ U,
-                  const uint4* __restrict__ dH, uint4* __restrict__ dGU, long long n8, int fq) {
-  pdl_trigger();
-  pdl_wait();
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const long long r = i / fq;
-    const int c = static_cast<int>(i - r * fq);
-    float g[8], u[8], dh[8], dg[8], du[8];
-    unpack8(G[i], g);
-    unpack8(U[i], u);
-    unpack8(dH[i], dh);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float s = 1.0f / (1.0f + expf(-g[q]));
-      du[q] = dh[q] * g[q] * s;
-      dg[q] = dh[q] * u[q] * (s * (1.0f + g[q] * (1.0f - s)));
-    }
-    dGU[r * 2 * fq + c] = pack8(dg);
-    dGU[r * 2 * fq + fq + c] = pack8(du);
   }
 }
 
@@ -330,14 +305,6 @@ cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos
   return launch_pdl(bwd_dy_kernel, dim3((T + warps - 1) / warps), dim3(warps * 32), 0, stream,
                     static_cast<const uint4*>(dout), static_cast<const uint4*>(y_perm), slot_pos,
                     topk_w, static_cast<uint4*>(dy), dw, T, d / 8, k);
-}
-
-cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
-                       int F, cudaStream_t stream) {
-  const long long n8 = n * (F / 8);
-  return launch_pdl(swiglu_bwd_kernel, dim3(grid_1d(n8)), dim3(256), 0, stream,
-                    static_cast<const uint4*>(G), static_cast<const uint4*>(U),
-                    static_cast<const uint4*>(dH), static_cast<uint4*>(dGU), n8, F / 8);
 }
 
 cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr, const void* dxs,

@@ -57,6 +57,11 @@ constexpr int MODE_PLAIN_BMN = 2;
 // As MODE_PLAIN_BMN with fp32 output, stored row by row from the registers
 // (the router's gradient products, whose sums stay in fp32).
 constexpr int MODE_PLAIN_BMN_F32 = 3;
+// The backward of the SwiGLU, fused into the recomputed gate/up pass: the
+// accumulator holds g = A W1^T and u = A W3^T as in MODE_SWIGLU_BF16, the
+// epilogue reads dH [rows, F] and writes dG = dH u silu'(g) and dU = dH
+// silu(g) into C = [dG | dU] [rows, 2F], bf16.
+constexpr int MODE_SWIGLU_BWD = 4;
 
 struct GemmArgs {
   const int32_t* offsets;  // [G+1] device, or nullptr: one group [0, rows_single)
@@ -82,6 +87,7 @@ struct GemmArgs {
   int x_ldc;
   int gather_limit;            // GATHER: entries of gather_rows
   int gather_src_rows;         // GATHER: rows of gather_src
+  const void* aux;             // SWIGLU_BWD: dH [rows, n_per_group] bf16
 };
 
 // Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
@@ -244,7 +250,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmC2, const GemmArgs args) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
-  constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16;
+  constexpr bool SWI_BWD = MODE == MODE_SWIGLU_BWD;
+  constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16 || SWI_BWD;
   constexpr bool BMN = MODE == MODE_PLAIN_BMN || MODE == MODE_PLAIN_BMN_F32;
   constexpr bool OUT_F32 = MODE == MODE_PLAIN_BMN_F32;
   constexpr int BN_OUT = SWIGLU ? BN_ACC / 2 : BN_ACC;
@@ -500,6 +507,47 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             tmem_ld16(t_addr + UP + c0, *reinterpret_cast<uint32_t(*)[16]>(&u[0]));
             tmem_ld16(t_addr + UP + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&u[16]));
             tmem_ld_wait();
+            if constexpr (SWI_BWD) {
+              if (valid) {
+                // dH of these 32 columns of the row; dG and dU as the
+                // SwiGLU backward: s = sigmoid(g), dU = dH g s,
+                // dG = dH u s (1 + g (1 - s))
+                const size_t rr = static_cast<size_t>(warp_row0 + lane);
+                const uint4* dhp = reinterpret_cast<const uint4*>(
+                    static_cast<const __nv_bfloat16*>(args.aux) + rr * args.n_per_group + ocol +
+                    half * 32);
+                uint4 dq[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dq[i] = dhp[i];
+                const __nv_bfloat162* dh2 = reinterpret_cast<const __nv_bfloat162*>(dq);
+                uint32_t pg[16], pu[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float2 dh = __bfloat1622float2(dh2[i]);
+                  float dgv[2], duv[2];
+#pragma unroll
+                  for (int e = 0; e < 2; ++e) {
+                    const float g = __uint_as_float(v[2 * i + e]);
+                    const float uu = __uint_as_float(u[2 * i + e]);
+                    const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
+                    const float d = e ? dh.y : dh.x;
+                    duv[e] = d * g * sg;
+                    dgv[e] = d * uu * (sg * (1.0f + g * (1.0f - sg)));
+                  }
+                  pg[i] = pack_bf16x2(dgv[0], dgv[1]);
+                  pu[i] = pack_bf16x2(duv[0], duv[1]);
+                }
+                uint4* dg_dst = reinterpret_cast<uint4*>(cbase + crow_off + ocol + half * 32);
+                uint4* du_dst = reinterpret_cast<uint4*>(cbase + crow_off + args.n_per_group +
+                                                         ocol + half * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+                  du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+                }
+              }
+              continue;
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float h0 = silu_f32(__uint_as_float(v[2 * i])) * __uint_as_float(u[2 * i]);
@@ -529,7 +577,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
             }
           }
         }
-        if constexpr (OUT_F32) continue;   // stored above
+        if constexpr (OUT_F32 || SWI_BWD) continue;   // stored above
         if (warp_full) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -668,7 +716,7 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
       !make_map(&tb1, W3, b_rows, K, bh) || !make_map(&tc, H, c_rows, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, F, K, H, F, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0};
+                0, 0, 0, nullptr, 0, 0, 0, nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, bh) ||
@@ -688,6 +736,26 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
                                             rows_upper, stream);
 }
 
+// The SwiGLU backward fused into the recomputed gate/up pass: with g and u
+// the rows of A W1^T and A W3^T, dGU [rows, 2F] = [dH u silu'(g) | dH silu(g)]
+// for dH [rows, F].  Groups as for grouped_swiglu_gateup_bf16.
+cudaError_t grouped_swiglu_bwd_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                    int num_groups, int rows_single, const void* W1,
+                                    const void* W3, int F, int K, const void* dH, void* dGU,
+                                    uint32_t* status, cudaStream_t stream) {
+  if (F % 128) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb0, tb1;
+  const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
+  if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, W1, b_rows, K, 128) ||
+      !make_map(&tb1, W3, b_rows, K, 128))
+    return cudaErrorInvalidValue;
+  GemmArgs args{offsets, num_groups, rows_single, F, K, dGU, 2 * F, status, nullptr, nullptr, 0,
+                0, 0, 0, 0, 0, 0, nullptr, 0, 0, 0, dH};
+  const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  return launch_pair<256, MODE_SWIGLU_BWD>(ta, tb0, tb1, ta, ta, tb0, tb1, ta, args, rows_upper,
+                                           stream);
+}
+
 // Gate/up pass whose A rows are gathered from X [x_rows, K]: output row r
 // (expert-contiguous order, r < R) reads X[rows[r]] (tile::gather4 loads in
 // the CTA-pair kernel).  H is [R, F].  extra as for the plain gate/up pass
@@ -703,7 +771,7 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
       !make_map(&tb1, W3, b_rows, K, 128) || !make_map(&tc, H, R, F, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, 0, F, K, H, F, status, rows, X, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows)};
+                0, 0, 0, nullptr, 0, static_cast<int>(R), static_cast<int>(x_rows), nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (!make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb0, extra->B0, extra->n, extra->K, 128) ||
@@ -745,7 +813,7 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0, 0, 0, 0,
-                0, 0, 0, nullptr, 0, 0, 0};
+                0, 0, 0, nullptr, 0, 0, 0, nullptr};
   if (extra != nullptr && extra->rows > 0) {
     if (extra->n != N || !make_map(&xa, extra->A, extra->rows, extra->K, BM) ||
         !make_map(&xb, extra->B0, N, extra->K, bn / 2) ||
@@ -784,7 +852,7 @@ cudaError_t grouped_gemm_bmn_f32out(const void* A, int64_t a_rows, const int32_t
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb0, B0, b0_total_rows, N, BK))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
-                K / BK, K, 0, 0, 0, 0, nullptr, 0, 0, 0};
+                K / BK, K, 0, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (N % 256 == 0)
     return launch_pair<256, MODE_PLAIN_BMN_F32>(ta, tb0, tb0, ta, ta, tb0, tb0, ta, args,
@@ -811,7 +879,7 @@ cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* 
       !make_map(&tc, Y, c_rows, N, 32))
     return cudaErrorInvalidValue;
   GemmArgs args{offsets, num_groups, rows_single, N, K, Y, N, status, nullptr, nullptr, 0,
-                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0};
+                b0_rows / BK, b0_rows, b1_rows, 0, 0, 0, nullptr, 0, 0, 0, nullptr};
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (N % 512 == 0 && K >= 4096)
     return launch_pair<512, MODE_PLAIN_BMN>(ta, tb0, tb1, tc, ta, tb0, tb1, tc, args,

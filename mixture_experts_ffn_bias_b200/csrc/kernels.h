@@ -116,6 +116,12 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
                                               const void* W1, const void* W3, int F, int K,
                                               void* H, uint32_t* status, cudaStream_t stream,
                                               const GemmExtraGroup* extra = nullptr);
+// dGU [rows, 2F] = [dH u silu'(g) | dH silu(g)] with g = A W1^T, u = A W3^T
+// recomputed on the tensor cores (groups as for the gate/up pass).
+cudaError_t grouped_swiglu_bwd_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
+                                    int num_groups, int rows_single, const void* W1,
+                                    const void* W3, int F, int K, const void* dH, void* dGU,
+                                    uint32_t* status, cudaStream_t stream);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream,
@@ -151,8 +157,6 @@ cudaError_t grouped_wgrad_bf16(const void* A, int lda, int a_col0, const void* B
 cudaError_t bwd_dy(const void* dout, const void* y_perm, const int32_t* slot_pos,
                    const float* topk_w, void* dy, float* dw, int T, int d, int k,
                    cudaStream_t stream);
-cudaError_t swiglu_bwd(const void* G, const void* U, const void* dH, void* dGU, long long n,
-                       int F, cudaStream_t stream);
 cudaError_t dx_gather(const void* dxp, const int32_t* slot_pos, const float* dxr, const void* dxs,
                       void* dx, int T, int d, int k, cudaStream_t stream);
 cudaError_t router_dlogits(const float* logits, const float* offset, const int32_t* topk_idx,

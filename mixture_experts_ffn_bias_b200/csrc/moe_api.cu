@@ -297,8 +297,8 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
 
 // Workspace of moe_backward (separate from the forward's, which it reads).
 struct BLayout {
-  size_t status, dw, logits, dlogits, adx, adw, wr3, pdw, goff, dxr, dy, dh, gb, ub, dgu, dxp,
-      dh_sh, g_sh, u_sh, dgu_sh, dxs, total;
+  size_t status, dw, logits, dlogits, adx, adw, wr3, pdw, goff, dxr, dy, dh, dgu, dxp, dh_sh,
+      dgu_sh, dxs, total;
 };
 
 BLayout blayout(const moe_config& c) {
@@ -321,13 +321,9 @@ BLayout blayout(const moe_config& c) {
   B.dxr = o;     o += up(T * d * 4);
   B.dy = o;      o += up(R * d * 2);
   B.dh = o;      o += up(R * F * 2);
-  B.gb = o;      o += up(R * F * 2);
-  B.ub = o;      o += up(R * F * 2);
   B.dgu = o;     o += up(R * 2 * F * 2);
   B.dxp = o;     o += up(R * d * 2);
   B.dh_sh = o;   o += up(T * Fs * 2);
-  B.g_sh = o;    o += up(T * Fs * 2);
-  B.u_sh = o;    o += up(T * Fs * 2);
   B.dgu_sh = o;  o += up(T * 2 * Fs * 2);
   B.dxs = o;     o += up(Fs ? T * d * 2 : 0);
   B.total = o;
@@ -361,15 +357,12 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
                                      F, d, at<void>(bws, B.dh), status, s));
   // x's rows in expert order: the forward's x_perm, written here from x by
   // the permutation when that forward gathered its rows instead (status
-  // word 2 set).  G and U are recomputed from it.
+  // word 2 set).  G and U are recomputed from it on the tensor cores, and the
+  // SwiGLU backward runs in that GEMM's epilogue: [dG | dU] from G, U, dH.
   void* x_perm = at<void>(fws, L.x_perm);
   MOE_TRY(moe::fill_xperm(x, perm_src, at<uint32_t>(fws, L.status) + 2, x_perm, R, T, d, s));
-  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w1, F, d, at<void>(bws, B.gb),
-                                 status, s));
-  MOE_TRY(moe::grouped_down_bf16(x_perm, R, offsets, E, 0, w->w3, F, d, at<void>(bws, B.ub),
-                                 status, s));
-  MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.gb), at<void>(bws, B.ub), at<void>(bws, B.dh),
-                          at<void>(bws, B.dgu), R, F, s));
+  MOE_TRY(moe::grouped_swiglu_bwd_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d,
+                                       at<void>(bws, B.dh), at<void>(bws, B.dgu), status, s));
   MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu), R, offsets, E, 0, w->w1, w->w3, F, d,
                                      2 * F, at<void>(bws, B.dxp), status, s));
   // weight gradients over each expert's rows, the row-major activations
@@ -386,12 +379,9 @@ moe_status backward_impl(const moe_config* c, const void* x, const void* w_route
     const int Fs = c->d_ff_shared;
     MOE_TRY(moe::grouped_gemm_bmn_bf16(dout, T, nullptr, 1, T, w->ws2, nullptr, d, Fs, d,
                                        at<void>(bws, B.dh_sh), status, s));
-    MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws1, Fs, d, at<void>(bws, B.g_sh),
-                                   status, s));
-    MOE_TRY(moe::grouped_down_bf16(x, T, nullptr, 1, T, w->ws3, Fs, d, at<void>(bws, B.u_sh),
-                                   status, s));
-    MOE_TRY(moe::swiglu_bwd(at<void>(bws, B.g_sh), at<void>(bws, B.u_sh),
-                            at<void>(bws, B.dh_sh), at<void>(bws, B.dgu_sh), T, Fs, s));
+    MOE_TRY(moe::grouped_swiglu_bwd_bf16(x, T, nullptr, 1, T, w->ws1, w->ws3, Fs, d,
+                                         at<void>(bws, B.dh_sh), at<void>(bws, B.dgu_sh), status,
+                                         s));
     MOE_TRY(moe::grouped_gemm_bmn_bf16(at<void>(bws, B.dgu_sh), T, nullptr, 1, T, w->ws1,
                                        w->ws3, Fs, d, 2 * Fs, at<void>(bws, B.dxs), status, s));
     dxs = at<void>(bws, B.dxs);
