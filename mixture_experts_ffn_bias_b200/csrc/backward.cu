@@ -44,55 +44,84 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return o;
 }
 
-// One warp per token.  oct = d / 8 (uint4 of 8 bf16 per lane step).
+// One warp per token.  oct = d / 8 (uint4 of 8 bf16 per lane step).  Lane j
+// holds the slot and weight of the token's j-th pair; the dout row is read
+// once, four 16-byte pieces per lane at a time, and each pair's y_perm
+// pieces are all requested before they are used.
 __global__ void __launch_bounds__(256)
 bwd_dy_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y_perm,
               const int32_t* __restrict__ slot_pos, const float* __restrict__ topk_w,
               uint4* __restrict__ dy, float* __restrict__ dw, int T, int oct, int k) {
   pdl_trigger();
   pdl_wait();
+  constexpr int U = 4;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  const uint4* drow = dout + static_cast<size_t>(t) * oct;
-  for (int j = 0; j < k; ++j) {
-    const size_t p = static_cast<size_t>(t) * k + j;
-    const int r = slot_pos[p];
-    if (r < 0) {
-      if (lane == 0) dw[p] = 0.f;
-      continue;
-    }
-    const float w = topk_w[p];
-    const uint4* yrow = y_perm + static_cast<size_t>(r) * oct;
-    uint4* dyrow = dy + static_cast<size_t>(r) * oct;
-    float dot = 0.f;
-    for (int c = lane; c < oct; c += 32) {
-      float a[8], b[8], o[8];
-      unpack8(drow[c], a);
-      unpack8(__ldcs(yrow + c), b);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        dot = fmaf(a[i], b[i], dot);
-        o[i] = w * a[i];
-      }
-      dyrow[c] = pack8(o);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (lane == 0) dw[p] = dot;
+  int my_slot = -1;
+  float my_w = 0.f;
+  if (lane < k) {
+    my_slot = slot_pos[static_cast<size_t>(t) * k + lane];
+    my_w = topk_w[static_cast<size_t>(t) * k + lane];
   }
+  const uint4* drow = dout + static_cast<size_t>(t) * oct;
+  float my_dot = 0.f;   // lane j: <dout[t], y_perm[slot j]>
+  for (int c0 = lane; c0 < oct; c0 += 32 * U) {
+    float a[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c < oct) unpack8(__ldg(drow + c), a[u]);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int r = __shfl_sync(0xffffffffu, my_slot, j);
+      const float w = __shfl_sync(0xffffffffu, my_w, j);
+      if (r < 0) continue;
+      const uint4* yrow = y_perm + static_cast<size_t>(r) * oct;
+      uint4* dyrow = dy + static_cast<size_t>(r) * oct;
+      uint4 yv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        yv[u] = c < oct ? __ldcs(yrow + c) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float dot = 0.f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= oct) continue;
+        float b[8], o[8];
+        unpack8(yv[u], b);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          dot = fmaf(a[u][i], b[i], dot);
+          o[i] = w * a[u][i];
+        }
+        dyrow[c] = pack8(o);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (lane == j) my_dot += dot;
+    }
+  }
+  if (lane < k) dw[static_cast<size_t>(t) * k + lane] = my_slot < 0 ? 0.f : my_dot;
 }
 
-// One warp per token: dx = sum_j dX[slot] + dxr (fp32) + dxs (bf16, may be null).
+// One warp per token: dx = sum_j dX[slot] + dxr (fp32) + dxs (bf16, may be
+// null).  Lane j holds the slot of the token's j-th pair; for each 16-byte
+// piece of the row all k rows are requested before they are added (pairs in
+// j order, k <= 32).
 __global__ void __launch_bounds__(256)
 dx_gather_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ slot_pos,
                  const float4* __restrict__ dxr, const uint4* __restrict__ dxs,
                  uint4* __restrict__ dx, int T, int oct, int k) {
   pdl_trigger();
   pdl_wait();
+  constexpr int KB = 8;   // rows requested together
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
+  const int my_slot = lane < k ? slot_pos[static_cast<size_t>(t) * k + lane] : -1;
   for (int c = lane; c < oct; c += 32) {
     float acc[8];
     const float4 a = dxr[(static_cast<size_t>(t) * oct + c) * 2];
@@ -105,13 +134,21 @@ dx_gather_kernel(const uint4* __restrict__ dxp, const int32_t* __restrict__ slot
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += s[i];
     }
-    for (int j = 0; j < k; ++j) {
-      const int r = slot_pos[static_cast<size_t>(t) * k + j];
-      if (r < 0) continue;
-      float v[8];
-      unpack8(dxp[static_cast<size_t>(r) * oct + c], v);
+    for (int j0 = 0; j0 < k; j0 += KB) {
+      uint4 v[KB];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += v[i];
+      for (int q = 0; q < KB; ++q) {
+        const int r = __shfl_sync(0xffffffffu, my_slot, (j0 + q) & 31);
+        v[q] = (j0 + q < k && r >= 0) ? __ldcs(dxp + static_cast<size_t>(r) * oct + c)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int q = 0; q < KB; ++q) {
+        float f[8];
+        unpack8(v[q], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += f[i];
+      }
     }
     dx[static_cast<size_t>(t) * oct + c] = pack8(acc);
   }
@@ -257,18 +294,29 @@ router_grad_split_kernel(const float* __restrict__ dlogits, int T, int E, int Ep
     if (j == 1) return h2;
     return __float2bfloat16_rn(r1 - __bfloat162float(h2));
   };
-  for (int i = threadIdx.x; i < 32 * C3; i += blockDim.x) {
-    const int r = i / C3, c = i - r * C3;
+  // 16-byte stores of eight terms: eight experts of one token (adx; Ep is a
+  // multiple of 64, so the eight share the term j), eight tokens of one
+  // expert (adw)
+  const int c8n = C3 / 8;
+  for (int i = threadIdx.x; i < 32 * c8n; i += blockDim.x) {
+    const int r = i / c8n, c = (i - r * c8n) * 8;
     if (t0 + r >= T) continue;
-    const int j = c / Ep, e = c - j * Ep;
-    adx[static_cast<size_t>(t0 + r) * C3 + c] = term(e < E ? s_v[r * ld + e] : 0.f, j);
+    const int j = c / Ep, e0 = c - j * Ep;
+    __align__(16) __nv_bfloat16 h[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) h[q] = term(e0 + q < E ? s_v[r * ld + e0 + q] : 0.f, j);
+    *reinterpret_cast<uint4*>(adx + static_cast<size_t>(t0 + r) * C3 + c) =
+        *reinterpret_cast<const uint4*>(h);
   }
   const int g = t0 / Ks, k0 = t0 - g * Ks;
-  for (int i = threadIdx.x; i < C3 * 32; i += blockDim.x) {
-    const int row = i >> 5, r = i & 31;
+  for (int i = threadIdx.x; i < C3 * 4; i += blockDim.x) {
+    const int row = i >> 2, r0 = (i & 3) * 8;
     const int j = row / Ep, e = row - j * Ep;
-    adw[(static_cast<size_t>(g) * C3 + row) * Ks + k0 + r] =
-        term(e < E ? s_v[r * ld + e] : 0.f, j);
+    __align__(16) __nv_bfloat16 h[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) h[q] = term(e < E ? s_v[(r0 + q) * ld + e] : 0.f, j);
+    *reinterpret_cast<uint4*>(adw + (static_cast<size_t>(g) * C3 + row) * Ks + k0 + r0) =
+        *reinterpret_cast<const uint4*>(h);
   }
 }
 
