@@ -473,8 +473,12 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         pb = path_bytes(shape)
         t_path = (phases[0] + phases[1] + phases[5]) * 1e-3
         path_gbs = sum(pb.values()) / t_path / 1e9
-        router_launches = 2   # bf16: fused TC router + refine; fp32: logits + select
-        per_step_launches = router_launches + 3 + 2 + 2 * shape.n_shared + 1 + 1
+        # router 2 (bf16: tensor-core router + refine; fp32: logits + select),
+        # dispatch 2 (rank with the scan, scatter), experts 2 (bf16: the shared
+        # expert runs inside the routed launches; fp32: 2 more for it),
+        # combine 1, bias update 1
+        shared_launches = 0 if shape.dtype == I.DTYPE_BF16 else 2 * shape.n_shared
+        per_step_launches = 2 + 2 + 2 + shared_launches + 1 + 1
         l2 = ("flushed: a 504 MB buffer is written before every timed step (the step's data "
               "would fit in L2)" if flush else
               f"not flushed: each step streams {step_bytes(shape) / 1e9:.2f} GB (weights + "
