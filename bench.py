@@ -73,6 +73,24 @@ def traffic_note(s: I.MoEShape) -> str:
             f"({same})")
 
 
+def near_tie_exclusions(s: I.MoEShape) -> dict:
+    """Tokens the parity bar excludes on this workload (the oracle's k-th and
+    (k+1)-th selection keys closer than 1e-6), as counted by
+    tests/golden/make_near_ties.py from the oracle; the GPU tests compare
+    every other token bit for bit."""
+    path = os.path.join(ROOT, "tests", "golden", "near_ties.json")
+    try:
+        with open(path) as f:
+            g = json.load(f)
+        w = g["workloads"][s.name]
+        if w["T"] != s.T:
+            return {"count": None, "note": f"counted at T={w['T']}, this run has T={s.T}"}
+        return {"count": w["excluded"], "of_tokens": w["T"], "rule": g["rule"],
+                "source": "tests/golden/near_ties.json"}
+    except (OSError, KeyError, ValueError):
+        return {"count": None, "note": "not counted for this workload"}
+
+
 def describe(s: I.MoEShape) -> str:
     gate = "softmax" if s.gate == I.GATE_SOFTMAX else "sigmoid"
     dt = "bf16" if s.dtype == I.DTYPE_BF16 else "fp32"
@@ -514,6 +532,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
                     "copies": "pinned host, one cudaMemcpyAsync per tensor per step, "
                               "double-buffered on two copy streams"},
             "router_refined_tokens_last_step": refined,
+            "near_tie_exclusions": near_tie_exclusions(shape),
             "gpu_launches": per_step_launches * args.steps,
             "clocks": clocks,
         }
