@@ -56,7 +56,7 @@ def layer_flops(s: I.MoEShape) -> dict:
 # DRAM bytes per launch of the routed gate/up GEMM, from the ncu capture in
 # profiles/grouped_gemm_gateup_qwen3_30b.md, and the kernel source it was
 # taken on (sha256 of csrc/grouped_gemm_sm100.cu, first 16 hex digits).
-GATEUP_TRAFFIC = {"qwen3_30b": (1537016064, "8281548d44192e04")}
+GATEUP_TRAFFIC = {"qwen3_30b": (1844455168, "4723d615b7c2e7f9")}
 
 
 def traffic_note(s: I.MoEShape) -> str:
