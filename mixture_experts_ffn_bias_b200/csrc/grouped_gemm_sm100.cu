@@ -238,6 +238,13 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_of
   return t;
 }
 
+// L2 hints of the pair kernel: the output tiles (h, y_perm: not read again
+// by this kernel) are stored evict-first so they do not push out the A and
+// B tiles that the other n-tile / m-tile pairs are about to re-read; A tiles
+// can be loaded evict-last.
+constexpr bool kStoreEvictFirst = true;
+constexpr bool kLoadAEvictLast = false;
+
 template <int BN_ACC, int MODE, bool GATHER>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -340,6 +347,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     int stage = 0;
     uint32_t phase = 0, issued_mask = 0, issued_phase = 0;
     bool ok = true;
+    const uint64_t a_policy = kLoadAEvictLast ? l2_policy_evict_last() : 0ull;
     // without gathers lane 0 alone drives the ring
     for (int tile = pair; tile < total_tiles && ok && (GATHER || lane == 0); tile += npairs) {
       const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
@@ -369,8 +377,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         if (!w_ok) { ok = false; break; }
         if (lane == 0) {
           if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * Cfg::STAGE_BYTES);
-          if (!gathered)
-            tma_load_2d_pair(smemA + stage * A_STAGE_BYTES, ma, &full_bar[stage], kb * BK, arow);
+          if (!gathered) {
+            if (kLoadAEvictLast)
+              tma_load_2d_pair_hint(smemA + stage * A_STAGE_BYTES, ma, &full_bar[stage], kb * BK,
+                                    arow, a_policy);
+            else
+              tma_load_2d_pair(smemA + stage * A_STAGE_BYTES, ma, &full_bar[stage], kb * BK,
+                               arow);
+          }
           if (BMN) {
             // this CTA's BN_ACC/2 columns of B, 64 columns (one box) at a time
             const bool first = kb < args.kb_split;
@@ -453,6 +467,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
+    const uint64_t c_policy = kStoreEvictFirst ? l2_policy_evict_first() : 0ull;
     int it = 0;
     for (int tile = pair; tile < total_tiles; tile += npairs, ++it) {
       const int acc = it % NACC;
@@ -589,7 +604,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           fence_async_shared();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(mc, stage_buf, ocol, warp_row0);
+            if (kStoreEvictFirst)
+              tma_store_2d_hint(mc, stage_buf, ocol, warp_row0, c_policy);
+            else
+              tma_store_2d(mc, stage_buf, ocol, warp_row0);
             bulk_commit();
           }
         } else if (valid) {
