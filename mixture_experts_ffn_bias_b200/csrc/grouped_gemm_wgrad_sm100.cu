@@ -237,6 +237,9 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
   } else {
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    // the weight gradients are not read again here: stored evict-first, so
+    // the L2 keeps the activation tiles other CTAs are about to re-read
+    const uint64_t c_policy = l2_policy_evict_first();
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const int g = tile / (MT * NT);
@@ -283,7 +286,7 @@ wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
         fence_async_shared();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmC, stage_buf, n * BN + cb * 64, crow0);
+          tma_store_2d_hint(&tmC, stage_buf, n * BN + cb * 64, crow0, c_policy);
           bulk_commit();
         }
       }
