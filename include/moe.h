@@ -270,15 +270,24 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  *   gather_rows 1 (bf16 layers only): dispatch writes no x_perm; the gate/up
  *     GEMM gathers each tile's rows from x through the permutation (TMA
  *     tile::gather4 loads, four rows per load).  Same results.
+ *   fold_combine 0 (default): a separate combine launch reads y_perm (and
+ *     the shared expert's rows) and writes out.
+ *   fold_combine 1 (bf16 layers only): the down GEMM forms out itself: after
+ *     a warp stores its 32 rows of an output tile it counts them per token,
+ *     and the warp that completes a token's column tile (its k routed rows
+ *     and the shared row) sums them into out in the combine's order.  Same
+ *     results; one launch fewer, but measured slower on B200 (the summing
+ *     warps hold the down GEMM's epilogue).  Combinable with gather_rows.
  *   reserved: must be 0. */
 typedef struct {
   int32_t gather_rows;
-  int32_t reserved[3];
+  int32_t fold_combine;
+  int32_t reserved[2];
 } moe_forward_opts;
 
 /* moe_forward with the options above (opts must not be NULL; a field
- * outside its values is MOE_ERR_INVALID; gather_rows on an fp32 layer is
- * MOE_ERR_UNSUPPORTED). */
+ * outside its values is MOE_ERR_INVALID; gather_rows or fold_combine on an
+ * fp32 layer is MOE_ERR_UNSUPPORTED). */
 moe_status moe_forward_ex(const moe_config* cfg, const void* x, const void* w_router,
                           const float* sel_bias, const float* logit_offset,
                           const moe_expert_weights* w, void* out,

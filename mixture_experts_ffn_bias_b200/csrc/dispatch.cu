@@ -87,11 +87,14 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
 // out, takes a ticket; the last block to finish turns all block counts into
 // block bases, counts and offsets (the same arithmetic as the scan kernel
 // below), then puts the ticket counter back to zero.  done: zero at launch.
+// fold_cnt (or null): the folded combine's per-(token, column tile) counts,
+// set to the number of the token's skipped pairs (rows that never arrive).
 __global__ void __launch_bounds__(kRankBlock)
 dispatch_rank_scan_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E,
                           int32_t* __restrict__ blk, int32_t* __restrict__ rank_out,
                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                          uint32_t* __restrict__ status, uint32_t* __restrict__ done) {
+                          uint32_t* __restrict__ status, uint32_t* __restrict__ done,
+                          int32_t* __restrict__ fold_cnt, int fold_nt) {
   pdl_trigger();
   pdl_wait();
   __shared__ uint32_t masks[kMaxE][kWords];
@@ -125,6 +128,11 @@ dispatch_rank_scan_kernel(const int32_t* __restrict__ topk_idx, int T, int k, in
     }
   }
   if (bad) atomicOr(status, kDevBadIndex);
+  if (fold_cnt != nullptr && t < T) {
+    int skipped = 0;
+    for (int j = 0; j < k; ++j) skipped += pair_valid(row, j, E) ? 0 : 1;
+    for (int c = 0; c < fold_nt; ++c) fold_cnt[static_cast<size_t>(t) * fold_nt + c] = skipped;
+  }
   for (int e = tid; e < E; e += kRankBlock) {
     int c = 0;
 #pragma unroll
@@ -315,10 +323,12 @@ cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t*
 
 cudaError_t dispatch_rank_scan(const int32_t* topk_idx, int T, int k, int E, int32_t* blk,
                                int32_t* rank_out, int32_t* counts, int32_t* offsets,
-                               uint32_t* status, uint32_t* done, cudaStream_t stream) {
+                               uint32_t* status, uint32_t* done, cudaStream_t stream,
+                               int32_t* fold_cnt, int fold_nt) {
   if (E > kMaxE || kRankBlock != kMaxE) return cudaErrorInvalidValue;
   return launch_pdl(dispatch_rank_scan_kernel, dim3(rank_blocks(T)), dim3(kRankBlock), 0, stream,
-                    topk_idx, T, k, E, blk, rank_out, counts, offsets, status, done);
+                    topk_idx, T, k, E, blk, rank_out, counts, offsets, status, done, fold_cnt,
+                    fold_nt);
 }
 
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,

@@ -88,6 +88,21 @@ struct GemmArgs {
   int gather_limit;            // GATHER: entries of gather_rows
   int gather_src_rows;         // GATHER: rows of gather_src
   const void* aux;             // SWIGLU_BWD: dH [rows, n_per_group] bf16
+  // Combine folded into a plain pass (null: not folded).  C is y_perm [R,
+  // n], x_C the shared expert's y_sh [T, n] (or no extra group).  For each
+  // (token, output tile) fold_cnt counts the rows written; the warp whose
+  // row brings it to fold_target (k, plus 1 with a shared expert) forms
+  // out[t] = y_sh[t] + sum_j w[t, j] y_perm[slot[t, j]] over those columns,
+  // in j order, as the separate combine would.
+  int32_t* fold_cnt;           // [T, fold_nt], the token's skipped pairs at launch
+  int fold_nt;
+  int fold_T;
+  int fold_target;
+  int fold_k;
+  const int32_t* fold_src;     // perm_src [R]: token of each routed row
+  const int32_t* fold_slot;    // slot_pos [T, k]
+  const float* fold_w;         // topk_w [T, k]
+  void* fold_out;              // out [T, n] bf16
 };
 
 // Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
@@ -214,11 +229,27 @@ struct PairCfg {
 };
 
 template <int BN_OUT>
+__device__ __forceinline__ int extra_tiles(const GemmArgs& a) {
+  return a.x_rows > 0 ? (a.x_rows + BM2 - 1) / BM2 * ((a.x_n + BN_OUT - 1) / BN_OUT) : 0;
+}
+
+// Whether `tile` is one of the extra group's.  They follow the routed
+// groups' tiles, except under the folded combine, where they come first:
+// every token's output waits for its shared-expert row, so those rows are
+// done early.
+__device__ __forceinline__ bool is_extra_tile(const GemmArgs& a, int routed_tiles, int x_tiles,
+                                              int tile) {
+  return a.fold_cnt != nullptr ? tile < x_tiles : tile >= routed_tiles;
+}
+
+template <int BN_OUT>
 __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_off,
                                               const int* s_prefix, int G, int n_tiles, int tile) {
   PairTile t;
-  if (tile >= s_prefix[G]) {
-    const int local = tile - s_prefix[G];
+  const int xt = extra_tiles<BN_OUT>(a);
+  const bool first = a.fold_cnt != nullptr;
+  if (is_extra_tile(a, s_prefix[G], xt, tile)) {
+    const int local = first ? tile : tile - s_prefix[G];
     const int xn = (a.x_n + BN_OUT - 1) / BN_OUT;
     t.x = true;
     t.g = 0;
@@ -228,6 +259,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_of
     t.rows = a.x_rows;
     t.kblocks = a.x_K / BK;
   } else {
+    if (first) tile -= xt;
     t.x = false;
     t.g = find_group(s_prefix, G, tile);
     t.row0 = s_off[t.g];
@@ -236,6 +268,99 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_of
     t.kblocks = a.K / BK;
   }
   return t;
+}
+
+// Folded combine, run by an epilogue warp once it has stored its 32 rows of
+// an output tile (columns [n BN_OUT, (n+1) BN_OUT) clipped to ncols).  The
+// stores are completed and published (TMA stores waited for, then a release
+// fence), each row's token takes a count for this column tile, and a warp
+// whose row brings a token to fold_target forms that token's output columns:
+// out[t] = y_sh[t] + sum_j w[t, j] y_perm[slot[t, j]], fp32 in j order, as
+// combine_kernel does, from L2 (the rows were written by other CTAs).  All
+// control flow around the shuffles is warp-uniform.
+template <int BN_OUT>
+__device__ __forceinline__ void fold_combine_rows(const GemmArgs& a, bool extra, int n, int ncols,
+                                                  bool valid, int warp_row0, int lane) {
+  if (lane == 0) bulk_wait_all();   // this warp's TMA stores have completed
+  __syncwarp();
+  __threadfence();                  // release: the rows before their counts
+  int t = -1;
+  if (valid) t = extra ? warp_row0 + lane : __ldg(a.fold_src + warp_row0 + lane);
+  bool last = false;
+  if (t >= 0 && t < a.fold_T) {
+    const int old = atomicAdd(a.fold_cnt + static_cast<size_t>(t) * a.fold_nt + n, 1);
+    last = old == a.fold_target - 1;
+  }
+  uint32_t todo = __ballot_sync(0xffffffffu, last);
+  if (todo == 0u) return;
+  __threadfence();   // acquire: the other rows of these tokens are visible from here on
+  const int k = a.fold_k;
+  const __nv_bfloat16* yp = static_cast<const __nv_bfloat16*>(a.C);
+  const __nv_bfloat16* ysh = static_cast<const __nv_bfloat16*>(a.x_C);
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.fold_out);
+  const long long rmax = static_cast<long long>(a.fold_T) * k;
+  while (todo != 0u) {
+    const int src = __ffs(todo) - 1;
+    todo &= todo - 1u;
+    const int tt = __shfl_sync(0xffffffffu, t, src);
+    int my_slot = -1;
+    float my_w = 0.f;
+    if (lane < k) {
+      my_slot = a.fold_slot[static_cast<size_t>(tt) * k + lane];
+      my_w = a.fold_w[static_cast<size_t>(tt) * k + lane];
+      if (static_cast<long long>(my_slot) >= rmax) my_slot = -1;
+    }
+    // lanes whose columns lie past ncols (a partial last tile) load and
+    // store nothing but still take part in the shuffles
+    for (int c0 = 0; c0 < BN_OUT; c0 += 256) {
+      const int col = n * BN_OUT + c0 + lane * 8;
+      const bool in = col < ncols;
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      if (ysh != nullptr && in) {
+        const uint4 v =
+            __ldcg(reinterpret_cast<const uint4*>(ysh + static_cast<size_t>(tt) * a.x_ldc + col));
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h[i]);
+          acc[2 * i] = f.x;
+          acc[2 * i + 1] = f.y;
+        }
+      }
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        uint4 v[8];
+        float wj[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + q;
+          const int sl = __shfl_sync(0xffffffffu, my_slot, j & 31);
+          wj[q] = __shfl_sync(0xffffffffu, my_w, j & 31);
+          v[q] = (in && j < k && sl >= 0)
+                     ? __ldcg(reinterpret_cast<const uint4*>(yp + static_cast<size_t>(sl) * a.ldc +
+                                                             col))
+                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (j0 + q >= k) break;
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[q]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __bfloat1622float2(h[i]);
+            acc[2 * i] = fmaf(wj[q], f.x, acc[2 * i]);
+            acc[2 * i + 1] = fmaf(wj[q], f.y, acc[2 * i + 1]);
+          }
+        }
+      }
+      uint4 o;
+      uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) op[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+      if (in) *reinterpret_cast<uint4*>(out + static_cast<size_t>(tt) * ncols + col) = o;
+    }
+  }
 }
 
 // L2 hints of the pair kernel: the output tiles (h, y_perm: not read again
@@ -331,8 +456,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
 
   const uint32_t tmem_base = s_tmem_base;
-  const int x_tiles =
-      args.x_rows > 0 ? (args.x_rows + BM2 - 1) / BM2 * ((args.x_n + BN_OUT - 1) / BN_OUT) : 0;
+  const int x_tiles = extra_tiles<BN_OUT>(args);
   const int total_tiles = s_prefix[G] + x_tiles;
   volatile int* abort_flag = &s_abort;
 
@@ -431,7 +555,8 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int tile = pair; tile < total_tiles && ok; tile += npairs, ++it) {
         const int acc = it % NACC;
         const uint32_t acc_phase = (it / NACC) & 1;
-        const int kblocks = tile >= s_prefix[G] ? args.x_K / BK : args.K / BK;
+        const int kblocks =
+            is_extra_tile(args, s_prefix[G], x_tiles, tile) ? args.x_K / BK : args.K / BK;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN_ACC;
@@ -621,6 +746,10 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_rank0(&tempty_bar[acc]);
+      if constexpr (MODE == MODE_PLAIN_BF16) {
+        if (args.fold_cnt != nullptr)
+          fold_combine_rows<BN_OUT>(args, pt.x, n, ncols, valid, warp_row0, lane);
+      }
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -810,22 +939,26 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
 
 // Y[r] = A[r] W2[g]^T, bf16 out; N = output columns per group.  extra: one
 // more group (the shared expert's down projection, same N), same launch.
+// Output columns per tile of grouped_down_bf16 for N x K: 512 accumulator
+// columns (one TMEM buffer) only for long K, where the exposed epilogue is a
+// small part of a tile: measured on B200, wide's down GEMM (K = 4352) 0.616
+// -> 0.551 ms, but qwen3_30b's (K = 768) 0.33 -> 0.38 ms.  N a multiple of
+// 128 but not of 256 (page-2 shape, d = 640): 256-column tiles with a
+// half-empty last one beat 128-column tiles, whose A tile is streamed twice
+// as often per MMA flop.
+int down_tile_cols(int N, int K) {
+  return (N % 512 == 0 && K >= 4096) ? 512
+         : (N % 256 == 0 || (N % 128 == 0 && N > 256)) ? 256 : 128;
+}
+
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream,
-                              const GemmExtraGroup* extra) {
+                              const GemmExtraGroup* extra, const GemmFold* fold) {
   CUtensorMap ta, tb, tc, xa, xb, xc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * N;
   const int64_t c_rows = offsets ? a_rows : rows_single;
-  // 512 accumulator columns (one TMEM buffer) only for long K, where the
-  // exposed epilogue is a small part of a tile: measured on B200, wide's
-  // down GEMM (K = 4352) 0.616 -> 0.551 ms, but qwen3_30b's (K = 768) 0.33 ->
-  // 0.38 ms
-  // N a multiple of 128 but not of 256 (page-2 shape, d = 640): 256-column
-  // tiles with a half-empty last one beat 128-column tiles, whose A tile
-  // is streamed twice as often per MMA flop.
-  const int bn = (N % 512 == 0 && K >= 4096) ? 512
-                 : (N % 256 == 0 || (N % 128 == 0 && N > 256)) ? 256 : 128;
+  const int bn = down_tile_cols(N, K);
   // each CTA of the pair loads half of the B tile
   if (!make_map(&ta, A, a_rows, K, BM) || !make_map(&tb, W2, b_rows, K, bn / 2) ||
       !make_map(&tc, Y, c_rows, N, 32))
@@ -844,6 +977,21 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
     args.x_ldc = N;
   } else {
     xa = ta; xb = tb; xc = tc;
+  }
+  if (fold != nullptr) {
+    const bool shared = extra != nullptr && extra->rows > 0;
+    if (fold->nt != (N + bn - 1) / bn || (shared && extra->rows != fold->T) || fold->k < 1 ||
+        fold->k > 32 || !fold->cnt || !fold->src || !fold->slot || !fold->w || !fold->out)
+      return cudaErrorInvalidValue;
+    args.fold_cnt = fold->cnt;
+    args.fold_nt = fold->nt;
+    args.fold_T = fold->T;
+    args.fold_target = fold->k + (shared ? 1 : 0);
+    args.fold_k = fold->k;
+    args.fold_src = fold->src;
+    args.fold_slot = fold->slot;
+    args.fold_w = fold->w;
+    args.fold_out = fold->out;
   }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   if (bn == 512)

@@ -78,9 +78,12 @@ cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t*
                           int32_t* rank_out, uint32_t* status, cudaStream_t stream);
 // dispatch_rank followed by dispatch_scan in one launch (the last block to
 // finish scans); done: a zeroed counter, zero again when the kernel ends.
+// fold_cnt [T, fold_nt] (or null) is set to each token's skipped pairs, the
+// starting counts of the combine folded into the down pass.
 cudaError_t dispatch_rank_scan(const int32_t* topk_idx, int T, int k, int E, int32_t* blk,
                                int32_t* rank_out, int32_t* counts, int32_t* offsets,
-                               uint32_t* status, uint32_t* done, cudaStream_t stream);
+                               uint32_t* status, uint32_t* done, cudaStream_t stream,
+                               int32_t* fold_cnt = nullptr, int fold_nt = 0);
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream);
 // slot_pos (in: rank inside its block of blk_tokens tokens, out: row) and
@@ -122,10 +125,23 @@ cudaError_t grouped_swiglu_bwd_bf16(const void* A, int64_t a_rows, const int32_t
                                     int num_groups, int rows_single, const void* W1,
                                     const void* W3, int F, int K, const void* dH, void* dGU,
                                     uint32_t* status, cudaStream_t stream);
+// The combine folded into the down pass (see GemmArgs in
+// grouped_gemm_sm100.cu): counts [T, nt] set by dispatch_rank_scan, nt =
+// ceil(N / down_tile_cols(N, K)); out [T, N] receives the combined rows.
+struct GemmFold {
+  int32_t* cnt;
+  int nt, T, k;
+  const int32_t* src;    // perm_src [T k]
+  const int32_t* slot;   // slot_pos [T, k]
+  const float* w;        // topk_w [T, k]
+  void* out;
+};
+int down_tile_cols(int N, int K);
 cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                               int num_groups, int rows_single, const void* W2, int N, int K,
                               void* Y, uint32_t* status, cudaStream_t stream,
-                              const GemmExtraGroup* extra = nullptr);
+                              const GemmExtraGroup* extra = nullptr,
+                              const GemmFold* fold = nullptr);
 // Y[r] = A[r] B_g, B_g [K, N] read MN-major (no transposed copy): its first
 // b0_rows rows from B0 [G * b0_rows, N], the others from B1.
 cudaError_t grouped_gemm_bmn_bf16(const void* A, int64_t a_rows, const int32_t* offsets,

@@ -16,7 +16,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
   size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, stats, logits, x_perm, h,
-      y_perm, h_sh, y_sh, total;
+      y_perm, h_sh, y_sh, fold, total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -42,6 +42,9 @@ Layout layout(const moe_config& c) {
   L.y_perm = o;   o += up(R * d * es);
   L.h_sh = o;     o += up(T * Fs * es);
   L.y_sh = o;     o += up(c.n_shared ? T * d * es : 0);
+  // the folded combine's counts: [T, column tiles of the down GEMM], at
+  // most d / 128 tiles (bf16 only)
+  L.fold = o;     o += up(c.dtype == MOE_BF16 ? T * ((d + 127) / 128) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -142,14 +145,16 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
   return MOE_OK;
 }
 
+// fold_nt > 0: also set the folded combine's counts ([T, fold_nt] in ws).
 moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void* x,
                        int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_src,
-                       void* x_perm, void* ws, cudaStream_t s) {
+                       void* x_perm, void* ws, cudaStream_t s, int fold_nt = 0) {
   const Layout L = layout(*c);
   int32_t* blk = at<int32_t>(ws, L.blk);
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_TRY(moe::dispatch_rank_scan(topk_idx, c->T, c->top_k, c->n_experts, blk, slot_pos, counts,
-                                  offsets, status, status + 3, s));
+                                  offsets, status, status + 3, s,
+                                  fold_nt > 0 ? at<int32_t>(ws, L.fold) : nullptr, fold_nt));
   if (x_perm == nullptr) {   // rows only; the experts gather x through perm_src
     MOE_TRY(moe::dispatch_positions(topk_idx, blk, slot_pos, perm_src, c->T, c->top_k,
                                     c->n_experts, moe::kRankBlock, s));
@@ -172,10 +177,12 @@ struct Marks {
 
 // x_perm == nullptr (bf16 only): the gate/up GEMM gathers its rows from x
 // through gather_rows (perm_src) instead of reading a permuted copy.
+// fold (bf16 only): the down GEMM also forms the combined output.
 moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* offsets,
                        const moe_expert_weights* w, const void* x, void* y_perm, void* y_shared,
                        void* ws, cudaStream_t s, const Marks& mk,
-                       const int32_t* gather_rows = nullptr) {
+                       const int32_t* gather_rows = nullptr,
+                       const moe::GemmFold* fold = nullptr) {
   const Layout L = layout(*c);
   uint32_t* status = at<uint32_t>(ws, L.status);
   const int64_t R = static_cast<int64_t>(c->T) * c->top_k;
@@ -197,7 +204,7 @@ moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* o
     }
     if (!mk.rec(3)) return MOE_ERR_CUDA;
     MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s,
-                                   c->n_shared ? &sh_down : nullptr));
+                                   c->n_shared ? &sh_down : nullptr, fold));
     if (!mk.rec(4)) return MOE_ERR_CUDA;
   } else {
     float* hf = static_cast<float*>(h);
@@ -241,11 +248,13 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   moe_status st = check_cfg(cfg);
   if (st != MOE_OK) return st;
   if (opts != nullptr &&
-      ((opts->gather_rows != 0 && opts->gather_rows != 1) || opts->reserved[0] != 0 ||
-       opts->reserved[1] != 0 || opts->reserved[2] != 0))
+      ((opts->gather_rows != 0 && opts->gather_rows != 1) ||
+       (opts->fold_combine != 0 && opts->fold_combine != 1) || opts->reserved[0] != 0 ||
+       opts->reserved[1] != 0))
     return MOE_ERR_INVALID;
   const bool gather = opts != nullptr && opts->gather_rows == 1;
-  if (gather && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const bool fold = opts != nullptr && opts->fold_combine == 1;
+  if ((gather || fold) && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!counts) return MOE_ERR_INVALID;
   if (cfg->T == 0) {
     MOE_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, S(stream)));
@@ -282,15 +291,24 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   // gathers the same rows again).
   int32_t* perm_src = at<int32_t>(ws, L.perm_src);
   if (gather) MOE_TRY(cudaMemsetAsync(at<uint32_t>(ws, L.status) + 2, 0xff, sizeof(uint32_t), s));
+  // fold_combine: the down GEMM's epilogue forms out (dispatch sets its
+  // per-token counts); no combine launch
+  const int fold_nt =
+      fold ? (cfg->d_model + moe::down_tile_cols(cfg->d_model, cfg->d_ff) - 1) /
+                 moe::down_tile_cols(cfg->d_model, cfg->d_ff)
+           : 0;
   if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
-                        gather ? nullptr : x_perm, ws, s)) != MOE_OK)
+                        gather ? nullptr : x_perm, ws, s, fold_nt)) != MOE_OK)
     return st;
   if (!mk.rec(2)) return MOE_ERR_CUDA;
+  const moe::GemmFold gf{at<int32_t>(ws, L.fold), fold_nt, cfg->T, cfg->top_k, perm_src,
+                         slot_pos, topk_w, out};
   if ((st = run_experts(cfg, gather ? nullptr : x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk,
-                        perm_src)) != MOE_OK)
+                        perm_src, fold ? &gf : nullptr)) != MOE_OK)
     return st;
-  MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_sh, out, cfg->T,
-                       cfg->d_model, cfg->top_k, s));
+  if (!fold)
+    MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_sh, out, cfg->T,
+                         cfg->d_model, cfg->top_k, s));
   if (!mk.rec(MOE_FORWARD_PHASES)) return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -130,6 +130,29 @@ def test_forward_with_gathered_gate_up_rows(name):
     _check_layer(shape, host, layer)
 
 
+@pytest.mark.parametrize("name,gather", [("page2_small", False), ("qwen3_small", False),
+                                         ("skew_small", True), ("qwen3_30b", False),
+                                         ("skew", False)])
+def test_forward_with_folded_combine(name, gather):
+    """The alternative (moe_forward_ex, fold_combine = 1) whose down GEMM
+    forms the combined output: against the oracle, and bit for bit against
+    the default path's separate combine (the same fp32 operations in the same
+    order).  page2_small's d = 640 ends in a half-empty 256-column tile; skew
+    has experts that no token chose."""
+    shape = SMALL[name] if name in SMALL else I.WORKLOADS[name]
+    host = I.make_inputs(shape)
+    layer = MoELayer(shape, host)
+    layer.forward()
+    torch.cuda.synchronize()
+    ref = layer.out.clone()
+    layer.out.fill_(float("nan"))
+    layer.forward(gather_rows=gather, fold_combine=True)
+    torch.cuda.synchronize()
+    assert layer.device_status()[0] == B.MOE_OK
+    assert torch.equal(layer.out.view(torch.int16), ref.view(torch.int16))
+    _check_layer(shape, host, layer)
+
+
 def test_skew_bias_update_then_deferred_forward():
     """Skewed workload: forward, bias update from its counts (bit-exact), then a
     second forward routes with the new bias (the update lands on the next
