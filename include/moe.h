@@ -278,16 +278,24 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  *     and the shared row) sums them into out in the combine's order.  Same
  *     results; one launch fewer, but measured slower on B200 (the summing
  *     warps hold the down GEMM's epilogue).  Combinable with gather_rows.
+ *   scatter_in_gemm 1 (bf16 layers only; not with gather_rows): dispatch
+ *     writes only the rows' positions, and the gate/up GEMM launch fills
+ *     x_perm itself while it runs: four extra warps per CTA copy x's rows in
+ *     row order and count them per 32-row block, and each tile's loads wait
+ *     (bounded) for the blocks of its rows.  Same results; x_perm is kept
+ *     for moe_backward as with the default.
  *   reserved: must be 0. */
 typedef struct {
   int32_t gather_rows;
   int32_t fold_combine;
-  int32_t reserved[2];
+  int32_t scatter_in_gemm;
+  int32_t reserved[1];
 } moe_forward_opts;
 
 /* moe_forward with the options above (opts must not be NULL; a field
- * outside its values is MOE_ERR_INVALID; gather_rows or fold_combine on an
- * fp32 layer is MOE_ERR_UNSUPPORTED). */
+ * outside its values, or gather_rows with scatter_in_gemm, is
+ * MOE_ERR_INVALID; any of the three on an fp32 layer is
+ * MOE_ERR_UNSUPPORTED). */
 moe_status moe_forward_ex(const moe_config* cfg, const void* x, const void* w_router,
                           const float* sel_bias, const float* logit_offset,
                           const moe_expert_weights* w, void* out,

@@ -54,7 +54,7 @@ class MoEExpertGrads(ctypes.Structure):
 
 class MoEForwardOpts(ctypes.Structure):
     _fields_ = [("gather_rows", ctypes.c_int32), ("fold_combine", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 2)]
+                ("scatter_in_gemm", ctypes.c_int32), ("reserved", ctypes.c_int32 * 1)]
 
 
 class MoERouterOpts(ctypes.Structure):
@@ -267,13 +267,15 @@ def moe_forward(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, to
 
 
 def moe_forward_ex(cfg, x, w_router, sel_bias, logit_offset, weights: Dict, out, topk_idx,
-                   topk_w, counts, ws, gather_rows=0, fold_combine=0, stream=None,
-                   check=True) -> int:
+                   topk_w, counts, ws, gather_rows=0, fold_combine=0, scatter_in_gemm=0,
+                   stream=None, check=True) -> int:
     """moe_forward with the expert-path options (gather_rows=1: the gate/up
     GEMM gathers its rows from x instead of reading a permuted copy;
-    fold_combine=1: the down GEMM forms the combined output itself)."""
+    fold_combine=1: the down GEMM forms the combined output itself;
+    scatter_in_gemm=1: the gate/up GEMM fills the permuted copy while it
+    runs)."""
     w = expert_weights(weights)
-    opts = MoEForwardOpts(int(gather_rows), int(fold_combine))
+    opts = MoEForwardOpts(int(gather_rows), int(fold_combine), int(scatter_in_gemm))
     st = lib().moe_forward_ex(ctypes.byref(cfg), _p(x), _p(w_router), _p(sel_bias),
                               _p(logit_offset), ctypes.byref(w), _p(out), _p(topk_idx),
                               _p(topk_w), _p(counts), ctypes.byref(opts), _p(ws),

@@ -284,14 +284,16 @@ dispatch_scatter_kernel(const uint4* __restrict__ x, const int32_t* __restrict__
   }
 }
 
-// One thread per token: final rows and the token of each row, no copy.
+// One thread per token: final rows and the token of each row, no copy;
+// zero[0, n_zero) set to zero on the way.
 __global__ void __launch_bounds__(256)
 dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ bases,
                           int32_t* __restrict__ slot_pos, int32_t* __restrict__ perm_src, int T,
-                          int k, int E, int blk_tokens) {
+                          int k, int E, int blk_tokens, int32_t* __restrict__ zero, int n_zero) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  for (int i = t; i < n_zero; i += gridDim.x * blockDim.x) zero[i] = 0;
   if (t >= T) return;
   const int32_t* b = bases + static_cast<size_t>(t / blk_tokens) * E;
   for (int j = 0; j < k; ++j) {
@@ -310,9 +312,10 @@ dispatch_positions_kernel(const int32_t* __restrict__ topk_idx, const int32_t* _
 
 cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
                                int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
-                               int blk_tokens, cudaStream_t stream) {
+                               int blk_tokens, cudaStream_t stream, int32_t* zero, int n_zero) {
   return launch_pdl(dispatch_positions_kernel, dim3((T + 255) / 256), dim3(256), 0, stream,
-                    topk_idx, blk_bases, slot_pos, perm_src, T, k, E, blk_tokens);
+                    topk_idx, blk_bases, slot_pos, perm_src, T, k, E, blk_tokens, zero,
+                    zero != nullptr ? n_zero : 0);
 }
 
 cudaError_t dispatch_rank(const int32_t* topk_idx, int T, int k, int E, int32_t* blk_counts,

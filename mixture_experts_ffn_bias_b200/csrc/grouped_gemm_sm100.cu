@@ -44,6 +44,10 @@ constexpr int BM = 128;
 constexpr int BK = 64;                    // 64 bf16 = 128 bytes = one swizzle row
 constexpr int A_STAGE_BYTES = BM * BK * 2;
 constexpr int NUM_THREADS = 192;          // 6 warps
+// A gate/up launch that fills its own A rows runs COPY_WARPS more warps.
+constexpr int COPY_WARPS = 2;
+constexpr int NUM_THREADS_COPY = NUM_THREADS + 32 * COPY_WARPS;
+
 constexpr int MAX_GROUPS = 257;
 
 
@@ -103,6 +107,16 @@ struct GemmArgs {
   const int32_t* fold_slot;    // slot_pos [T, k]
   const float* fold_w;         // topk_w [T, k]
   void* fold_out;              // out [T, n] bf16
+  // A rows filled by the launch itself (gate/up, null: A is complete at
+  // launch).  Warps 6.. copy row r of A (cp_dst) from row cp_perm[r] of
+  // cp_src, in increasing row order over all CTAs, and add the rows to
+  // cp_ready[1 + r / 32] once they are stored; a producer waits for the blocks
+  // of its tile's A rows before loading them.
+  const void* cp_src;          // x [cp_src_rows, K] bf16
+  const int32_t* cp_perm;      // perm_src [rows]
+  int32_t* cp_ready;           // [1 + ceil(rows / 32)]: next unit, block counts; zero at launch
+  void* cp_dst;                // A = x_perm [rows, K] bf16
+  int cp_src_rows;
 };
 
 // Where a tile of the CTA-pair kernel lies: a routed group's (m, n) tile, or
@@ -363,6 +377,89 @@ __device__ __forceinline__ void fold_combine_rows(const GemmArgs& a, bool extra,
   }
 }
 
+// Copy role of a gate/up launch that fills its own A rows (see GemmArgs).
+// The rows go in 8-row units handed out in increasing order by a counter
+// (cp_ready[0]), so they complete roughly in the order the
+// tiles consume them, and only running warps take work: a producer never
+// waits for a CTA that is not resident.  Each warp asks for its next unit
+// before copying the current one, hiding the counter's latency.  x rows
+// are loaded with an L2 evict-last hint (each is read k times).  After a
+// unit's stores every lane fences, and lane 0 (fencing again after the warp
+// barrier) adds the rows to their 32-row block's count.
+__device__ __forceinline__ void copy_a_rows(const GemmArgs& a, int rows, int lane) {
+  const int vecs = a.K / 8;   // 16-byte pieces per row
+  const uint4* src = static_cast<const uint4*>(a.cp_src);
+  uint4* dst = static_cast<uint4*>(a.cp_dst);
+  const uint64_t keep = l2_policy_evict_last();
+  const int units = (rows + 7) / 8;
+  int* next = a.cp_ready;
+  int u = 0;
+  if (lane == 0) u = atomicAdd(next, 1);
+  u = __shfl_sync(0xffffffffu, u, 0);
+  while (u < units) {
+    int nu = 0;
+    if (lane == 0) nu = atomicAdd(next, 1);
+    const int r0 = u * 8;
+    const int nr = rows - r0 < 8 ? rows - r0 : 8;
+    for (int h = 0; h < 8; h += 4) {
+      size_t sb[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = r0 + h + q < rows ? r0 + h + q : rows - 1;
+        int t = __ldg(a.cp_perm + r);
+        t = (t < 0 || t >= a.cp_src_rows) ? 0 : t;
+        sb[q] = static_cast<size_t>(t) * vecs;
+      }
+      for (int c0 = 0; c0 < vecs; c0 += 128) {
+        uint4 v[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = c0 + lane + 32 * j;
+            v[q][j] =
+                c < vecs ? ld_global_hint(src + sb[q] + c, keep) : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int c = c0 + lane + 32 * j;
+            if (c < vecs && h + q < nr) dst[static_cast<size_t>(r0 + h + q) * vecs + c] = v[q][j];
+          }
+      }
+    }
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) {
+      __threadfence();
+      atomicAdd(a.cp_ready + 1 + r0 / 32, nr);
+    }
+    u = __shfl_sync(0xffffffffu, nu, 0);
+  }
+}
+
+// Producer side: wait (bounded) until the A rows [lo, hi) of a tile are
+// stored, then order the later TMA loads after that observation.  `rows`
+// is the copied total (blocks before the last hold 32 rows).
+__device__ __forceinline__ bool wait_a_rows(const GemmArgs& a, int lo, int hi, int rows,
+                                            volatile int* abort_flag) {
+  if (lo >= hi) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (int b = lo / 32; b <= (hi - 1) / 32; ++b) {
+    const int need = rows - 32 * b < 32 ? rows - 32 * b : 32;
+    while (ld_acquire_gpu(a.cp_ready + 1 + b) < need) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // L2 hints of the pair kernel: the output tiles (h, y_perm: not read again
 // by this kernel) are stored evict-first so they do not push out the A and
 // B tiles that the other n-tile / m-tile pairs are about to re-read; A tiles
@@ -370,8 +467,14 @@ __device__ __forceinline__ void fold_combine_rows(const GemmArgs& a, bool extra,
 constexpr bool kStoreEvictFirst = true;
 constexpr bool kLoadAEvictLast = false;
 
+// Threads a launch of the pair kernel may have: only the forward gate/up
+// kernel carries the copy warps.
+constexpr int pair_max_threads(int mode, bool gather) {
+  return mode == MODE_SWIGLU_BF16 && !gather ? NUM_THREADS_COPY : NUM_THREADS;
+}
+
 template <int BN_ACC, int MODE, bool GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_max_threads(MODE, GATHER), 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1,
@@ -484,6 +587,14 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const CUtensorMap* mb = (SWIGLU && rank == 1) ? (pt.x ? &tmB1_2 : &tmB1)
                                                     : (pt.x ? &tmB0_2 : &tmB0);
       const bool gathered = GATHER && !pt.x;
+      if constexpr (MODE == MODE_SWIGLU_BF16 && !GATHER) {
+        // lane 0 alone runs this loop here
+        if (args.cp_ready != nullptr && !pt.x &&
+            !wait_a_rows(args, arow, min(arow + BM, pt.row0 + pt.rows), s_off[G], abort_flag)) {
+          ok = false;
+          break;
+        }
+      }
       int tok[4] = {0, 0, 0, 0};
       if (gathered) {
 #pragma unroll
@@ -589,7 +700,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           if (globaltimer_ns() - t0 > kWaitLimitNs) break;
       }
     }
-  } else {
+  } else if (warp < NUM_THREADS / 32) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const uint64_t c_policy = kStoreEvictFirst ? l2_policy_evict_first() : 0ull;
@@ -753,6 +864,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
+  } else {
+    // ------------------------------------------------- A-row copy (gate/up)
+    if constexpr (MODE == MODE_SWIGLU_BF16 && !GATHER) {
+      if (args.cp_ready != nullptr) copy_a_rows(args, s_off[G], lane);
+    }
   }
 
   tc_fence_before();
@@ -811,7 +927,7 @@ template <int BN_ACC, int MODE, bool GATHER = false>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& c, const CUtensorMap& a2, const CUtensorMap& b0_2,
                         const CUtensorMap& b1_2, const CUtensorMap& c2, const GemmArgs& args,
-                        int rows_upper, cudaStream_t stream) {
+                        int rows_upper, cudaStream_t stream, int threads = NUM_THREADS) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
   auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE, GATHER>;
@@ -839,7 +955,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
   if (tiles_upper <= 0) return cudaSuccess;
   const int max_pairs = num_sms() / 2;
   const int pairs = static_cast<int>(tiles_upper < max_pairs ? tiles_upper : max_pairs);
-  return launch_pdl(kern, dim3(2 * pairs), dim3(NUM_THREADS), Cfg::SMEM_BYTES, stream, a, b0, b1,
+  return launch_pdl(kern, dim3(2 * pairs), dim3(threads), Cfg::SMEM_BYTES, stream, a, b0, b1,
                     c, a2, b0_2, b1_2, c2, a2r);
 }
 
@@ -850,7 +966,8 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
-                                       cudaStream_t stream, const GemmExtraGroup* extra) {
+                                       cudaStream_t stream, const GemmExtraGroup* extra,
+                                       const GemmCopy* copy) {
   CUtensorMap ta, tb0, tb1, tc, xa, xb0, xb1, xc;
   const int64_t b_rows = static_cast<int64_t>(offsets ? num_groups : 1) * F;
   const int64_t c_rows = offsets ? a_rows : rows_single;
@@ -878,9 +995,20 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
   } else {
     xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
   }
+  if (copy != nullptr) {
+    if (offsets == nullptr || !copy->src || !copy->perm || !copy->ready || copy->src_rows < 1 ||
+        (reinterpret_cast<uintptr_t>(copy->src) & 15) || (reinterpret_cast<uintptr_t>(A) & 15))
+      return cudaErrorInvalidValue;
+    args.cp_src = copy->src;
+    args.cp_perm = copy->perm;
+    args.cp_ready = copy->ready;
+    args.cp_dst = const_cast<void*>(A);
+    args.cp_src_rows = copy->src_rows;
+  }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
   return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
-                                            rows_upper, stream);
+                                            rows_upper, stream,
+                                            copy != nullptr ? NUM_THREADS_COPY : NUM_THREADS);
 }
 
 // The SwiGLU backward fused into the recomputed gate/up pass: with g and u

@@ -87,10 +87,12 @@ cudaError_t dispatch_rank_scan(const int32_t* topk_idx, int T, int k, int E, int
 cudaError_t dispatch_scan(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                           int32_t* offsets, cudaStream_t stream);
 // slot_pos (in: rank inside its block of blk_tokens tokens, out: row) and
-// perm_src only, no row copy.
+// perm_src only, no row copy.  zero (or null): n_zero int32 set to zero,
+// the counters of a gate/up launch that copies its own rows.
 cudaError_t dispatch_positions(const int32_t* topk_idx, const int32_t* blk_bases,
                                int32_t* slot_pos, int32_t* perm_src, int T, int k, int E,
-                               int blk_tokens, cudaStream_t stream);
+                               int blk_tokens, cudaStream_t stream, int32_t* zero = nullptr,
+                               int n_zero = 0);
 cudaError_t dispatch_scatter(bool bf16, const void* x, const int32_t* topk_idx,
                              const int32_t* blk_bases, int32_t* slot_pos, int32_t* perm_src,
                              void* x_perm, int T, int d, int k, int E, int blk_tokens,
@@ -109,11 +111,22 @@ struct GemmExtraGroup {
   int K;
   void* C;
 };
+// The routed gate/up launch copies its own A rows (A = x_perm, row r = x
+// row perm[r]) while it runs, instead of reading a copy made before it:
+// ready [1 + ceil(a_rows / 32)] int32, zero at launch (a unit counter and
+// per-32-row block counts).
+struct GemmCopy {
+  const void* src;       // x [src_rows, K] bf16
+  int src_rows;
+  const int32_t* perm;   // perm_src [a_rows]
+  int32_t* ready;
+};
 cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int32_t* offsets,
                                        int num_groups, int rows_single, const void* W1,
                                        const void* W3, int F, int K, void* H, uint32_t* status,
                                        cudaStream_t stream,
-                                       const GemmExtraGroup* extra = nullptr);
+                                       const GemmExtraGroup* extra = nullptr,
+                                       const GemmCopy* copy = nullptr);
 cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, const int32_t* rows,
                                               int64_t R, const int32_t* offsets, int num_groups,
                                               const void* W1, const void* W3, int F, int K,

@@ -16,7 +16,7 @@ inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 // Workspace layout shared by every call.  Byte offsets from the base.
 struct Layout {
   size_t status, blk, offsets, slot_pos, perm_src, refine, refine_cand, stats, logits, x_perm, h,
-      y_perm, h_sh, y_sh, fold, total;
+      y_perm, h_sh, y_sh, fold, copy_ready, total;
 };
 
 inline size_t esize(const moe_config& c) { return c.dtype == MOE_BF16 ? 2 : 4; }
@@ -45,6 +45,8 @@ Layout layout(const moe_config& c) {
   // the folded combine's counts: [T, column tiles of the down GEMM], at
   // most d / 128 tiles (bf16 only)
   L.fold = o;     o += up(c.dtype == MOE_BF16 ? T * ((d + 127) / 128) * 4 : 0);
+  // the counters of a gate/up launch that copies its own rows (bf16 only)
+  L.copy_ready = o; o += up(c.dtype == MOE_BF16 ? (1 + (R + 31) / 32) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -146,9 +148,12 @@ moe_status run_router(const moe_config* c, const void* x, const void* w_router,
 }
 
 // fold_nt > 0: also set the folded combine's counts ([T, fold_nt] in ws).
+// copy_counters (x_perm == nullptr only): also zero the counters of a gate/up
+// launch that copies its own rows.
 moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void* x,
                        int32_t* counts, int32_t* offsets, int32_t* slot_pos, int32_t* perm_src,
-                       void* x_perm, void* ws, cudaStream_t s, int fold_nt = 0) {
+                       void* x_perm, void* ws, cudaStream_t s, int fold_nt = 0,
+                       bool copy_counters = false) {
   const Layout L = layout(*c);
   int32_t* blk = at<int32_t>(ws, L.blk);
   uint32_t* status = at<uint32_t>(ws, L.status);
@@ -156,8 +161,13 @@ moe_status run_permute(const moe_config* c, const int32_t* topk_idx, const void*
                                   offsets, status, status + 3, s,
                                   fold_nt > 0 ? at<int32_t>(ws, L.fold) : nullptr, fold_nt));
   if (x_perm == nullptr) {   // rows only; the experts gather x through perm_src
+    const int n_zero =
+        copy_counters ? 1 + static_cast<int>((static_cast<int64_t>(c->T) * c->top_k + 31) / 32)
+                      : 0;
     MOE_TRY(moe::dispatch_positions(topk_idx, blk, slot_pos, perm_src, c->T, c->top_k,
-                                    c->n_experts, moe::kRankBlock, s));
+                                    c->n_experts, moe::kRankBlock, s,
+                                    copy_counters ? at<int32_t>(ws, L.copy_ready) : nullptr,
+                                    n_zero));
     return MOE_OK;
   }
   MOE_TRY(moe::dispatch_scatter(c->dtype == MOE_BF16, x, topk_idx, blk, slot_pos, perm_src,
@@ -178,11 +188,13 @@ struct Marks {
 // x_perm == nullptr (bf16 only): the gate/up GEMM gathers its rows from x
 // through gather_rows (perm_src) instead of reading a permuted copy.
 // fold (bf16 only): the down GEMM also forms the combined output.
+// copy (bf16 only, with x_perm): the gate/up GEMM fills x_perm itself.
 moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* offsets,
                        const moe_expert_weights* w, const void* x, void* y_perm, void* y_shared,
                        void* ws, cudaStream_t s, const Marks& mk,
                        const int32_t* gather_rows = nullptr,
-                       const moe::GemmFold* fold = nullptr) {
+                       const moe::GemmFold* fold = nullptr,
+                       const moe::GemmCopy* copy = nullptr) {
   const Layout L = layout(*c);
   uint32_t* status = at<uint32_t>(ws, L.status);
   const int64_t R = static_cast<int64_t>(c->T) * c->top_k;
@@ -200,7 +212,8 @@ moe_status run_experts(const moe_config* c, const void* x_perm, const int32_t* o
                                                      c->n_shared ? &sh_up : nullptr));
     } else {
       MOE_TRY(moe::grouped_swiglu_gateup_bf16(x_perm, R, offsets, E, 0, w->w1, w->w3, F, d, h,
-                                              status, s, c->n_shared ? &sh_up : nullptr));
+                                              status, s, c->n_shared ? &sh_up : nullptr,
+                                              copy));
     }
     if (!mk.rec(3)) return MOE_ERR_CUDA;
     MOE_TRY(moe::grouped_down_bf16(h, R, offsets, E, 0, w->w2, d, F, y_perm, status, s,
@@ -249,12 +262,14 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
   if (st != MOE_OK) return st;
   if (opts != nullptr &&
       ((opts->gather_rows != 0 && opts->gather_rows != 1) ||
-       (opts->fold_combine != 0 && opts->fold_combine != 1) || opts->reserved[0] != 0 ||
-       opts->reserved[1] != 0))
+       (opts->fold_combine != 0 && opts->fold_combine != 1) ||
+       (opts->scatter_in_gemm != 0 && opts->scatter_in_gemm != 1) || opts->reserved[0] != 0 ||
+       (opts->gather_rows == 1 && opts->scatter_in_gemm == 1)))
     return MOE_ERR_INVALID;
   const bool gather = opts != nullptr && opts->gather_rows == 1;
   const bool fold = opts != nullptr && opts->fold_combine == 1;
-  if ((gather || fold) && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  const bool scat = opts != nullptr && opts->scatter_in_gemm == 1;
+  if ((gather || fold || scat) && cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (!counts) return MOE_ERR_INVALID;
   if (cfg->T == 0) {
     MOE_TRY(cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, S(stream)));
@@ -297,14 +312,17 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* w_rout
       fold ? (cfg->d_model + moe::down_tile_cols(cfg->d_model, cfg->d_ff) - 1) /
                  moe::down_tile_cols(cfg->d_model, cfg->d_ff)
            : 0;
+  // scatter_in_gemm: dispatch writes the rows' positions only, and the
+  // gate/up GEMM copies x's rows into x_perm while it runs
   if ((st = run_permute(cfg, topk_idx, x, counts, offsets, slot_pos, perm_src,
-                        gather ? nullptr : x_perm, ws, s, fold_nt)) != MOE_OK)
+                        (gather || scat) ? nullptr : x_perm, ws, s, fold_nt, scat)) != MOE_OK)
     return st;
   if (!mk.rec(2)) return MOE_ERR_CUDA;
   const moe::GemmFold gf{at<int32_t>(ws, L.fold), fold_nt, cfg->T, cfg->top_k, perm_src,
                          slot_pos, topk_w, out};
+  const moe::GemmCopy gc{x, cfg->T, perm_src, at<int32_t>(ws, L.copy_ready)};
   if ((st = run_experts(cfg, gather ? nullptr : x_perm, offsets, w, x, y_perm, y_sh, ws, s, mk,
-                        perm_src, fold ? &gf : nullptr)) != MOE_OK)
+                        perm_src, fold ? &gf : nullptr, scat ? &gc : nullptr)) != MOE_OK)
     return st;
   if (!fold)
     MOE_TRY(moe::combine(cfg->dtype == MOE_BF16, y_perm, slot_pos, topk_w, y_sh, out, cfg->T,

@@ -55,16 +55,17 @@ class MoELayer:
 
     # ----------------------------------------------------------------- calls
     def forward(self, x: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                stream=None, gather_rows: bool = False,
-                fold_combine: bool = False) -> torch.Tensor:
-        """The layer forward (moe_forward; moe_forward_ex with gather_rows or
-        fold_combine)."""
+                stream=None, gather_rows: bool = False, fold_combine: bool = False,
+                scatter_in_gemm: bool = False) -> torch.Tensor:
+        """The layer forward (moe_forward; moe_forward_ex with gather_rows,
+        fold_combine or scatter_in_gemm)."""
         args = (self.cfg, self.x if x is None else x, self.w_router, self.sel_bias,
                 self.logit_offset, self.weights, self.out if out is None else out,
                 self.topk_idx, self.topk_w, self.counts, self.ws)
-        if gather_rows or fold_combine:
+        if gather_rows or fold_combine or scatter_in_gemm:
             B.moe_forward_ex(*args, gather_rows=int(gather_rows),
-                             fold_combine=int(fold_combine), stream=stream)
+                             fold_combine=int(fold_combine),
+                             scatter_in_gemm=int(scatter_in_gemm), stream=stream)
         else:
             B.moe_forward(*args, stream=stream)
         return self.out if out is None else out

@@ -173,8 +173,17 @@ def test_forward_options_layout_and_validation(lib):
     st = B.moe_forward_ex(tiny, ok, ok, None, None, w, ok, ok, ok, ok, ws32, fold_combine=1,
                           stream=0, check=False)
     assert st == B.MOE_ERR_UNSUPPORTED
-    opts = B.MoEForwardOpts(0, 0)
-    opts.reserved[1] = 1
+    st = B.moe_forward_ex(cfg, ok, ok, None, None, w, ok, ok, ok, ok, ws, scatter_in_gemm=2,
+                          stream=0, check=False)
+    assert st == B.MOE_ERR_INVALID
+    st = B.moe_forward_ex(cfg, ok, ok, None, None, w, ok, ok, ok, ok, ws, gather_rows=1,
+                          scatter_in_gemm=1, stream=0, check=False)
+    assert st == B.MOE_ERR_INVALID
+    st = B.moe_forward_ex(tiny, ok, ok, None, None, w, ok, ok, ok, ok, ws32, scatter_in_gemm=1,
+                          stream=0, check=False)
+    assert st == B.MOE_ERR_UNSUPPORTED
+    opts = B.MoEForwardOpts(0, 0, 0)
+    opts.reserved[0] = 1
     st = B.lib().moe_forward_ex(ctypes.byref(cfg), None, None, None, None,
                                 ctypes.byref(B.expert_weights(w)), None, None, None, None,
                                 ctypes.byref(opts), None, 0, None)

@@ -153,6 +153,28 @@ def test_forward_with_folded_combine(name, gather):
     _check_layer(shape, host, layer)
 
 
+@pytest.mark.parametrize("name,fold", [("page2_small", False), ("qwen3_small", False),
+                                       ("skew_small", True), ("wide_small", False),
+                                       ("qwen3_30b", False), ("skew", False), ("page2", True)])
+def test_forward_with_scatter_in_gemm(name, fold):
+    """The alternative (moe_forward_ex, scatter_in_gemm = 1) whose gate/up
+    GEMM copies x's rows into x_perm while it runs: against the oracle and
+    bit for bit against the default path, with the device status clear (no
+    wait gave up).  The backward tests read that x_perm too."""
+    shape = SMALL[name] if name in SMALL else I.WORKLOADS[name]
+    host = I.make_inputs(shape)
+    layer = MoELayer(shape, host)
+    layer.forward()
+    torch.cuda.synchronize()
+    ref = layer.out.clone()
+    layer.out.fill_(float("nan"))
+    layer.forward(scatter_in_gemm=True, fold_combine=fold)
+    torch.cuda.synchronize()
+    assert layer.device_status()[0] == B.MOE_OK
+    assert torch.equal(layer.out.view(torch.int16), ref.view(torch.int16))
+    _check_layer(shape, host, layer)
+
+
 def test_skew_bias_update_then_deferred_forward():
     """Skewed workload: forward, bias update from its counts (bit-exact), then a
     second forward routes with the new bias (the update lands on the next
