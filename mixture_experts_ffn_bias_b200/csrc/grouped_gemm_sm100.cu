@@ -51,6 +51,17 @@ constexpr int NUM_THREADS_COPY = NUM_THREADS + 32 * COPY_WARPS;
 constexpr int MAX_GROUPS = 257;
 
 
+// Variants of a mode, each its own instantiation, so the default path
+// compiles without the alternatives' code:
+//   VAR_NONE    A by TMA tiles, output by TMA stores
+//   VAR_GATHER  (gate/up) A rows gathered from x by tile::gather4 loads
+//   VAR_COPY    (gate/up) A rows copied into place by the launch itself
+//   VAR_FOLD    (plain) the combine folded into the epilogue
+constexpr int VAR_NONE = 0;
+constexpr int VAR_GATHER = 1;
+constexpr int VAR_COPY = 2;
+constexpr int VAR_FOLD = 3;
+
 // Epilogue / operand modes.
 constexpr int MODE_PLAIN_BF16 = 0;    // C = A B^T, rounded to bf16
 constexpr int MODE_SWIGLU_BF16 = 1;   // C = silu(A B0^T) * (A B1^T), rounded to bf16
@@ -248,22 +259,21 @@ __device__ __forceinline__ int extra_tiles(const GemmArgs& a) {
 }
 
 // Whether `tile` is one of the extra group's.  They follow the routed
-// groups' tiles, except under the folded combine, where they come first:
-// every token's output waits for its shared-expert row, so those rows are
-// done early.
-__device__ __forceinline__ bool is_extra_tile(const GemmArgs& a, int routed_tiles, int x_tiles,
-                                              int tile) {
-  return a.fold_cnt != nullptr ? tile < x_tiles : tile >= routed_tiles;
+// groups' tiles, except under the folded combine (XFIRST), where they come
+// first: every token's output waits for its shared-expert row, so those
+// rows are done early.
+template <bool XFIRST>
+__device__ __forceinline__ bool is_extra_tile(int routed_tiles, int x_tiles, int tile) {
+  return XFIRST ? tile < x_tiles : tile >= routed_tiles;
 }
 
-template <int BN_OUT>
+template <int BN_OUT, bool XFIRST>
 __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_off,
                                               const int* s_prefix, int G, int n_tiles, int tile) {
   PairTile t;
   const int xt = extra_tiles<BN_OUT>(a);
-  const bool first = a.fold_cnt != nullptr;
-  if (is_extra_tile(a, s_prefix[G], xt, tile)) {
-    const int local = first ? tile : tile - s_prefix[G];
+  if (is_extra_tile<XFIRST>(s_prefix[G], xt, tile)) {
+    const int local = XFIRST ? tile : tile - s_prefix[G];
     const int xn = (a.x_n + BN_OUT - 1) / BN_OUT;
     t.x = true;
     t.g = 0;
@@ -273,7 +283,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& a, const int* s_of
     t.rows = a.x_rows;
     t.kblocks = a.x_K / BK;
   } else {
-    if (first) tile -= xt;
+    if (XFIRST) tile -= xt;
     t.x = false;
     t.g = find_group(s_prefix, G, tile);
     t.row0 = s_off[t.g];
@@ -467,14 +477,9 @@ __device__ __forceinline__ bool wait_a_rows(const GemmArgs& a, int lo, int hi, i
 constexpr bool kStoreEvictFirst = true;
 constexpr bool kLoadAEvictLast = false;
 
-// Threads a launch of the pair kernel may have: only the forward gate/up
-// kernel carries the copy warps.
-constexpr int pair_max_threads(int mode, bool gather) {
-  return mode == MODE_SWIGLU_BF16 && !gather ? NUM_THREADS_COPY : NUM_THREADS;
-}
-
-template <int BN_ACC, int MODE, bool GATHER>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair_max_threads(MODE, GATHER), 1)
+template <int BN_ACC, int MODE, int VAR>
+__global__ void __cluster_dims__(2, 1, 1)
+__launch_bounds__(VAR == VAR_COPY ? NUM_THREADS_COPY : NUM_THREADS, 1)
 grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmB0,
                          const __grid_constant__ CUtensorMap tmB1,
@@ -485,6 +490,11 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                          const __grid_constant__ CUtensorMap tmC2, const GemmArgs args) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr bool GATHER = VAR == VAR_GATHER;
+  constexpr bool COPY = VAR == VAR_COPY;
+  constexpr bool FOLD = VAR == VAR_FOLD;
+  static_assert(!(GATHER || COPY) || MODE == MODE_SWIGLU_BF16, "gate/up variants");
+  static_assert(!FOLD || MODE == MODE_PLAIN_BF16, "plain-mode variant");
   constexpr bool SWI_BWD = MODE == MODE_SWIGLU_BWD;
   constexpr bool SWIGLU = MODE == MODE_SWIGLU_BF16 || SWI_BWD;
   constexpr bool BMN = MODE == MODE_PLAIN_BMN || MODE == MODE_PLAIN_BMN_F32;
@@ -577,7 +587,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint64_t a_policy = kLoadAEvictLast ? l2_policy_evict_last() : 0ull;
     // without gathers lane 0 alone drives the ring
     for (int tile = pair; tile < total_tiles && ok && (GATHER || lane == 0); tile += npairs) {
-      const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
+      const PairTile pt = pair_tile<BN_OUT, FOLD>(args, s_off, s_prefix, G, n_tiles, tile);
       const int g = pt.g, n = pt.n, kblocks = pt.kblocks;
       const int arow = pt.row0 + pt.m * BM2 + static_cast<int>(rank) * BM;
       const int gbase = pt.x ? 0 : g * args.n_per_group;
@@ -587,9 +597,9 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const CUtensorMap* mb = (SWIGLU && rank == 1) ? (pt.x ? &tmB1_2 : &tmB1)
                                                     : (pt.x ? &tmB0_2 : &tmB0);
       const bool gathered = GATHER && !pt.x;
-      if constexpr (MODE == MODE_SWIGLU_BF16 && !GATHER) {
+      if constexpr (COPY) {
         // lane 0 alone runs this loop here
-        if (args.cp_ready != nullptr && !pt.x &&
+        if (!pt.x &&
             !wait_a_rows(args, arow, min(arow + BM, pt.row0 + pt.rows), s_off[G], abort_flag)) {
           ok = false;
           break;
@@ -667,7 +677,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
         const int acc = it % NACC;
         const uint32_t acc_phase = (it / NACC) & 1;
         const int kblocks =
-            is_extra_tile(args, s_prefix[G], x_tiles, tile) ? args.x_K / BK : args.K / BK;
+            is_extra_tile<FOLD>(s_prefix[G], x_tiles, tile) ? args.x_K / BK : args.K / BK;
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN_ACC;
@@ -700,7 +710,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
           if (globaltimer_ns() - t0 > kWaitLimitNs) break;
       }
     }
-  } else if (warp < NUM_THREADS / 32) {
+  } else if (!COPY || warp < NUM_THREADS / 32) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const uint64_t c_policy = kStoreEvictFirst ? l2_policy_evict_first() : 0ull;
@@ -711,7 +721,7 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      const PairTile pt = pair_tile<BN_OUT>(args, s_off, s_prefix, G, n_tiles, tile);
+      const PairTile pt = pair_tile<BN_OUT, FOLD>(args, s_off, s_prefix, G, n_tiles, tile);
       const int rows_g = pt.rows, n = pt.n;
       const int r0 = pt.m * BM2 + static_cast<int>(rank) * BM;   // first row (in group) of this CTA
       const bool valid = (r0 + q * 32 + lane) < rows_g;
@@ -857,18 +867,13 @@ grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_rank0(&tempty_bar[acc]);
-      if constexpr (MODE == MODE_PLAIN_BF16) {
-        if (args.fold_cnt != nullptr)
-          fold_combine_rows<BN_OUT>(args, pt.x, n, ncols, valid, warp_row0, lane);
-      }
+      if constexpr (FOLD) fold_combine_rows<BN_OUT>(args, pt.x, n, ncols, valid, warp_row0, lane);
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
   } else {
     // ------------------------------------------------- A-row copy (gate/up)
-    if constexpr (MODE == MODE_SWIGLU_BF16 && !GATHER) {
-      if (args.cp_ready != nullptr) copy_a_rows(args, s_off[G], lane);
-    }
+    if constexpr (COPY) copy_a_rows(args, s_off[G], lane);
   }
 
   tc_fence_before();
@@ -923,14 +928,14 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int BN_ACC, int MODE, bool GATHER = false>
+template <int BN_ACC, int MODE, int VAR = VAR_NONE>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& c, const CUtensorMap& a2, const CUtensorMap& b0_2,
                         const CUtensorMap& b1_2, const CUtensorMap& c2, const GemmArgs& args,
                         int rows_upper, cudaStream_t stream, int threads = NUM_THREADS) {
   using Cfg = PairCfg<BN_ACC>;
   constexpr int BN_OUT = MODE == MODE_SWIGLU_BF16 ? BN_ACC / 2 : BN_ACC;
-  auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE, GATHER>;
+  auto kern = grouped_gemm_pair_kernel<BN_ACC, MODE, VAR>;
   static unsigned long long attr_done = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1006,9 +1011,11 @@ cudaError_t grouped_swiglu_gateup_bf16(const void* A, int64_t a_rows, const int3
     args.cp_src_rows = copy->src_rows;
   }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (copy != nullptr)
+    return launch_pair<256, MODE_SWIGLU_BF16, VAR_COPY>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
+                                                        rows_upper, stream, NUM_THREADS_COPY);
   return launch_pair<256, MODE_SWIGLU_BF16>(ta, tb0, tb1, tc, xa, xb0, xb1, xc, args,
-                                            rows_upper, stream,
-                                            copy != nullptr ? NUM_THREADS_COPY : NUM_THREADS);
+                                            rows_upper, stream);
 }
 
 // The SwiGLU backward fused into the recomputed gate/up pass: with g and u
@@ -1061,7 +1068,7 @@ cudaError_t grouped_swiglu_gateup_gather_bf16(const void* X, int64_t x_rows, con
   } else {
     xa = ta; xb0 = tb0; xb1 = tb1; xc = tc;
   }
-  return launch_pair<256, MODE_SWIGLU_BF16, true>(ta, tb0, tb1, tc, xa, xb0, xb1, xc,
+  return launch_pair<256, MODE_SWIGLU_BF16, VAR_GATHER>(ta, tb0, tb1, tc, xa, xb0, xb1, xc,
                                                   args, static_cast<int>(R), stream);
 }
 
@@ -1122,6 +1129,16 @@ cudaError_t grouped_down_bf16(const void* A, int64_t a_rows, const int32_t* offs
     args.fold_out = fold->out;
   }
   const int rows_upper = offsets ? static_cast<int>(a_rows) : rows_single;
+  if (fold != nullptr) {
+    if (bn == 512)
+      return launch_pair<512, MODE_PLAIN_BF16, VAR_FOLD>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                                         rows_upper, stream);
+    if (bn == 256)
+      return launch_pair<256, MODE_PLAIN_BF16, VAR_FOLD>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                                         rows_upper, stream);
+    return launch_pair<128, MODE_PLAIN_BF16, VAR_FOLD>(ta, tb, tb, tc, xa, xb, xb, xc, args,
+                                                       rows_upper, stream);
+  }
   if (bn == 512)
     return launch_pair<512, MODE_PLAIN_BF16>(ta, tb, tb, tc, xa, xb, xb, xc, args,
                                              rows_upper, stream);
