@@ -56,21 +56,25 @@ def layer_flops(s: I.MoEShape) -> dict:
 # DRAM bytes per launch of the routed gate/up GEMM, from the ncu capture in
 # profiles/grouped_gemm_gateup_qwen3_30b.md, and the kernel source it was
 # taken on (sha256 of csrc/grouped_gemm_sm100.cu, first 16 hex digits).
-GATEUP_TRAFFIC = {"qwen3_30b": (1844455168, "4723d615b7c2e7f9")}
+GATEUP_TRAFFIC = {"qwen3_30b": (1761350912, "fec88564d8c301e2")}
 
 
-def traffic_note(s: I.MoEShape) -> str:
+def gateup_traffic(s: I.MoEShape):
+    """(DRAM bytes per gate/up launch or None, note): the bytes of the ncu
+    capture when it was taken on the kernel source in the tree, else None."""
     import hashlib
     src = os.path.join(ROOT, "mixture_experts_ffn_bias_b200", "csrc", "grouped_gemm_sm100.cu")
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()[:16]
     if s.name not in GATEUP_TRAFFIC:
-        return "not measured in this run; no ncu capture of this workload's gate/up launch"
+        return None, "not measured: no ncu capture of this workload's gate/up launch"
     nbytes, at = GATEUP_TRAFFIC[s.name]
-    same = "the same source" if sha == at else f"an older source (now {sha})"
-    return (f"not measured in this run; {nbytes} DRAM bytes per launch in the ncu capture of "
-            f"profiles/grouped_gemm_gateup_qwen3_30b.md, taken on kernel source {at} "
-            f"({same})")
+    where = ("ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one launch) in "
+             "profiles/grouped_gemm_gateup_qwen3_30b.md")
+    if sha != at:
+        return None, (f"{nbytes} DRAM bytes per launch in the {where}, taken on kernel source "
+                      f"{at}; the source is now {sha}, so not reported")
+    return nbytes, f"from the {where}, on this kernel source ({sha}); not measured in this run"
 
 
 def near_tie_exclusions(s: I.MoEShape) -> dict:
@@ -486,7 +490,12 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         t_gateup = phases[2] * 1e-3
         t_gemm = (phases[2] + phases[3] + phases[4]) * 1e-3
-        achieved = fl["gate_up"] / t_gateup / 1e12
+        # the gate/up launch also runs the shared expert's gate/up as one more
+        # group (bf16 layers), so its work counts toward that launch
+        launch_flops = fl["gate_up"] + (4 * shape.T * shape.d_model * shape.d_ff_shared *
+                                        shape.n_shared if shape.dtype == I.DTYPE_BF16 else 0)
+        achieved = launch_flops / t_gateup / 1e12
+        traffic = gateup_traffic(shape)
         gemm_tflops = (fl["gate_up"] + fl["down"] + fl["shared"]) / t_gemm / 1e12
         pb = path_bytes(shape)
         t_path = (phases[0] + phases[1] + phases[5]) * 1e-3
@@ -518,14 +527,17 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
                                         "peaks": peak_kind},
             "phases_ms": dict(zip(["router", "dispatch", "gate_up", "down", "shared", "combine"],
                                   phases)),
-            "roofline": {"kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)", "bound": "tensor",
+            "roofline": {"kernel": "grouped gate/up GEMM + SwiGLU (tcgen05)" +
+                         (", shared expert as one more group"
+                          if shape.n_shared and shape.dtype == I.DTYPE_BF16 else ""),
+                         "bound": "tensor", "flops_per_launch": launch_flops,
                          "achieved": achieved, "peak": burst, "unit": "TFLOP/s",
                          "frac": achieved / burst,
                          "peak_kind": f"bf16_tflops, burst ({peak_kind})",
                          "frac_of_sustained": achieved / sus,
                          "frac_of_nominal": achieved / NOMINAL_BF16_TFLOPS,
-                         "traffic": None,
-                         "traffic_note": traffic_note(shape)},
+                         "traffic": traffic[0],
+                         "traffic_note": traffic[1]},
             "e2e": {"value": shape.T * world / (e2e_ms * 1e-3), "unit": UNIT,
                     "h2d_bytes_per_step": layer.x.numel() * layer.x.element_size(),
                     "d2h_bytes_per_step": layer.out.numel() * layer.out.element_size(),
