@@ -280,7 +280,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* w_route
  *     warps hold the down GEMM's epilogue).  Combinable with gather_rows.
  *   scatter_in_gemm 1 (bf16 layers only; not with gather_rows): dispatch
  *     writes only the rows' positions, and the gate/up GEMM launch fills
- *     x_perm itself while it runs: four extra warps per CTA copy x's rows in
+ *     x_perm itself while it runs: two extra warps per CTA copy x's rows in
  *     row order and count them per 32-row block, and each tile's loads wait
  *     (bounded) for the blocks of its rows.  Same results; x_perm is kept
  *     for moe_backward as with the default.
