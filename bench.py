@@ -53,6 +53,16 @@ def layer_flops(s: I.MoEShape) -> dict:
     }
 
 
+def gateup_launch_flops(s: I.MoEShape) -> int:
+    """Algorithmic FLOPs of one gate/up GEMM launch: the routed experts'
+    4 R d F, plus the shared expert's 4 T d Fs on bf16 layers, whose gate/up
+    runs as one more group of the same launch."""
+    fl = layer_flops(s)["gate_up"]
+    if s.dtype == I.DTYPE_BF16:
+        fl += 4 * s.T * s.d_model * s.d_ff_shared * s.n_shared
+    return fl
+
+
 # DRAM bytes per launch of the routed gate/up GEMM, from the ncu capture in
 # profiles/grouped_gemm_gateup_qwen3_30b.md, and the kernel source it was
 # taken on (sha256 of csrc/grouped_gemm_sm100.cu, first 16 hex digits).
@@ -490,10 +500,7 @@ def run_ours(args, shape, rank: int, world: int, local_rank: int):
         hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
         t_gateup = phases[2] * 1e-3
         t_gemm = (phases[2] + phases[3] + phases[4]) * 1e-3
-        # the gate/up launch also runs the shared expert's gate/up as one more
-        # group (bf16 layers), so its work counts toward that launch
-        launch_flops = fl["gate_up"] + (4 * shape.T * shape.d_model * shape.d_ff_shared *
-                                        shape.n_shared if shape.dtype == I.DTYPE_BF16 else 0)
+        launch_flops = gateup_launch_flops(shape)
         achieved = launch_flops / t_gateup / 1e12
         traffic = gateup_traffic(shape)
         gemm_tflops = (fl["gate_up"] + fl["down"] + fl["shared"]) / t_gemm / 1e12
