@@ -254,6 +254,43 @@ def test_every_token_on_one_expert():
     _check_layer(shape, host, layer)
 
 
+def _edge_shape(name):
+    if name == "single_token":
+        return SMALL["qwen3_small"].replace(T=1), None
+    if name == "one_expert_top1":
+        return I.MoEShape("one", 300, 256, 1, 256, 1, 0, 0, I.GATE_SOFTMAX, 1, I.DTYPE_BF16,
+                          "none", 0.0, 7), None
+    if name == "top_k_all":
+        return I.MoEShape("all", 257, 128, 8, 128, 8, 0, 0, I.GATE_SOFTMAX, 1, I.DTYPE_BF16,
+                          "none", 0.0, 8), None
+    bias = np.zeros(64, np.float32)   # every token on expert 37, with a shared expert
+    bias[37] = 50.0
+    return SMALL["skew_small"].replace(T=700), bias
+
+
+@pytest.mark.parametrize("name", ["single_token", "one_expert_top1", "top_k_all", "one_hot"])
+@pytest.mark.parametrize("opt", ["fold_combine", "scatter_in_gemm", "gather_rows"])
+def test_forward_options_on_edge_shapes(name, opt):
+    """Each per-call alternative on the degenerate shapes (one token; one
+    expert, top-1; top-k = E; every token on one expert next to 63 empty
+    ones and a shared expert): bit for bit against the default path and
+    element-wise against the oracle."""
+    shape, bias = _edge_shape(name)
+    host = I.make_inputs(shape)
+    if bias is not None:
+        host["sel_bias"] = bias
+    layer = MoELayer(shape, host)
+    layer.forward()
+    torch.cuda.synchronize()
+    ref = layer.out.clone()
+    layer.out.fill_(float("nan"))
+    layer.forward(**{opt: True})
+    torch.cuda.synchronize()
+    assert layer.device_status()[0] == B.MOE_OK
+    assert torch.equal(layer.out.view(torch.int16), ref.view(torch.int16))
+    _check_layer(shape, host, layer)
+
+
 @pytest.mark.parametrize("E,k,gate", [(256, 4, I.GATE_SOFTMAX), (32, 12, I.GATE_SIGMOID),
                                       (200, 3, I.GATE_SIGMOID)])
 def test_router_paths_without_fused_select(E, k, gate):
