@@ -71,12 +71,12 @@ def test_backward_small_elementwise(name, mode):
         assert err <= GRAD_TOL, f"{gk}: relative error {err:.3e}"
 
 
-@pytest.mark.parametrize("name", ["page2", "qwen3_30b"])
+@pytest.mark.parametrize("name", ["page2", "qwen3_30b", "skew", "wide"])
 def test_backward_full_size_every_element(name):
     """Full-size workloads (qwen3_30b is the one the benchmark's backward
     mode times, in the same configuration): every element of dx, the router
     weight gradient and every expert weight gradient (the shared expert's
-    too, on page2) against the oracle.  The stored near-tie lists of these
+    too, on page2 and skew) against the oracle.  The stored near-tie lists of these
     workloads are empty, so the GPU's routing is the oracle's on every token
     (checked)."""
     shape = I.WORKLOADS[name]
