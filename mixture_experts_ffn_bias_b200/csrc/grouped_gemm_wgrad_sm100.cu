@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "kernels.h"
@@ -312,16 +313,18 @@ using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, voi
                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once per process; the initialisation of a function-local
+// static is thread-safe.
 EncodeFn encode() {
-  static EncodeFn fn = nullptr;
-  if (fn == nullptr) {
+  static const EncodeFn fn = []() -> EncodeFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(p);
-  }
+      return reinterpret_cast<EncodeFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -344,15 +347,15 @@ cudaError_t launch_wgrad(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
                          const WgradArgs& a, cudaStream_t stream) {
   using Cfg = WCfg<BN>;
   auto kern = wgrad_kernel<BN>;
-  static unsigned long long attr_done = 0;
+  static std::atomic<unsigned long long> attr_done{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned long long bit = 1ull << (dev & 63);
-  if (!(attr_done & bit)) {
+  if (!(attr_done.load(std::memory_order_acquire) & bit)) {
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_done |= bit;
+    attr_done.fetch_or(bit, std::memory_order_acq_rel);
   }
   int sms = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
