@@ -66,7 +66,7 @@ def gateup_launch_flops(s: I.MoEShape) -> int:
 # DRAM bytes per launch of the routed gate/up GEMM, from the ncu capture in
 # profiles/grouped_gemm_gateup_qwen3_30b.md, and the kernel source it was
 # taken on (sha256 of csrc/grouped_gemm_sm100.cu, first 16 hex digits).
-GATEUP_TRAFFIC = {"qwen3_30b": (1761350912, "fec88564d8c301e2")}
+GATEUP_TRAFFIC = {"qwen3_30b": (2154375424, "0a08a2e8d9e85551")}
 
 
 def gateup_traffic(s: I.MoEShape):
